@@ -1,0 +1,278 @@
+"""Pins for the fp64 oracle: closed forms, invariants, brute force, a library
+routine and the pages' worked example.  None of these re-types an oracle
+formula; each would fail on a plausible slip (a dropped term, a wrong sign,
+index or window, a transposed operand, a wrong head-to-group map)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import infllm2_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------- bf16 rounding
+def test_bf16_round_matches_library_on_fp32_values():
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(200000) * np.exp(rng.uniform(-20, 20, 200000))).astype(np.float32)
+    # exact halfway cases: a bf16 value plus half of its last place
+    base = _bf16(rng.standard_normal(5000).astype(np.float32))
+    m, e = np.frexp(base)
+    ties = (base + np.ldexp(np.sign(base), e - 9)).astype(np.float32)
+    for arr in (x, ties):
+        ref = torch.from_numpy(arr).to(torch.bfloat16).to(torch.float64).numpy()
+        np.testing.assert_array_equal(O.bf16_round(arr.astype(np.float64)), ref)
+
+
+def test_bf16_round_hand_cases():
+    cases = {
+        1.0 + 2.0 ** -8: 1.0,                       # tie -> even (1.0)
+        1.0 + 3 * 2.0 ** -8: 1.0 + 2.0 ** -6,       # tie -> even (odd last bit rounds up)
+        1.0 + 2.0 ** -8 + 2.0 ** -30: 1.0 + 2.0 ** -7,   # just above a tie rounds up
+        -(1.0 + 2.0 ** -8): -1.0,
+        3.4e38: math.inf,                           # beyond the largest bf16 + half a place
+        2.0 ** -140: 0.0,
+        0.0: 0.0,
+    }
+    for x, want in cases.items():
+        assert O.bf16_round(np.array([x]))[0] == want, x
+
+
+# ---------------------------------------------------------------- pooling
+def test_window_counts_and_visibility():
+    # n=1024: 63 stage-1 windows (l=32, s=16) and 15 coarse windows (l=128, s=64)
+    assert O.window_count(1024, 32, 16) == 63
+    assert O.window_count(1024, 128, 64) == 15
+    assert O.window_count(31, 32, 16) == 0
+    assert O.window_count(32768, 32, 16) == 2047
+    assert O.window_count(131072, 128, 64) == 2047
+    # visibility = windows whose whole token range is <= t, by enumeration
+    for (l, s) in ((32, 16), (128, 64)):
+        for t in range(0, 700):
+            brute = sum(1 for j in range(0, 100) if all(u <= t for u in range(s * j, s * j + l)))
+            assert O.visible_windows(t, l, s) == brute
+
+
+def test_pool_constant_blocks():
+    # K constant inside each 64-token block: windows inside a block give its
+    # value, a window over two blocks gives the average of the two.
+    rng = np.random.default_rng(1)
+    n, h, d = 512, 2, 8
+    mu = _bf16(rng.standard_normal((n // 64, h, d)))
+    K = np.repeat(mu, 64, axis=0)
+    c1 = O.pool_keys(K, 32, 16)
+    c2 = O.pool_keys(K, 128, 64)
+    assert c1.shape == (h, 31, d) and c2.shape == (h, 7, d)
+    for j in range(31):
+        b0, b1 = (16 * j) // 64, (16 * j + 31) // 64
+        want = mu[b0] if b0 == b1 else _bf16((mu[b0] + mu[b1]) / 2)
+        np.testing.assert_array_equal(c1[:, j, :], want)
+    for m in range(7):
+        np.testing.assert_array_equal(c2[:, m, :], _bf16((mu[m] + mu[m + 1]) / 2))
+
+
+def test_pool_mean_of_ramp():
+    # K[u] = u (exact in bf16 for u < 256): window j of length l, stride s has
+    # mean s*j + (l-1)/2.
+    n = 256
+    K = np.arange(n, dtype=np.float64).reshape(n, 1, 1)
+    c1 = O.pool_keys(K, 32, 16)[0, :, 0]
+    assert np.array_equal(c1, O.bf16_round(16 * np.arange(15) + 15.5))
+    c2 = O.pool_keys(K, 128, 64)[0, :, 0]
+    assert np.array_equal(c2, O.bf16_round(64 * np.arange(3) + 63.5))
+
+
+# ---------------------------------------------------------------- scoring
+def _seq(n, h_q, h_kv, d, seed, p=O.Params(), q_zero_heads=()):
+    rng = np.random.default_rng(seed)
+    Q = _bf16(rng.standard_normal((n, h_q, d)))
+    for h in q_zero_heads:
+        Q[:, h, :] = 0.0
+    K = _bf16(rng.standard_normal((n, h_kv, d)))
+    V = _bf16(rng.standard_normal((n, h_kv, d)))
+    return O.Sequence1(Q, K, V, p)
+
+
+def test_scores_with_zero_query_are_uniform():
+    # q = 0: every score is 0, LSE = ln(#visible C2 windows), so each visible
+    # C1 window gets G / #C2-windows; before any C2 window is visible the
+    # exact normaliser over the C1 windows gives G / #C1-windows.
+    s = _seq(600, 4, 1, 16, 2, q_zero_heads=range(4))
+    for t in (31, 47, 126, 127, 128, 191, 192, 400, 599):
+        S = s.shared_scores(t, 0)
+        n1 = O.visible_windows(t, 32, 16)
+        n2 = O.visible_windows(t, 128, 64)
+        assert S.shape == (n1,)
+        want = 4.0 / (n2 if n2 > 0 else n1)
+        np.testing.assert_allclose(S, want, rtol=1e-14)
+    assert s.shared_scores(30, 0).shape == (0,)
+
+
+def test_head_to_group_map_is_contiguous():
+    # h_q=4, h_kv=2: group 0 owns heads 0 and 1.  Zero exactly those.
+    s = _seq(400, 4, 2, 16, 3, q_zero_heads=(0, 1))
+    t = 300
+    n2 = O.visible_windows(t, 128, 64)
+    np.testing.assert_allclose(s.shared_scores(t, 0), 2.0 / n2, rtol=1e-14)
+    assert np.ptp(s.shared_scores(t, 1)) > 1e-3
+
+
+def test_exact_lse_rows_sum_to_group_size():
+    # with the exact normaliser each head's probabilities sum to 1 over the
+    # visible windows, so the group sum adds up to G
+    p = O.Params(lse_mode="exact")
+    s = _seq(700, 8, 2, 32, 4, p=p)
+    for t in (31, 100, 333, 699):
+        for g in range(2):
+            assert abs(s.shared_scores(t, g).sum() - 4.0) < 1e-12
+
+
+def test_scale_and_lse_by_hand():
+    # d=64, scale 1/8.  Two C1 windows: k0 = 0, k1 = e_0; every head has
+    # q = 8 e_0, so s = (0, 1).  Exact mode: S = G * (1, e) / (1 + e).
+    d, G = 64, 3
+    q = np.zeros((G, d)); q[:, 0] = 8.0
+    Kc1 = np.zeros((2, d)); Kc1[1, 0] = 1.0
+    p = O.Params(lse_mode="exact")
+    S = O.shared_scores(q, Kc1, np.zeros((0, d)), 47, p, 1.0 / 8.0)
+    e = math.e
+    np.testing.assert_allclose(S, [G / (1 + e), G * e / (1 + e)], rtol=1e-14)
+    # approximate mode: the normaliser comes from the C2 keys only.  One C2
+    # window with k = 2 e_0 gives s2 = 2, LSE = 2, so S = G * (e^-2, e^-1).
+    # At t=127 seven C1 windows are visible: k1 = e_0, the others 0.
+    Kc2 = np.zeros((1, d)); Kc2[0, 0] = 2.0
+    Kc1 = np.zeros((7, d)); Kc1[1, 0] = 1.0
+    S = O.shared_scores(q, Kc1, Kc2, 127, O.Params(), 1.0 / 8.0)
+    want = [G * math.exp(-2)] * 7
+    want[1] = G * math.exp(-1)
+    np.testing.assert_allclose(S, want, rtol=1e-14)
+
+
+# ---------------------------------------------------------------- max-pool
+def test_block_scores_match_token_overlap_definition():
+    # Block b's score is the maximum over the visible C1 windows whose token
+    # span [16j, 16j+31] overlaps the block's span [64b, 64b+63].
+    rng = np.random.default_rng(5)
+    p = O.Params()
+    for t in (63, 64, 200, 777, 1023, 2047):
+        n1 = O.visible_windows(t, 32, 16)
+        S = rng.random(n1)
+        bs = O.block_scores(S, t, p)
+        assert bs.shape == (t // 64 + 1,)
+        for b in range(t // 64 + 1):
+            js = [j for j in range(n1) if 16 * j <= 64 * b + 63 and 16 * j + 31 >= 64 * b]
+            want = max(S[j] for j in js) if js else -np.inf
+            assert bs[b] == want
+    # the max-pool compresses by 4 windows = 64 tokens = one block per output
+    assert O.block_scores(np.ones(8191), 131071, p).shape == (2048,)
+
+
+# ---------------------------------------------------------------- selection
+def test_worked_example_32k():
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    p = O.Params()
+    assert p.block == g["block"] and p.n_sel == g["n_selected_blocks"] and p.n_local == g["n_local"]
+    rng = np.random.default_rng(6)
+    for t in (g["token_1based"] - 1, g["token_1based"]):   # either reading of "the 20000th token"
+        b_t = t // p.block
+        assert b_t + 1 == g["block_1based"]
+        S = rng.random(O.visible_windows(t, 32, 16))
+        sel = O.select_blocks(S, t, p)
+        assert len(sel) == g["n_selected_blocks"] and (sel >= 0).all()
+        assert np.all(np.diff(sel) > 0)
+        s1 = set((sel + 1).tolist())
+        assert set(g["init_blocks_1based"]) <= s1
+        assert set(range(g["local_first_block_1based"], g["local_last_block_1based"] + 1)) <= s1
+        far = s1 - set(g["init_blocks_1based"]) - set(range(g["local_first_block_1based"], 314))
+        assert len(far) == 63 and max(far) < g["local_first_block_1based"]
+        assert len(sel) * p.block == g["visible_tokens"]
+
+
+def test_topk_matches_bruteforce_subsets():
+    # tiny parameters; scores drawn from a few values so ties are common.
+    # The chosen far blocks must be the maximum-sum k-subset, ties broken
+    # toward the lexicographically smallest index set.
+    p = O.Params(n_init=1, n_local=2, top_k=3)
+    rng = np.random.default_rng(7)
+    for trial in range(200):
+        t = int(rng.integers(64 * 5, 64 * 12))
+        n1 = O.visible_windows(t, 32, 16)
+        S = rng.integers(0, 4, n1).astype(np.float64)
+        sel = set(O.select_blocks(S, t, p).tolist()) - {-1}
+        b_t = t // 64
+        bs = O.block_scores(S, t, p)
+        cand = list(range(1, b_t - 1))
+        best = max(itertools.combinations(cand, 3), key=lambda c: (sum(bs[b] for b in c), [-b for b in c]))
+        assert sel == {0, b_t - 1, b_t} | set(best), (trial, t)
+
+
+def test_topk_ties_take_lowest_blocks():
+    # zero query: all block scores tie, so the top-k are the lowest candidates
+    s = _seq(1024 * 8, 4, 1, 16, 8, q_zero_heads=range(4))
+    p = s.p
+    t = 8000
+    sel = s.select(t, 0)
+    b_t = t // 64
+    want = [0] + list(range(1, 1 + p.top_k)) + list(range(b_t - 31, b_t + 1))
+    assert sel.tolist() == want
+
+
+def test_selected_count_and_always_selected():
+    s = _seq(5000, 4, 1, 16, 9)
+    for t in (0, 63, 64, 2111, 2112, 4000, 4999):
+        sel = s.select(t, 0)
+        b_t = t // 64
+        valid = sel[sel >= 0]
+        assert len(valid) == min(96, b_t + 1)
+        assert 0 in valid
+        assert set(range(max(0, b_t - 31), b_t + 1)) <= set(valid.tolist())
+        assert (sel[len(valid):] == -1).all()
+
+
+# ---------------------------------------------------------------- attention
+def test_dense_matches_library_sdpa():
+    rng = np.random.default_rng(10)
+    n, h_q, h_kv, d = 200, 4, 2, 16
+    s = _seq(n, h_q, h_kv, d, 10)
+    G = h_q // h_kv
+    q = torch.from_numpy(s.Q).permute(1, 0, 2)[None]
+    k = torch.from_numpy(s.K).permute(1, 0, 2).repeat_interleave(G, 0)[None]
+    v = torch.from_numpy(s.V).permute(1, 0, 2).repeat_interleave(G, 0)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)[0].permute(1, 0, 2).numpy()
+    for t in range(0, n, 7):
+        for g in range(h_kv):
+            np.testing.assert_allclose(s.dense_out(t, g), ref[t, g * G:(g + 1) * G], rtol=1e-12, atol=1e-13)
+
+
+def test_sparse_equals_dense_when_every_block_is_selected():
+    # |I| >= number of causal blocks -> sparse attention is dense attention
+    p = O.Params(n_init=1, n_local=16, top_k=2)
+    s = _seq(1024, 4, 1, 64, 11, p=p)
+    for t in range(0, 1024, 13):
+        sel = s.select(t, 0)
+        assert sorted(sel[sel >= 0].tolist()) == list(range(t // 64 + 1))
+        np.testing.assert_allclose(s.sparse_out(t, 0, sel), s.dense_out(t, 0), rtol=1e-13, atol=1e-14)
+
+
+def test_zero_query_gives_mean_of_visible_values():
+    s = _seq(3000, 4, 1, 16, 12, q_zero_heads=range(4))
+    for t in (5, 64, 130, 2500, 2999):
+        sel = s.select(t, 0)
+        keys = [u for u in range(t + 1) if (u // 64) in set(sel.tolist())]
+        want = s.V[keys, 0, :].mean(axis=0)
+        out = s.sparse_out(t, 0, sel)
+        for h in range(4):
+            np.testing.assert_allclose(out[h], want, rtol=1e-12, atol=1e-14)
+
+
+def test_dense_route_threshold():
+    assert O.dense_route(8192) and not O.dense_route(8193) and O.dense_route(1)
