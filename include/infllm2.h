@@ -1,0 +1,201 @@
+/*
+ * libinfllm2 — InfLLM-V2 sparse-attention forward path for grouped-query
+ * attention on NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The method (InfLLM-V2: dense-sparse switchable attention) is described on
+ * these pages, cited below by their titles:
+ *   [blog]   "论文阅读：InfLLM-V2 — 把可训练稀疏注意力做成全注意力的'受限版本'"
+ *            (xiaohongrsx.github.io paper-reading notes)
+ *   [news]   "从密集到稀疏：InfLLM-V2 如何实现零参数开销的长文本高效处理" (dtcms.com)
+ *   [top168] top168.com article on InfLLM-V2 (Tsinghua / OpenBMB,
+ *            arXiv 2509.24663), sections 三, 四, 七
+ *
+ * Data layout (all calls).
+ *   Sequences are packed token-major ("THD"): Q [total, h_q, d],
+ *   K and V [total, h_kv, d], bf16, row-major, contiguous in d.  Sequence s
+ *   holds rows cu_seqlens[s] .. cu_seqlens[s+1]-1.  Blocks (64 tokens) and
+ *   pooling windows restart at every sequence start.  Query head h belongs
+ *   to kv group h / (h_q / h_kv).  d is 64 or 128; h_q % h_kv == 0 and
+ *   G = h_q / h_kv is a power of two <= 16.  Every device pointer must be
+ *   16-byte aligned.
+ *
+ * Ownership.  The caller allocates every buffer (workspaces included) and
+ * keeps ownership; no call allocates or frees device memory, none
+ * synchronises the stream, and no pointer is kept after a call returns.
+ * Calls are asynchronous on the given stream (a cudaStream_t passed as
+ * void*; NULL is the legacy default stream).
+ *
+ * Errors.  Every call returns INFLLM2_OK (0) or a negative INFLLM2_ERR_*
+ * code.  Arguments are checked before anything is launched; on an argument
+ * error nothing is written.  INFLLM2_ERR_CUDA means a launch failed (the
+ * CUDA error text is kept for infllm2_status_string).  Kernels that detect a
+ * problem on the device (a bounded wait that ran out, an index out of range)
+ * record it in a per-device status word instead of trapping; read it with
+ * infllm2_get_device_status after synchronising.
+ */
+#ifndef INFLLM2_H_
+#define INFLLM2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  INFLLM2_OK = 0,
+  INFLLM2_ERR_INVALID_ARG = -1,        /* null pointer, bad size, misalignment */
+  INFLLM2_ERR_UNSUPPORTED = -2,        /* valid but not implemented (d, G, params) */
+  INFLLM2_ERR_WORKSPACE_TOO_SMALL = -3,
+  INFLLM2_ERR_CUDA = -4,               /* a CUDA runtime call or launch failed */
+  INFLLM2_ERR_DEVICE_TIMEOUT = -5,     /* device status: a bounded wait ran out */
+  INFLLM2_ERR_DEVICE_BOUNDS = -6       /* device status: an index check failed */
+};
+
+enum { INFLLM2_OUT_BF16 = 0, INFLLM2_OUT_F32 = 1 };
+enum { INFLLM2_LSE_APPROX = 0 };
+
+/* Method parameters.  Defaults (infllm2_default_params) are the pages'
+ * values: block B = 64 ([blog] worked example "每块 64 个 token");
+ * stage-1 windows l_C1 = B/2 = 32, s_C1 = B/4 = 16 and stage-3 max-pool
+ * kernel 5, stride 4 ([top168] §三); coarse windows for the LSE approximation
+ * l_C2 = 4 l_C1 = 128, s_C2 = 4 s_C1 = 64 ([top168] §四); 1 initial block,
+ * 32 local blocks and 63 top-k blocks, |I| = 96 ([blog] worked example).
+ * The kernels implement exactly these pooling geometries; any other value of
+ * block_size, c1_*, c2_*, pool_* returns INFLLM2_ERR_UNSUPPORTED.  n_init,
+ * n_local (>= 1) and top_k are free (|I| = n_init + n_local + top_k <= 4096). */
+typedef struct {
+  int32_t block_size;      /* B = 64 */
+  int32_t c1_len;          /* 32 */
+  int32_t c1_stride;       /* 16 */
+  int32_t c2_len;          /* 128 */
+  int32_t c2_stride;       /* 64 */
+  int32_t pool_len;        /* 5 */
+  int32_t pool_stride;     /* 4 */
+  int32_t pool_pad;        /* 1 */
+  int32_t n_init;          /* 1 */
+  int32_t n_local;         /* 32, includes the query's own block */
+  int32_t top_k;           /* 63 */
+  float scale;             /* softmax scale; <= 0 selects 1/sqrt(d) */
+  int32_t lse_mode;        /* INFLLM2_LSE_APPROX */
+  int32_t dense_threshold; /* 8192: sequences of at most this length take the dense path */
+} infllm2_params;
+
+/* Packed variable-length batch geometry.  cu_seqlens is a DEVICE array of
+ * batch+1 int32 offsets (cu_seqlens[0] = 0, cu_seqlens[batch] = total);
+ * the other fields are host values: max_seqlen = longest sequence, total =
+ * number of packed tokens, total_c1 / total_c2 = number of pooled rows
+ * (the sum over sequences of infllm2_window_count(len, 32, 16) and
+ * infllm2_window_count(len, 128, 64)); these are the row capacities of the
+ * pooled-key buffers. */
+typedef struct {
+  const int32_t* cu_seqlens;
+  int32_t batch;
+  int32_t max_seqlen;
+  int64_t total;
+  int64_t total_c1;
+  int64_t total_c2;
+} infllm2_varlen;
+
+infllm2_params infllm2_default_params(void);
+const char* infllm2_status_string(int status);
+
+/* Number of complete pooling windows of `len` tokens taken every `stride`
+ * tokens inside a sequence of n tokens (partial windows are dropped). */
+int64_t infllm2_window_count(int64_t n, int32_t len, int32_t stride);
+
+/* Leading dimension (floats) of the S_shared rows for this batch:
+ * max window count rounded up to a multiple of 4. */
+int64_t infllm2_scores_ld(const infllm2_varlen* vl, const infllm2_params* p);
+
+/* ---------------------------------------------------------------------
+ * Step 1: stage-1 and coarse mean pooling of K  ([top168] §三 first stage,
+ * §四 coarse scores S_C2).  For each sequence and kv head g:
+ *   K_c1[g, c1_off(s) + j] = bf16_rne(mean(K[16j .. 16j+31, g]))  j < n_c1(len)
+ *   K_c2[g, c2_off(s) + m] = bf16_rne(mean(K[64m .. 64m+127, g])) m < n_c2(len)
+ * where c1_off(s) is the number of C1 windows of the sequences before s.
+ * The mean is exact (fp64 sum) before the single rounding to bf16.
+ *   K     bf16 [total, h_kv, d]                  (input)
+ *   K_c1  bf16 [h_kv, total_c1, d]               (output)
+ *   K_c2  bf16 [h_kv, total_c2, d]               (output)
+ * ------------------------------------------------------------------- */
+int infllm2_compress_k(const void* K, const infllm2_varlen* vl, int32_t h_kv, int32_t d,
+                       void* K_c1, void* K_c2, const infllm2_params* p, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Step 2: compressed scores with the LSE approximation and the fused
+ * head-group sum ([top168] §三 second stage, §四).  For query token t of a
+ * sequence and kv group g, with s_h(j) = scale * q[t,h] . K_c1[g,j]:
+ *   LSE_h  = log sum_{m visible} exp(scale * q[t,h] . K_c2[g,m])
+ *   S[g, t, j] = sum_{h in group g} exp(s_h(j) - LSE_h)   for visible j
+ * A C1 window j is visible when 16j+31 <= t, a C2 window m when 64m+127 <= t
+ * (positions within the sequence).  Rows with no visible C2 window
+ * (t < 127) take the exact log-sum-exp over their visible C1 windows.
+ * Only visible entries are written; the per-head scores never reach HBM.
+ *   Q          bf16 [total, h_q, d]
+ *   K_c1, K_c2 as written by infllm2_compress_k
+ *   S          fp32 [h_kv, total, ld], ld = infllm2_scores_ld(vl, p)
+ * ------------------------------------------------------------------- */
+int infllm2_shared_scores(const void* Q, const void* K_c1, const void* K_c2,
+                          const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
+                          float* S, int64_t ld, const infllm2_params* p, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Step 3: stage-3 max-pool and block selection ([top168] §三 third stage,
+ * §七; [blog] worked example).  For query token t (block b_t = t / 64):
+ *   score(b) = max{ S[g,t,j] : 4b-1 <= j <= 4b+3, j visible }
+ *   I = {0..n_init-1} U {b_t-n_local+1 .. b_t} U top_k of the remaining
+ *       blocks 0..b_t by score (ties go to the lower block index),
+ * clipped to [0, b_t]; listed ascending, padded with -1.
+ *   S          fp32 [h_kv, total, ld]
+ *   block_idx  int32 [h_kv, total, n_init+n_local+top_k]   (output)
+ * ------------------------------------------------------------------- */
+int infllm2_topk_blocks(const float* S, int64_t ld, const infllm2_varlen* vl, int32_t h_kv,
+                        int32_t* block_idx, const infllm2_params* p, void* stream);
+
+/* Steps 2 and 3 in one call.  S_shared goes to `workspace` (at least
+ * infllm2_select_workspace_bytes bytes) unless s_shared_out is non-NULL, in
+ * which case it is written there ([h_kv, total, ld] fp32) and the workspace
+ * may be NULL. */
+size_t infllm2_select_workspace_bytes(const infllm2_varlen* vl, int32_t h_kv, const infllm2_params* p);
+int infllm2_select_blocks(const void* Q, const void* K_c1, const void* K_c2,
+                          const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
+                          void* workspace, size_t workspace_bytes, int32_t* block_idx,
+                          float* s_shared_out, const infllm2_params* p, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Step 4: block-sparse causal attention ([blog] "对齐计算图": selected and
+ * sliding attention merged into one sparse attention with a single output;
+ * [top168] §七).  For token t of a sequence and query head h of group g:
+ *   out[t,h] = softmax_u(scale * q[t,h] . K[u,g]) V[u,g]
+ * over u <= t with u / 64 in block_idx[g, t, :] (entries < 0 ignored).
+ *   out  [total, h_q, d], bf16 (INFLLM2_OUT_BF16) or fp32 (INFLLM2_OUT_F32)
+ * ------------------------------------------------------------------- */
+int infllm2_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* block_idx,
+                        const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
+                        void* out, int32_t out_dtype, const infllm2_params* p, void* stream);
+
+/* Dense causal attention, the short-sequence side of the dense/sparse switch
+ * ([blog] "Dense-Sparse Switchable Attention"; [news] §二.2.c).  Same
+ * arguments and output form as infllm2_sparse_attn, all u <= t attended. */
+int infllm2_dense_attn(const void* Q, const void* K, const void* V,
+                       const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
+                       void* out, int32_t out_dtype, const infllm2_params* p, void* stream);
+
+/* Device status word (per device).  Returns INFLLM2_OK or the first
+ * INFLLM2_ERR_DEVICE_* recorded by a kernel since the last clear.
+ * Synchronises the device. */
+int infllm2_get_device_status(void);
+int infllm2_clear_device_status(void);
+
+/* Diagnostic: launches one block that waits on a barrier nothing will ever
+ * complete, with a bound of `limit_ns` nanoseconds; the wait gives up,
+ * records INFLLM2_ERR_DEVICE_TIMEOUT in the device status word and returns.
+ * Used to test the bounded-wait path without hanging a GPU. */
+int infllm2_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* INFLLM2_H_ */

@@ -1,0 +1,99 @@
+"""The C-ABI library builds, loads without a GPU, exports every entry
+point that include/infllm2.h declares, and rejects bad arguments on the host
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import trainable_block_sparse_pool_b200 as T
+from trainable_block_sparse_pool_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "infllm2.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return T.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(infllm2_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_defaults_follow_the_pages(L):
+    p = T.default_params()
+    assert (p.block_size, p.c1_len, p.c1_stride, p.c2_len, p.c2_stride) == (64, 32, 16, 128, 64)
+    assert (p.pool_len, p.pool_stride, p.pool_pad) == (5, 4, 1)
+    assert (p.n_init, p.n_local, p.top_k, p.n_sel) == (1, 32, 63, 96)
+    assert p.dense_threshold == 8192
+
+
+def test_window_count_and_ld(L):
+    assert T.window_count(1024, 32, 16) == 63
+    assert T.window_count(1024, 128, 64) == 15
+    assert T.window_count(31, 32, 16) == 0
+    vl = T.Varlen()
+    vl.max_seqlen = 131072
+    assert T.infllm2_scores_ld(vl) == 8192      # 8191 windows rounded up to a multiple of 4
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert L.infllm2_status_string(code)
+
+
+def _vl(batch=1, max_seqlen=1024, total=1024):
+    vl = T.Varlen()
+    vl.cu_seqlens = 0x1000
+    vl.batch, vl.max_seqlen, vl.total = batch, max_seqlen, total
+    vl.total_c1, vl.total_c2 = 63, 15
+    return vl
+
+
+def test_argument_errors_are_caught_on_host(L):
+    p = T.default_params()
+    vl = _vl()
+    by = ctypes.byref
+    # null pointers
+    assert L.infllm2_compress_k(None, by(vl), 1, 64, 0x1000, 0x1000, by(p), None) == -1
+    # misaligned pointer
+    assert L.infllm2_compress_k(0x1008, by(vl), 1, 64, 0x1000, 0x1000, by(p), None) == -1
+    # unsupported head dim and group size
+    assert L.infllm2_shared_scores(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 96, 0x1000, 64, by(p), None) == -2
+    assert L.infllm2_shared_scores(0x1000, 0x1000, 0x1000, by(vl), 6, 2, 64, 0x1000, 64, by(p), None) == -2
+    assert L.infllm2_shared_scores(0x1000, 0x1000, 0x1000, by(vl), 5, 2, 64, 0x1000, 64, by(p), None) == -1
+    # ld too small
+    assert L.infllm2_shared_scores(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 60, by(p), None) == -1
+    # unsupported pooling geometry
+    q = T.default_params(c1_len=48)
+    assert L.infllm2_topk_blocks(0x1000, 64, by(vl), 1, 0x1000, by(q), None) == -2
+    q = T.default_params(n_local=0)
+    assert L.infllm2_topk_blocks(0x1000, 64, by(vl), 1, 0x1000, by(q), None) == -1
+    # workspace too small
+    assert L.infllm2_select_blocks(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 16, 0x1000, None, by(p),
+                                   None) == -3
+    # bad output dtype
+    assert L.infllm2_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 7, by(p), None) == -1
+    # inconsistent varlen
+    bad = _vl(batch=0)
+    assert L.infllm2_dense_attn(0x1000, 0x1000, 0x1000, by(bad), 4, 1, 64, 0x1000, 0, by(p), None) == -1
+    bad = _vl(max_seqlen=2048, total=1024)
+    assert L.infllm2_dense_attn(0x1000, 0x1000, 0x1000, by(bad), 4, 1, 64, 0x1000, 0, by(p), None) == -1
+    assert L.infllm2_debug_wait_timeout(0, None) == -1
+
+
+def test_workspace_size(L):
+    vl = _vl(max_seqlen=131072, total=131072)
+    assert T.infllm2_select_workspace_bytes(vl, 2) == 2 * 131072 * 8192 * 4

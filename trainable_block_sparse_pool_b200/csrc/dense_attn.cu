@@ -1,0 +1,334 @@
+// Dense causal attention: the short-sequence side of InfLLM-V2's dense/sparse
+// switch (paper-reading blog, "Dense-Sparse Switchable Attention"; dtcms
+// article §二.2.c).  Same inputs and output form as the sparse kernel.
+//
+// A CTA owns one kv group and TQ = 128/G consecutive query tokens: its 128
+// query rows (t, h) share every key of the group, so one K/V tile feeds all
+// of them (GQA packing).  Per 128-key tile:
+//   S[128 rows, 128 keys] = Q . K^T        tcgen05, A = Q (smem), B = K (smem)
+//   softmax, one thread per row (two passes over the TMEM row: max, then
+//   exp2 + bf16 P written to shared memory in the 128-byte-swizzled K-major
+//   layout the next MMA reads)
+//   O_tile[128 rows, d] = P . V            A = P (smem), B = V (MN-major)
+// O_tile lands in a fresh TMEM accumulator and is folded into registers
+// (O = O * alpha + O_tile) by the row's thread.
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer / TMEM owner,
+// warps 2-5 softmax + correction.
+#include "sm100.cuh"
+
+namespace infllm2 {
+
+namespace dense {
+
+constexpr int kThreads = 192;
+constexpr int kKeys = 128;
+constexpr int kStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, int G>
+struct Cfg {
+  static constexpr int TQ = 128 / G;
+  static constexpr int KCH = D / 64;
+  static constexpr uint32_t kQBytes = 128 * 128 * KCH;
+  static constexpr uint32_t kChunk = kKeys * 128;            // 16 KB
+  static constexpr uint32_t kKBytes = kChunk * KCH;
+  static constexpr uint32_t kStageBytes = 2 * kKBytes;
+  static constexpr uint32_t kPBytes = 128 * 128 * 2;         // 128 rows x 128 keys bf16, 2 chunks
+  static constexpr uint32_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + 512;
+  static constexpr uint32_t kOCol = 256;                     // O buffers after the two S buffers
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t s_empty[2];
+  uint64_t p_full;
+  uint64_t o_full[2];
+  uint64_t o_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool aborted(const Bars* b) { return *reinterpret_cast<const volatile int*>(&b->abort) != 0; }
+__device__ __forceinline__ void set_abort(Bars* b) { *reinterpret_cast<volatile int*>(&b->abort) = 1; }
+
+template <int D, int G, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu, int h_q, float scale,
+    void* __restrict__ out) {
+  using C = Cfg<D, G>;
+  constexpr int TQ = C::TQ;
+  static_assert(G >= 1 && G <= 16 && (16 % G) == 0, "group size must be a power of two <= 16");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + C::kQBytes;
+  uint8_t* sP = sKV + kStages * C::kStageBytes;
+  Bars* bars = reinterpret_cast<Bars*>(sP + C::kPBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.y, g = blockIdx.z;
+  const int row0 = cu[s];
+  const int len = cu[s + 1] - row0;
+  const int ntiles = (len + TQ - 1) / TQ;
+  if (static_cast<int>(blockIdx.x) >= ntiles) return;
+  const int t0 = (ntiles - 1 - blockIdx.x) * TQ;        // heaviest query tiles first
+  const int t_last = min(len - 1, t0 + TQ - 1);
+  const int nkt = t_last / kKeys + 1;                    // key tiles covering 0 .. t_last
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_empty[i], 4);
+      mbar_init(&bars->o_full[i], 1);
+      mbar_init(&bars->o_empty[i], 4);
+    }
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(&bars->tmem_base, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bars->q_full, C::kQBytes);
+      for (int ch = 0; ch < C::KCH; ++ch) tma_load_4d(sQ + ch * 16384, &tmQ, &bars->q_full, ch * 64, 0, g, row0 + t0);
+      int it = 0;
+      for (; it < nkt; ++it) {
+        const int st = it % kStages;
+        if (!mbar_wait(&bars->kv_empty[st], ((it / kStages) & 1) ^ 1) || aborted(bars)) { set_abort(bars); break; }
+        uint8_t* dK = sKV + st * C::kStageBytes;
+        uint8_t* dV = dK + C::kKBytes;
+        mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
+        for (int ch = 0; ch < C::KCH; ++ch) {
+          tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, g, row0 + it * kKeys);
+          tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, g, row0 + it * kKeys);
+        }
+      }
+      mbar_wait(&bars->q_full, 0);
+      for (int i = max(0, it - kStages); i < it; ++i) mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(128, kKeys, 0, 0);
+      const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t p_base = smem_u32(sP);
+      bool ok = mbar_wait(&bars->q_full, 0);
+      if (!ok) set_abort(bars);
+      auto issue_pv = [&](int j) -> bool {
+        const int pb = j & 1;
+        const int st = j % kStages;
+        if (!mbar_wait(&bars->p_full, j & 1)) return false;
+        if (!mbar_wait(&bars->o_empty[pb], ((j >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(sKV + st * C::kStageBytes + C::kKBytes);
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k) {
+          const uint64_t a = make_sdesc(p_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kLayoutSW128);
+          const uint64_t b = make_sdesc(v_base + k * 2048, C::kChunk, 1024, kLayoutSW128);
+          umma_bf16(tmem + C::kOCol + pb * D, a, b, idO, k > 0);
+        }
+        umma_commit(&bars->kv_empty[st]);
+        umma_commit(&bars->o_full[pb]);
+        return true;
+      };
+      int it = 0;
+      for (; ok && it < nkt; ++it) {
+        const int st = it % kStages;
+        const int sb = it & 1;
+        if (!mbar_wait(&bars->kv_full[st], (it / kStages) & 1) ||
+            !mbar_wait(&bars->s_empty[sb], ((it >> 1) & 1) ^ 1) || aborted(bars)) {
+          set_abort(bars); ok = false; break;
+        }
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(sKV + st * C::kStageBytes);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t a = make_sdesc(q_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kLayoutSW128);
+          const uint64_t b = make_sdesc(k_base + (k >> 2) * C::kChunk + (k & 3) * 32, 16, 1024, kLayoutSW128);
+          umma_bf16(tmem + sb * kKeys, a, b, idS, k > 0);
+        }
+        umma_commit(&bars->s_full[sb]);
+        if (it > 0 && !issue_pv(it - 1)) { set_abort(bars); ok = false; break; }
+      }
+      if (ok && nkt > 0 && !issue_pv(nkt - 1)) set_abort(bars);
+      umma_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0);
+    }
+  } else {
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;                 // query row (t_loc, h)
+    const int t = t0 + r / G;
+    const int h = r % G;
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const float c = scale * kLog2e;
+    float o_acc[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) o_acc[j] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    // swizzled P row: 16-byte unit q of 128-byte row r sits at unit q ^ (r & 7)
+    uint8_t* prow = sP + (r >> 3) * 1024 + (r & 7) * 128;
+    bool ok = true;
+    for (int it = 0; it < nkt; ++it) {
+      const int sb = it & 1;
+      if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_addr + sb * kKeys;
+      const int kbase = it * kKeys;
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int cc = 0; cc < kKeys; cc += 16) {
+        float v[16];
+        tmem_ld16(s_addr + cc, v);
+        tmem_wait_ld16(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) if (kbase + cc + i <= t) mx = fmaxf(mx, v[i] * c);
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const bool none = (m_new == -INFINITY);
+      const float alpha = none ? 1.f : ex2(m_run - m_new);
+      float lsum = 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < kKeys; cc += 16) {
+        float v[16];
+        tmem_ld16(s_addr + cc, v);
+        tmem_wait_ld16(v);
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          const float p0 = (!none && kbase + cc + i <= t) ? ex2(fmaf(v[i], c, -m_new)) : 0.f;
+          const float p1 = (!none && kbase + cc + i + 1 <= t) ? ex2(fmaf(v[i + 1], c, -m_new)) : 0.f;
+          lsum += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[i >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        // keys cc .. cc+15 of this tile: chunk cc/64, 16-byte units (cc%64)/8 and +1
+        const int chunk = cc >> 6;
+        const int u0 = (cc & 63) >> 3;
+        uint8_t* base = prow + chunk * 16384;
+        *reinterpret_cast<uint4*>(base + ((u0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(base + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) { mbar_arrive(&bars->p_full); mbar_arrive(&bars->s_empty[sb]); }
+      // fold this tile's P.V into the registers
+      const int pb = it & 1;
+      if (!mbar_wait(&bars->o_full[pb], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_addr + C::kOCol + pb * D + cc, v);
+        tmem_wait_ld16(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o_acc[cc + i] = fmaf(o_acc[cc + i], alpha, v[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_empty[pb]);
+    }
+    if (ok && t < len) {
+      const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const int64_t base = (static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h) * D;
+      if (OUT_F32) {
+        float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + base);
+#pragma unroll
+        for (int j = 0; j < D; j += 4)
+          o4[j / 4] = make_float4(o_acc[j] * inv, o_acc[j + 1] * inv, o_acc[j + 2] * inv, o_acc[j + 3] * inv);
+      } else {
+        uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + base);
+#pragma unroll
+        for (int j = 0; j < D; j += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(o_acc[j + 2 * q] * inv, o_acc[j + 2 * q + 1] * inv);
+            w[q] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          o4[j / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace dense
+
+bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+               const uint32_t* box);
+
+template <int D, int G, bool F32>
+static cudaError_t launch_dense_t(const void* Q, const void* K, const void* V, const int32_t* cu, int batch,
+                                  int max_seqlen, int64_t total, int h_q, int h_kv, float scale, void* out,
+                                  cudaStream_t st, bool* map_fail) {
+  using C = dense::Cfg<D, G>;
+  CUtensorMap mQ, mK, mV;
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)G, (uint64_t)h_kv, (uint64_t)total};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)G * D * 2, (uint64_t)h_q * D * 2};
+    const uint32_t box[4] = {64, (uint32_t)G, 1, (uint32_t)C::TQ};
+    if (!make_tmap(&mQ, Q, 4, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)h_kv, (uint64_t)total};
+    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)h_kv * D * 2};
+    const uint32_t box[3] = {64, 1, dense::kKeys};
+    if (!make_tmap(&mK, K, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
+    if (!make_tmap(&mV, V, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
+  }
+  auto kern = dense::dense_attn_kernel<D, G, F32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((max_seqlen + C::TQ - 1) / C::TQ, batch, h_kv);
+  if (grid.x == 0) return cudaSuccess;
+  kern<<<grid, dense::kThreads, C::kSmem, st>>>(mQ, mK, mV, cu, h_q, scale, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense_attn(const void* Q, const void* K, const void* V, const int32_t* cu, int batch,
+                              int max_seqlen, int64_t total, int h_q, int h_kv, int d, float scale, void* out,
+                              bool out_f32, cudaStream_t st, bool* map_fail) {
+  const int G = h_q / h_kv;
+#define INFLLM2_DENSE_CASE(DD, GG)                                                                               \
+  if (d == DD && G == GG)                                                                                       \
+    return out_f32 ? launch_dense_t<DD, GG, true>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, out, st, \
+                                                  map_fail)                                                    \
+                   : launch_dense_t<DD, GG, false>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, out, \
+                                                   st, map_fail);
+  INFLLM2_DENSE_CASE(128, 16)
+  INFLLM2_DENSE_CASE(128, 8)
+  INFLLM2_DENSE_CASE(128, 4)
+  INFLLM2_DENSE_CASE(128, 2)
+  INFLLM2_DENSE_CASE(128, 1)
+  INFLLM2_DENSE_CASE(64, 16)
+  INFLLM2_DENSE_CASE(64, 8)
+  INFLLM2_DENSE_CASE(64, 4)
+  INFLLM2_DENSE_CASE(64, 2)
+  INFLLM2_DENSE_CASE(64, 1)
+#undef INFLLM2_DENSE_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace infllm2

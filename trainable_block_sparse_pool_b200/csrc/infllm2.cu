@@ -1,0 +1,267 @@
+// libinfllm2: the C-ABI entry points declared in include/infllm2.h.
+//
+// The library is one translation unit (the kernel files are included
+// below) so that the per-device status word has a single definition.
+// Host code here checks arguments, builds TMA tensor maps and launches; it
+// never allocates device memory and never synchronises a stream (except
+// infllm2_get_device_status, which is documented to).
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "sm100.cuh"
+
+#include "compress.cu"
+#include "score.cu"
+#include "select.cu"
+#include "sparse_attn.cu"
+#include "dense_attn.cu"
+#include "decode.cu"
+
+namespace infllm2 {
+
+static thread_local char g_err_text[256] = "";
+
+static int cuda_fail(cudaError_t e) {
+  snprintf(g_err_text, sizeof(g_err_text), "CUDA error: %s", cudaGetErrorString(e));
+  return INFLLM2_ERR_CUDA;
+}
+
+PFN_encodeTiled get_encode_tiled() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool geometry_supported(const infllm2_params* p) {
+  return p->block_size == 64 && p->c1_len == 32 && p->c1_stride == 16 && p->c2_len == 128 &&
+         p->c2_stride == 64 && p->pool_len == 5 && p->pool_stride == 4 && p->pool_pad == 1 &&
+         p->lse_mode == INFLLM2_LSE_APPROX;
+}
+
+static int check_varlen(const infllm2_varlen* vl) {
+  if (!vl || !vl->cu_seqlens || vl->batch < 1 || vl->batch > 65535 || vl->max_seqlen < 0 || vl->total < 0 ||
+      vl->total_c1 < 0 || vl->total_c2 < 0 || vl->total > INT32_MAX || vl->max_seqlen > vl->total)
+    return INFLLM2_ERR_INVALID_ARG;
+  return INFLLM2_OK;
+}
+
+static int check_heads(int32_t h_q, int32_t h_kv, int32_t d) {
+  if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0) return INFLLM2_ERR_INVALID_ARG;
+  const int G = h_q / h_kv;
+  if (d != 64 && d != 128) return INFLLM2_ERR_UNSUPPORTED;
+  if (G > 16 || (G & (G - 1)) != 0) return INFLLM2_ERR_UNSUPPORTED;
+  return INFLLM2_OK;
+}
+
+static int check_params(const infllm2_params* p) {
+  if (!p) return INFLLM2_ERR_INVALID_ARG;
+  if (!geometry_supported(p)) return INFLLM2_ERR_UNSUPPORTED;
+  if (p->n_init < 0 || p->n_local < 1 || p->top_k < 0) return INFLLM2_ERR_INVALID_ARG;
+  if (p->n_init + p->n_local + p->top_k > 4096) return INFLLM2_ERR_UNSUPPORTED;
+  return INFLLM2_OK;
+}
+
+// A single thread waits on a barrier that nothing will ever complete; the
+// bounded wait gives up after limit_ns and records the timeout status.
+__global__ void debug_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, limit_ns);
+  __syncthreads();
+}
+
+static float softmax_scale(const infllm2_params* p, int d) {
+  return p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(d));
+}
+
+}  // namespace infllm2
+
+using namespace infllm2;
+
+extern "C" {
+
+infllm2_params infllm2_default_params(void) {
+  infllm2_params p;
+  p.block_size = 64;
+  p.c1_len = 32;
+  p.c1_stride = 16;
+  p.c2_len = 128;
+  p.c2_stride = 64;
+  p.pool_len = 5;
+  p.pool_stride = 4;
+  p.pool_pad = 1;
+  p.n_init = 1;
+  p.n_local = 32;
+  p.top_k = 63;
+  p.scale = 0.f;
+  p.lse_mode = INFLLM2_LSE_APPROX;
+  p.dense_threshold = 8192;
+  return p;
+}
+
+const char* infllm2_status_string(int status) {
+  switch (status) {
+    case INFLLM2_OK: return "ok";
+    case INFLLM2_ERR_INVALID_ARG: return "invalid argument";
+    case INFLLM2_ERR_UNSUPPORTED: return "unsupported configuration";
+    case INFLLM2_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case INFLLM2_ERR_CUDA: return g_err_text[0] ? g_err_text : "CUDA error";
+    case INFLLM2_ERR_DEVICE_TIMEOUT: return "device: a bounded wait ran out";
+    case INFLLM2_ERR_DEVICE_BOUNDS: return "device: an index check failed";
+    default: return "unknown status";
+  }
+}
+
+int64_t infllm2_window_count(int64_t n, int32_t len, int32_t stride) {
+  if (len <= 0 || stride <= 0 || n < len) return 0;
+  return (n - len) / stride + 1;
+}
+
+int64_t infllm2_scores_ld(const infllm2_varlen* vl, const infllm2_params* p) {
+  if (!vl || !p || vl->max_seqlen < 0) return 0;
+  const int64_t n1 = infllm2_window_count(vl->max_seqlen, p->c1_len, p->c1_stride);
+  return std::max<int64_t>(4, (n1 + 3) & ~int64_t(3));
+}
+
+int infllm2_compress_k(const void* K, const infllm2_varlen* vl, int32_t h_kv, int32_t d, void* K_c1, void* K_c2,
+                       const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p))) return r;
+  if (!K || !K_c1 || !K_c2 || !aligned16(K) || !aligned16(K_c1) || !aligned16(K_c2)) return INFLLM2_ERR_INVALID_ARG;
+  if (h_kv <= 0) return INFLLM2_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INFLLM2_ERR_UNSUPPORTED;
+  cudaError_t e = launch_compress_k(K, vl->cu_seqlens, vl->batch, vl->max_seqlen, h_kv, d, K_c1, vl->total_c1,
+                                    K_c2, vl->total_c2, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_shared_scores(const void* Q, const void* K_c1, const void* K_c2, const infllm2_varlen* vl, int32_t h_q,
+                          int32_t h_kv, int32_t d, float* S, int64_t ld, const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
+  if (!Q || !K_c1 || !K_c2 || !S || !aligned16(Q) || !aligned16(K_c1) || !aligned16(K_c2) || !aligned16(S))
+    return INFLLM2_ERR_INVALID_ARG;
+  if (ld < infllm2_scores_ld(vl, p) || (ld & 3)) return INFLLM2_ERR_INVALID_ARG;
+  bool map_fail = false;
+  cudaError_t e = launch_shared_scores(Q, K_c1, K_c2, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total,
+                                       vl->total_c1, vl->total_c2, h_q, h_kv, d, S, ld, softmax_scale(p, d),
+                                       static_cast<cudaStream_t>(stream), &map_fail);
+  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_topk_blocks(const float* S, int64_t ld, const infllm2_varlen* vl, int32_t h_kv, int32_t* block_idx,
+                        const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p))) return r;
+  if (!S || !block_idx || !aligned16(S) || h_kv <= 0) return INFLLM2_ERR_INVALID_ARG;
+  if (ld < infllm2_scores_ld(vl, p) || (ld & 3)) return INFLLM2_ERR_INVALID_ARG;
+  cudaError_t e = launch_topk(S, ld, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_kv, p->n_init,
+                              p->n_local, p->top_k, static_cast<cudaStream_t>(stream), block_idx);
+  if (e == cudaErrorInvalidValue) return INFLLM2_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+size_t infllm2_select_workspace_bytes(const infllm2_varlen* vl, int32_t h_kv, const infllm2_params* p) {
+  if (!vl || !p || h_kv <= 0 || vl->total < 0) return 0;
+  return static_cast<size_t>(h_kv) * static_cast<size_t>(vl->total) * static_cast<size_t>(infllm2_scores_ld(vl, p)) *
+         sizeof(float);
+}
+
+int infllm2_select_blocks(const void* Q, const void* K_c1, const void* K_c2, const infllm2_varlen* vl, int32_t h_q,
+                          int32_t h_kv, int32_t d, void* workspace, size_t workspace_bytes, int32_t* block_idx,
+                          float* s_shared_out, const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
+  if (!block_idx) return INFLLM2_ERR_INVALID_ARG;
+  float* S = s_shared_out;
+  if (!S) {
+    if (!workspace) return INFLLM2_ERR_INVALID_ARG;
+    if (workspace_bytes < infllm2_select_workspace_bytes(vl, h_kv, p)) return INFLLM2_ERR_WORKSPACE_TOO_SMALL;
+    S = static_cast<float*>(workspace);
+  }
+  const int64_t ld = infllm2_scores_ld(vl, p);
+  if ((r = infllm2_shared_scores(Q, K_c1, K_c2, vl, h_q, h_kv, d, S, ld, p, stream))) return r;
+  return infllm2_topk_blocks(S, ld, vl, h_kv, block_idx, p, stream);
+}
+
+int infllm2_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* block_idx,
+                        const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d, void* out, int32_t out_dtype,
+                        const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
+  if (!Q || !K || !V || !block_idx || !out || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+    return INFLLM2_ERR_INVALID_ARG;
+  if (out_dtype != INFLLM2_OUT_BF16 && out_dtype != INFLLM2_OUT_F32) return INFLLM2_ERR_INVALID_ARG;
+  bool map_fail = false;
+  const int n_sel = p->n_init + p->n_local + p->top_k;
+  cudaError_t e = launch_sparse_attn(Q, K, V, block_idx, vl->cu_seqlens, vl->batch, vl->total, h_q, h_kv, d, n_sel,
+                                     softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32,
+                                     static_cast<cudaStream_t>(stream), &map_fail);
+  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_dense_attn(const void* Q, const void* K, const void* V, const infllm2_varlen* vl, int32_t h_q,
+                       int32_t h_kv, int32_t d, void* out, int32_t out_dtype, const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
+  if (!Q || !K || !V || !out || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+    return INFLLM2_ERR_INVALID_ARG;
+  if (out_dtype != INFLLM2_OUT_BF16 && out_dtype != INFLLM2_OUT_F32) return INFLLM2_ERR_INVALID_ARG;
+  bool map_fail = false;
+  cudaError_t e = launch_dense_attn(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d,
+                                    softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32,
+                                    static_cast<cudaStream_t>(stream), &map_fail);
+  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_get_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return v;
+}
+
+int infllm2_clear_device_status(void) {
+  const int zero = 0;
+  cudaError_t e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceSynchronize();
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_debug_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return INFLLM2_ERR_INVALID_ARG;
+  debug_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+}  // extern "C"
