@@ -1,0 +1,374 @@
+#!/usr/bin/env python3
+"""Benchmark of the InfLLM-V2 sparse-attention prefill path on B200.
+
+One step = the whole prefill hot path over one 131072-token sequence
+(h_q=32, h_kv=2, d=128, |I|=96): pool K (stage-1 and coarse windows),
+compressed scores with the LSE approximation and the fused group sum,
+max-pool + top-k block selection, block-sparse attention.  Inputs are
+seeded synthetic tensors (inputs/gen.py), resident in HBM before the timed
+region; the working set (Q 1 GiB, S_shared 4.3 GB) is larger than L2, so no
+extra flush is needed between steps.
+
+Output: one JSON line (rank 0).  `value` is tokens/s over all ranks;
+`e2e` repeats the measurement through the public API with the inputs copied
+from pinned host memory and the output copied back inside the timed region;
+`roofline` describes the dominant kernel; `cpu_baseline` times the fp64
+oracle on a bounded sample of rows on the host cores.
+
+`--impl reference` times the oracle alone (the reference arm for this build:
+there is no installable reference implementation; the pages carry no code).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "128K prefill attn tokens/s (select+sparse) & decode µs/step; % of roofline"
+WORKLOAD = "prefill_128k"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- work counts
+def visible_counts(n: int):
+    """Per query position t of an n-token sequence: visible C1 windows, C2
+    windows and sparse keys (96 blocks of 64; the query's own block is the
+    only partial one)."""
+    t = np.arange(n, dtype=np.int64)
+    n1 = np.where(t >= 31, (t - 31) // 16 + 1, 0)
+    n2 = np.where(t >= 127, (t - 127) // 64 + 1, 0)
+    b_t = t // 64
+    nsel = np.minimum(96, b_t + 1)
+    keys = (nsel - 1) * 64 + (t % 64) + 1
+    return n1, n2, keys
+
+
+def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
+    n1, n2, keys = visible_counts(n)
+    G = h_q // h_kv
+    ld = ((n - 32) // 16 + 1 + 3) // 4 * 4
+    w = {}
+    # compress: read K, write both pooled key sets
+    w["compress_bytes"] = n * h_kv * d * 2 + h_kv * (int(n1[-1]) + int(n2[-1])) * d * 2
+    # scores: 2d flop per (head, token, visible window) for both passes; one exp each
+    w["score_flops"] = 2 * d * h_q * int(n1.sum() + n2.sum())
+    w["score_exps"] = h_q * int(n1.sum() + n2.sum())
+    w["score_bytes"] = n * h_q * d * 2 + 4 * h_kv * int(n1.sum())
+    # top-k: read the visible part of S_shared, write the block lists
+    w["topk_bytes"] = 4 * h_kv * int(n1.sum()) + 4 * h_kv * n * 96
+    # sparse attention: QK^T and PV over the visible selected keys
+    w["sparse_flops"] = 4 * d * h_q * int(keys.sum())
+    w["sparse_exps"] = h_q * int(keys.sum())
+    w["sparse_gather_bytes"] = h_kv * 2 * d * 2 * int(keys.sum())
+    w["ld"] = ld
+    return w
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self):
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        sel = []
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200", *sel],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle baseline
+def oracle_sample(w, data, seconds: float):
+    """Time the fp64 oracle on rows of the workload until ~`seconds` of CPU
+    time: pooling of the whole sequence, then scores, selection and sparse
+    attention for uniformly sampled (token, group) rows.  Returns tokens/s
+    extrapolated to the full sequence, the rows done, and the threads used."""
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    from oracle import infllm2_oracle as O
+    p = O.Params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+    t0 = time.perf_counter()
+    seq = O.Sequence1(O.to_f64(data["Q"]), O.to_f64(data["K"]), O.to_f64(data["V"]), p)
+    t_pool = time.perf_counter() - t0
+    rng = np.random.default_rng(123)
+    n = seq.n
+    rows = 0
+    t1 = time.perf_counter()
+    while time.perf_counter() - t1 < seconds:
+        t = int(rng.integers(0, n))
+        g = int(rng.integers(0, seq.h_kv))
+        sel = seq.select(t, g)
+        seq.sparse_out(t, g, sel)
+        rows += 1
+    t_rows = time.perf_counter() - t1
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    per_row = t_rows / max(rows, 1)
+    total_s = t_pool + per_row * n * seq.h_kv
+    return n / total_s, rows, t_pool + t_rows
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from inputs import gen
+    w = gen.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        data = gen.make_prefill(w)
+        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds / max(1, args.steps) * args.steps)
+        line = {
+            "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.seqlen / tok_s,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q,
+                                             "h_kv": w.h_kv, "d": w.d, "n_sel": w.n_sel},
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"pooling of the whole sequence + {rows} sampled (token, group) rows, "
+                                       f"{secs:.1f} s, extrapolated to all rows"},
+            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import trainable_block_sparse_pool_b200 as T
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    T.lib()
+
+    data = gen.make_prefill(w)
+    p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+    Q, K, V = data["Q"].to(dev), data["K"].to(dev), data["V"].to(dev)
+    cu = data["cu_seqlens"].to(dev)
+    vl = T.make_varlen(data["lens"], cu, p)
+    Kc1 = torch.empty(w.h_kv, vl.total_c1, w.d, dtype=torch.bfloat16, device=dev)
+    Kc2 = torch.empty(w.h_kv, vl.total_c2, w.d, dtype=torch.bfloat16, device=dev)
+    ld = T.infllm2_scores_ld(vl, p)
+    S = torch.empty(w.h_kv, vl.total, ld, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.h_kv, vl.total, p.n_sel, dtype=torch.int32, device=dev)
+    out = torch.empty(vl.total, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    kernels = ["compress", "scores", "topk", "sparse"]
+
+    def step(ev=None):
+        if ev is not None: ev[0].record(stream)
+        T.infllm2_compress_k(K, vl, Kc1, Kc2, p, stream)
+        if ev is not None: ev[1].record(stream)
+        T.infllm2_shared_scores(Q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
+        if ev is not None: ev[2].record(stream)
+        T.infllm2_topk_blocks(S, ld, vl, w.h_kv, idx, p, stream)
+        if ev is not None: ev[3].record(stream)
+        T.infllm2_sparse_attn(Q, K, V, idx, vl, out, p, stream)
+        if ev is not None: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if T.infllm2_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up: %d" % T.infllm2_get_device_status())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, nm in enumerate(kernels)}
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    tokens = w.seqlen * world
+    value = tokens / (ms_per_step / 1e3)
+    status = T.infllm2_get_device_status()
+
+    # ---- e2e through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Qh, Kh, Vh = data["Q"].pin_memory(), data["K"].pin_memory(), data["V"].pin_memory()
+        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            Q.copy_(Qh, non_blocking=True); K.copy_(Kh, non_blocking=True); V.copy_(Vh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / args.steps
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
+        d2h = outh.numel() * outh.element_size()
+        e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    # ---- roofline of the dominant kernel
+    hbm, tflops, tflops_sus, src = _peaks()
+    work = algorithmic_work(w.seqlen, w.h_q, w.h_kv, w.d)
+    dom = max(per_kernel, key=per_kernel.get)
+    if dom == "sparse":
+        ach = work["sparse_flops"] / (per_kernel["sparse"] / 1e3) / 1e12
+        roof = {"kernel": "sparse_attn", "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
+                "frac": ach / tflops, "traffic": None, "peak_source": f"{src} bf16 burst"}
+    elif dom == "scores":
+        ach = work["score_flops"] / (per_kernel["scores"] / 1e3) / 1e12
+        roof = {"kernel": "shared_scores", "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
+                "frac": ach / tflops, "traffic": None, "peak_source": f"{src} bf16 burst"}
+    else:
+        b = work[f"{dom}_bytes"]
+        ach = b / (per_kernel[dom] / 1e3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": None, "peak_source": f"{src} HBM copy"}
+
+    kern_detail = {}
+    for nm in kernels:
+        ms = per_kernel[nm]
+        d_ = {"ms": ms}
+        if nm == "compress":
+            d_["GB/s"] = work["compress_bytes"] / (ms / 1e3) / 1e9
+        elif nm == "scores":
+            d_["TFLOP/s"] = work["score_flops"] / (ms / 1e3) / 1e12
+            d_["Gexp/s"] = work["score_exps"] / (ms / 1e3) / 1e9
+        elif nm == "topk":
+            d_["GB/s"] = work["topk_bytes"] / (ms / 1e3) / 1e9
+        elif nm == "sparse":
+            d_["TFLOP/s"] = work["sparse_flops"] / (ms / 1e3) / 1e12
+            d_["gather_GB/s"] = work["sparse_gather_bytes"] / (ms / 1e3) / 1e9
+        kern_detail[nm] = d_
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q,V; K with per-block offsets)",
+        "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
+                   "n_sel": w.n_sel, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "working set larger than L2 (Q 1 GiB, S_shared 4.3 GB); no extra flush"},
+        "e2e": e2e,
+        "gpu_launches": len(kernels) * args.steps,
+        "kernels": kern_detail,
+        "roofline": roof,
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"pooling of the whole 128K sequence + {rows} uniformly sampled "
+                                          f"(token, group) rows ({secs:.1f} s), extrapolated to all rows"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

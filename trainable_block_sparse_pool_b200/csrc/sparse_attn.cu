@@ -7,31 +7,36 @@
 // unit is too small for the M dimension of tcgen05 (64 or 128), so the
 // contractions are transposed ("swap AB"): keys fill M, heads fill N.
 //   S^T [128 keys, 16] = K_pair[128, d]  . Q_t[16, d]^T      (M=128, N=16)
-//   O^T [d, 16]       = V_pair[128, d]^T . P^T[128, 16]      (M=d,   N=16)
-// A "pair" is two selected blocks side by side in shared memory (each
-// loaded by TMA straight from K / V — the gather is the TMA coordinate).
-// Softmax: one thread per key lane holds the 16 head scores of its key;
-// the per-head maximum over the 128 keys is a shuffle + shared-memory
-// reduction; each thread keeps partial row sums and every thread holds the
-// running maxima, so the rescale factors are known everywhere.  P goes to
-// shared memory as bf16 in the no-swizzle MN-major core-matrix layout.  The
-// PV product of each pair lands in a fresh TMEM accumulator and is folded
-// into registers (O = O * alpha + O_pair) by the thread that owns that row
-// of d, so TMEM never needs an in-place rescale.
+//   O^T [d, 16]      += V_pair[128, d]^T . P^T[128, 16]      (M=d,   N=16)
+// A "pair" is two selected blocks side by side in shared memory, each
+// loaded by TMA straight from K / V (the gather is the TMA coordinate).
+//
+// Throughput comes from keeping the per-tile critical path short:
+//  * O accumulates in TMEM across the unit's tiles.  The softmax uses a
+//    per-head reference maximum m_ref that is only raised when a score
+//    exceeds it by more than 2^8 (then O and the partial row sums are
+//    rescaled once); otherwise P = 2^(x - m_ref) <= 2^8 is exact enough in
+//    bf16/fp32, so the common tile needs no cross-thread maximum, and no
+//    round trip through the PV product.
+//  * The rescale decision is one `bar.red.or` over the warpgroup.
+//  * Two softmax warpgroups work on alternating units of the CTA, so one
+//    group's waits overlap the other's work; the TMA producer and the MMA
+//    issuer interleave the two units' tiles.
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer / TMEM owner,
-// warps 2-5 softmax + correction.  Persistent CTAs, one per SM, take units
-// round-robin (consecutive CTAs work on consecutive tokens of one group, so
-// the group's shared init/local blocks stay hot in L2).
+// warps 2-5 softmax group 0, warps 6-9 softmax group 1.  Persistent CTAs,
+// one per SM, take units round-robin (consecutive CTAs work on consecutive
+// tokens of one group, so the group's init/local blocks stay hot in L2).
 #include "sm100.cuh"
 
 namespace infllm2 {
 
 namespace sparse {
 
-constexpr int kThreads = 192;
-constexpr int kWG = 128;         // softmax / correction threads
-constexpr int kPairKeys = 128;   // keys per tile (two 64-key blocks)
+constexpr int kNumWG = 2;
+constexpr int kThreads = 64 + 128 * kNumWG;
+constexpr int kPairKeys = 128;       // keys per tile (two 64-key blocks)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.f;      // raise m_ref only past this margin (log2 units)
 
 template <int D>
 struct Cfg {
@@ -40,25 +45,25 @@ struct Cfg {
   static constexpr uint32_t kHalf = 64 * 128;                 // one block inside a chunk
   static constexpr uint32_t kKBytes = kChunk * KCH;
   static constexpr uint32_t kStageBytes = 2 * kKBytes;        // K then V
-  static constexpr int kStages = (D == 128) ? 3 : 5;
-  static constexpr uint32_t kQBuf = 16 * 128 * KCH;           // 16 head rows
+  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr uint32_t kQBuf = 2048 * KCH;               // 16 head rows x d
   static constexpr uint32_t kPBuf = kPairKeys * 16 * 2;       // 4 KB
+  static constexpr uint32_t kRed = kNumWG * 4 * 16 * 4;       // per-warp partial maxima / sums
   static constexpr uint32_t kSmem =
-      1024 + kStages * kStageBytes + 2 * kQBuf + 2 * kPBuf + 2 * 4 * 16 * 4 + 4 * 16 * 4 + 512;
+      1024 + kStages * kStageBytes + kNumWG * 2 * kQBuf + kNumWG * 2 * kPBuf + kRed + 512;
 };
 
 struct Bars {
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
-  uint64_t q_full[2];
-  uint64_t q_empty[2];
-  uint64_t s_full[2];
-  uint64_t s_empty[2];
-  uint64_t p_full[2];
-  uint64_t o_full[2];
-  uint64_t o_empty[2];
+  uint64_t q_full[kNumWG][2];
+  uint64_t q_empty[kNumWG][2];
+  uint64_t s_full[kNumWG][2];
+  uint64_t s_empty[kNumWG][2];
+  uint64_t p_full[kNumWG][2];
+  uint64_t pv_done[kNumWG][2];
+  uint64_t o_free[kNumWG][2];
   uint64_t mma_done;
-  uint64_t wg;          // rendezvous of the four softmax warps
   uint32_t tmem_base;
   int abort;
 };
@@ -70,15 +75,30 @@ __device__ __forceinline__ void set_abort(Bars* b) {
   *reinterpret_cast<volatile int*>(&b->abort) = 1;
 }
 
-// Rendezvous of the four softmax warps on an mbarrier (count 4) with a
-// bounded wait, so a warp that gave up cannot leave the others blocked.
-__device__ __forceinline__ bool wg_sync(uint64_t* bar, uint32_t& phase) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase & 1);
-  ++phase;
-  return ok;
+// Barrier over `nthreads` threads on named barrier `id` that also ORs a
+// predicate across them; every participant gets the same result.
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pin, pout;\n\t"
+      "setp.ne.u32 pin, %1, 0;\n\t"
+      "bar.red.or.pred pout, %2, %3, pin;\n\t"
+      "selp.u32 %0, 1, 0, pout;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct Unit {
   int g, t, seq_start, nvalid;
@@ -101,6 +121,8 @@ __device__ __forceinline__ Unit get_unit(int64_t u, const int32_t* cu, int batch
   return x;
 }
 
+__device__ __forceinline__ int ntiles_of(const Unit& x) { return (x.nvalid + 1) >> 1; }
+
 template <int D, int G, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -111,79 +133,95 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem;
-  uint8_t* sQ = sKV + C::kStages * C::kStageBytes;
-  uint8_t* sP = sQ + 2 * C::kQBuf;
-  float* red_max = reinterpret_cast<float*>(sP + 2 * C::kPBuf);  // [2][4][16]
-  float* red_l = red_max + 2 * 4 * 16;                             // [4][16]
-  Bars* bars = reinterpret_cast<Bars*>(red_l + 4 * 16);
+  uint8_t* sQ = sKV + C::kStages * C::kStageBytes;                    // [wg][2]
+  uint8_t* sP = sQ + kNumWG * 2 * C::kQBuf;                           // [wg][2]
+  float* red = reinterpret_cast<float*>(sP + kNumWG * 2 * C::kPBuf);  // [wg][4][16]
+  Bars* bars = reinterpret_cast<Bars*>(red + kNumWG * 4 * 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_units = static_cast<int64_t>(h_kv) * total;
+  // units of this CTA: u_k = blockIdx.x + k * gridDim.x; unit k goes to group k & 1
+  const int64_t my_units = (n_units > blockIdx.x) ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-  // zero both Q buffers so the head rows past G contribute zeros
-  for (int i = threadIdx.x; i < static_cast<int>(2 * C::kQBuf / 16); i += kThreads)
-    reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < static_cast<int>(kNumWG * 2 * C::kQBuf / 16); i += kThreads)
+    reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);   // head rows past G stay zero
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->q_full[i], 1);
-      mbar_init(&bars->q_empty[i], 1);
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_empty[i], 4);
-      mbar_init(&bars->p_full[i], 4);
-      mbar_init(&bars->o_full[i], 1);
-      mbar_init(&bars->o_empty[i], 4);
-    }
+    for (int w = 0; w < kNumWG; ++w)
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bars->q_full[w][i], 1);
+        mbar_init(&bars->q_empty[w][i], 1);
+        mbar_init(&bars->s_full[w][i], 1);
+        mbar_init(&bars->s_empty[w][i], 4);
+        mbar_init(&bars->p_full[w][i], 4);
+        mbar_init(&bars->pv_done[w][i], 1);
+        mbar_init(&bars->o_free[w][i], 4);
+      }
     mbar_init(&bars->mma_done, 1);
-    mbar_init(&bars->wg, 4);
     bars->abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) { tmem_alloc(&bars->tmem_base, 64); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(&bars->tmem_base, 128); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // TMEM columns of group w: S buffers at w*64 + {0,16}, O buffers at w*64 + {32,48}
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
-      int it = 0, qi = 0;
+      int it = 0;
+      int ucnt[kNumWG] = {0, 0};
       bool ok = true;
-      for (int64_t u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++qi) {
-        const Unit x = get_unit(u, cu, batch, total, block_idx, n_sel);
-        const int qb = qi & 1;
-        if (!mbar_wait(&bars->q_empty[qb], ((qi >> 1) & 1) ^ 1)) { set_abort(bars); break; }
-        mbar_arrive_expect_tx(&bars->q_full[qb], C::KCH * G * 128);
-        for (int ch = 0; ch < C::KCH; ++ch)
-          tma_load_4d(sQ + qb * C::kQBuf + ch * 2048, &tmQ, &bars->q_full[qb], ch * 64, 0, x.g,
-                      static_cast<int>(x.row));
-        const int ntile = (x.nvalid + 1) >> 1;
-        for (int i = 0; i < ntile; ++i, ++it) {
-          const int st = it % C::kStages;
-          if (!mbar_wait(&bars->kv_empty[st], ((it / C::kStages) & 1) ^ 1) || aborted(bars)) {
-            set_abort(bars); ok = false; break;
-          }
-          const int b0 = x.I[2 * i];
-          const int b1 = (2 * i + 1 < x.nvalid) ? x.I[2 * i + 1] : b0;   // odd count: reload, masked later
-          uint8_t* dK = sKV + st * C::kStageBytes;
-          uint8_t* dV = dK + C::kKBytes;
-          mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
-          for (int ch = 0; ch < C::KCH; ++ch) {
-            tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, x.g, x.seq_start + 64 * b0);
-            tma_load_3d(dK + ch * C::kChunk + C::kHalf, &tmK, &bars->kv_full[st], ch * 64, x.g,
-                        x.seq_start + 64 * b1);
-            tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, x.g, x.seq_start + 64 * b0);
-            tma_load_3d(dV + ch * C::kChunk + C::kHalf, &tmV, &bars->kv_full[st], ch * 64, x.g,
-                        x.seq_start + 64 * b1);
+      for (int64_t k0 = 0; ok && k0 < my_units; k0 += kNumWG) {
+        Unit x[kNumWG];
+        int nt[kNumWG];
+        for (int w = 0; w < kNumWG; ++w) {
+          nt[w] = 0;
+          if (k0 + w >= my_units) continue;
+          x[w] = get_unit(blockIdx.x + (k0 + w) * gridDim.x, cu, batch, total, block_idx, n_sel);
+          nt[w] = ntiles_of(x[w]);
+          const int qb = ucnt[w] & 1;
+          if (!mbar_wait(&bars->q_empty[w][qb], ((ucnt[w] >> 1) & 1) ^ 1)) { set_abort(bars); ok = false; break; }
+          mbar_arrive_expect_tx(&bars->q_full[w][qb], C::KCH * G * 128);
+          for (int ch = 0; ch < C::KCH; ++ch)
+            tma_load_4d(sQ + (w * 2 + qb) * C::kQBuf + ch * 2048, &tmQ, &bars->q_full[w][qb], ch * 64, 0, x[w].g,
+                        static_cast<int>(x[w].row));
+          ++ucnt[w];
+        }
+        const int nmax = max(nt[0], nt[1]);
+        for (int j = 0; ok && j < nmax; ++j) {
+          for (int w = 0; w < kNumWG; ++w) {
+            if (j >= nt[w]) continue;
+            const int st = it % C::kStages;
+            if (!mbar_wait(&bars->kv_empty[st], ((it / C::kStages) & 1) ^ 1) || aborted(bars)) {
+              set_abort(bars); ok = false; break;
+            }
+            const int b0 = x[w].I[2 * j];
+            const int b1 = (2 * j + 1 < x[w].nvalid) ? x[w].I[2 * j + 1] : b0;   // odd count: reload, masked
+            uint8_t* dK = sKV + st * C::kStageBytes;
+            uint8_t* dV = dK + C::kKBytes;
+            mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
+            for (int ch = 0; ch < C::KCH; ++ch) {
+              tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
+              tma_load_3d(dK + ch * C::kChunk + C::kHalf, &tmK, &bars->kv_full[st], ch * 64, x[w].g,
+                          x[w].seq_start + 64 * b1);
+              tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
+              tma_load_3d(dV + ch * C::kChunk + C::kHalf, &tmV, &bars->kv_full[st], ch * 64, x[w].g,
+                          x[w].seq_start + 64 * b1);
+            }
+            ++it;
           }
         }
       }
       // wait for every copy still in flight before the CTA may exit
-      for (int i = max(0, it - C::kStages); i < it; ++i) mbar_wait(&bars->kv_full[i % C::kStages], (i / C::kStages) & 1);
-      for (int i = max(0, qi - 2); i < qi; ++i) mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1);
+      for (int i = max(0, it - C::kStages); i < it; ++i)
+        mbar_wait(&bars->kv_full[i % C::kStages], (i / C::kStages) & 1);
+      for (int w = 0; w < kNumWG; ++w)
+        for (int i = max(0, ucnt[w] - 2); i < ucnt[w]; ++i) mbar_wait(&bars->q_full[w][i & 1], (i >> 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -191,173 +229,221 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       const uint32_t idS = idesc_bf16_f32(128, 16, 0, 0);
       const uint32_t idO = idesc_bf16_f32(128, 16, 1, 1);
       const uint32_t lboV = (D == 128) ? C::kChunk : 0u;   // d = 64: rows 64-127 of O^T repeat 0-63
-      int it = 0, qi = 0;
+      int it = 0;
+      int tcnt[kNumWG] = {0, 0}, ucnt[kNumWG] = {0, 0};
       bool ok = true;
-      auto issue_pv = [&](int j) -> bool {
-        const int pb = j & 1;
-        const int st = j % C::kStages;
-        if (!mbar_wait(&bars->p_full[pb], (j >> 1) & 1)) return false;
-        if (!mbar_wait(&bars->o_empty[pb], ((j >> 1) & 1) ^ 1)) return false;
+      // the PV product waiting for the softmax of its tile
+      struct Pend { int w, tile, st, obuf; bool first, valid; } pend = {0, 0, 0, 0, false, false};
+      auto issue_pv = [&](const Pend& q) -> bool {
+        const int pb = q.tile & 1;
+        if (!mbar_wait(&bars->p_full[q.w][pb], (q.tile >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(sKV + st * C::kStageBytes + C::kKBytes);
-        const uint32_t p_base = smem_u32(sP + pb * C::kPBuf);
+        const uint32_t v_base = smem_u32(sKV + q.st * C::kStageBytes + C::kKBytes);
+        const uint32_t p_base = smem_u32(sP + (q.w * 2 + pb) * C::kPBuf);
+        const uint32_t o_addr = tmem + q.w * 64 + 32 + q.obuf * 16;
 #pragma unroll
         for (int k = 0; k < kPairKeys / 16; ++k) {
           const uint64_t a = make_sdesc(v_base + k * 2048, lboV, 1024, kLayoutSW128);
           const uint64_t b = make_sdesc(p_base + k * 512, 256, 128, kLayoutNone);
-          umma_bf16(tmem + 32 + pb * 16, a, b, idO, k > 0);
+          umma_bf16(o_addr, a, b, idO, (q.first && k == 0) ? 0u : 1u);
         }
-        umma_commit(&bars->kv_empty[st]);
-        umma_commit(&bars->o_full[pb]);
+        umma_commit(&bars->kv_empty[q.st]);
+        umma_commit(&bars->pv_done[q.w][pb]);
         return true;
       };
-      for (int64_t u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++qi) {
-        const Unit x = get_unit(u, cu, batch, total, block_idx, n_sel);
-        const int qb = qi & 1;
-        if (!mbar_wait(&bars->q_full[qb], (qi >> 1) & 1)) { set_abort(bars); break; }
-        const uint32_t q_base = smem_u32(sQ + qb * C::kQBuf);
-        const int ntile = (x.nvalid + 1) >> 1;
-        for (int i = 0; i < ntile; ++i, ++it) {
-          const int st = it % C::kStages;
-          const int sb = it & 1;
-          if (!mbar_wait(&bars->kv_full[st], (it / C::kStages) & 1) ||
-              !mbar_wait(&bars->s_empty[sb], ((it >> 1) & 1) ^ 1) || aborted(bars)) {
+      for (int64_t k0 = 0; ok && k0 < my_units; k0 += kNumWG) {
+        int nt[kNumWG], qb[kNumWG], ob[kNumWG];
+        for (int w = 0; w < kNumWG; ++w) {
+          nt[w] = 0;
+          if (k0 + w >= my_units) continue;
+          const Unit x = get_unit(blockIdx.x + (k0 + w) * gridDim.x, cu, batch, total, block_idx, n_sel);
+          nt[w] = ntiles_of(x);
+          qb[w] = ucnt[w] & 1;
+          ob[w] = ucnt[w] & 1;
+          if (!mbar_wait(&bars->q_full[w][qb[w]], (ucnt[w] >> 1) & 1) ||
+              !mbar_wait(&bars->o_free[w][ob[w]], ((ucnt[w] >> 1) & 1) ^ 1)) {
             set_abort(bars); ok = false; break;
           }
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(sKV + st * C::kStageBytes);
+          if (nt[w] == 0) umma_commit(&bars->q_empty[w][qb[w]]);   // an empty block list: Q is free at once
+          ++ucnt[w];
+        }
+        const int nmax = max(nt[0], nt[1]);
+        for (int j = 0; ok && j < nmax; ++j) {
+          for (int w = 0; w < kNumWG; ++w) {
+            if (j >= nt[w]) continue;
+            const int st = it % C::kStages;
+            const int sb = tcnt[w] & 1;
+            if (!mbar_wait(&bars->kv_full[st], (it / C::kStages) & 1) ||
+                !mbar_wait(&bars->s_empty[w][sb], ((tcnt[w] >> 1) & 1) ^ 1) || aborted(bars)) {
+              set_abort(bars); ok = false; break;
+            }
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(sKV + st * C::kStageBytes);
+            const uint32_t q_base = smem_u32(sQ + (w * 2 + qb[w]) * C::kQBuf);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t a = make_sdesc(k_base + (k >> 2) * C::kChunk + (k & 3) * 32, 16, 1024, kLayoutSW128);
-            const uint64_t b = make_sdesc(q_base + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024, kLayoutSW128);
-            umma_bf16(tmem + sb * 16, a, b, idS, k > 0);
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t a = make_sdesc(k_base + (k >> 2) * C::kChunk + (k & 3) * 32, 16, 1024, kLayoutSW128);
+              const uint64_t b = make_sdesc(q_base + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024, kLayoutSW128);
+              umma_bf16(tmem + w * 64 + sb * 16, a, b, idS, k > 0);
+            }
+            umma_commit(&bars->s_full[w][sb]);
+            if (j == nt[w] - 1) umma_commit(&bars->q_empty[w][qb[w]]);
+            if (pend.valid && !issue_pv(pend)) { set_abort(bars); ok = false; break; }
+            pend = {w, tcnt[w], st, ob[w], j == 0, true};
+            ++tcnt[w];
+            ++it;
           }
-          umma_commit(&bars->s_full[sb]);
-          if (i == ntile - 1) umma_commit(&bars->q_empty[qb]);
-          if (it > 0 && !issue_pv(it - 1)) { set_abort(bars); ok = false; ++it; break; }
         }
       }
-      if (ok && it > 0 && !issue_pv(it - 1)) set_abort(bars);
+      if (ok && pend.valid && !issue_pv(pend)) set_abort(bars);
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax + correction
+    // ------------------------------------------------------------ softmax groups
+    const int w = (warp - 2) >> 2;           // softmax group
     const int wq = warp & 3;                 // TMEM lane quadrant of this warp
-    const int kl = wq * 32 + lane;           // key lane (softmax) / d row (correction)
+    const int kl = wq * 32 + lane;           // key lane (softmax) / d row (output)
+    const int bar_id = 1 + w;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem + w * 64;
+    const uint32_t t_o = tmem + w * 64 + 32;
+    float* red_w = red + w * 64;
     const float c = scale * kLog2e;
-    uint32_t wg_phase = 0;
-    int it = 0;
-    for (int64_t u = blockIdx.x; u < n_units && !aborted(bars); u += gridDim.x) {
-      const Unit x = get_unit(u, cu, batch, total, block_idx, n_sel);
-      float m_run[16], l_part[16], o_acc[16];
+    int tcnt = 0, ucnt = 0;
+    bool stop = false;
+    for (int64_t k = w; !stop && k < my_units; k += kNumWG, ++ucnt) {
+      const Unit x = get_unit(blockIdx.x + k * gridDim.x, cu, batch, total, block_idx, n_sel);
+      const int nt = ntiles_of(x);
+      const int obuf = ucnt & 1;
+      float m_ref[16], l_part[16];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) { m_run[h] = -INFINITY; l_part[h] = 0.f; o_acc[h] = 0.f; }
-      const int ntile = (x.nvalid + 1) >> 1;
-      bool ok = true;
-      for (int i = 0; i < ntile; ++i, ++it) {
-        const int sb = it & 1;
-        // ---- softmax of tile it
-        if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
+      for (int h = 0; h < 16; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
+      for (int j = 0; j < nt; ++j, ++tcnt) {
+        const int sb = tcnt & 1;
+        bool ab = !mbar_wait(&bars->s_full[w][sb], (tcnt >> 1) & 1);
+        if (ab) set_abort(bars);
         tc_fence_after();
         float v[16];
-        tmem_ld16(tmem + lane_addr + sb * 16, v);
+        tmem_ld16(t_s + lane_addr + sb * 16, v);
         tmem_wait_ld16(v);
-        const int half = kl >> 6;
-        const int bsel = 2 * i + half;
+        const int bsel = 2 * j + (kl >> 6);
         const int blk = (bsel < x.nvalid) ? x.I[bsel] : -1;
         const int pos = 64 * blk + (kl & 63);
         const bool valid = (blk >= 0) && (pos <= x.t);
-        float mx[16];
+        bool exceed = false;
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
           v[h] = valid ? v[h] * c : -INFINITY;
-          mx[h] = v[h];
+          exceed |= v[h] > m_ref[h] + kRescale;
         }
+        ab = ab || aborted(bars);
+        if (bar_red_or(bar_id, 128, exceed || ab)) {
+          if (bar_red_or(bar_id, 128, ab)) { stop = true; break; }
+          // raise the reference maxima: full per-head maximum over the 128 keys
+          float mx[16];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
+          for (int h = 0; h < 16; ++h) {
+            mx[h] = v[h];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
+            for (int o = 16; o > 0; o >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
+          }
+          if (lane < 16) {
+            float mine = mx[0];
+#pragma unroll
+            for (int h = 1; h < 16; ++h) if (lane == h) mine = mx[h];
+            red_w[wq * 16 + lane] = mine;
+          }
+          named_bar_sync(bar_id, 128);
+          float alpha[16];
+          bool any_scale = false;
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            const float tmax = fmaxf(fmaxf(red_w[h], red_w[16 + h]), fmaxf(red_w[32 + h], red_w[48 + h]));
+            const float m_new = fmaxf(m_ref[h], tmax);
+            alpha[h] = (m_ref[h] == -INFINITY) ? 0.f : ex2(m_ref[h] - m_new);
+            any_scale |= (m_ref[h] != -INFINITY) && (m_new > m_ref[h]);
+            m_ref[h] = m_new;
+            l_part[h] *= alpha[h];
+          }
+          named_bar_sync(bar_id, 128);   // red_w is read by everyone before it is reused
+          if (j > 0 && any_scale) {
+            // rescale O in TMEM once every PV of this unit so far is done
+            const int prev = tcnt - 1;
+            const bool okw = mbar_wait(&bars->pv_done[w][prev & 1], (prev >> 1) & 1);
+            if (!okw) set_abort(bars);
+            tc_fence_after();
+            float o[16];
+            tmem_ld16(t_o + lane_addr + obuf * 16, o);
+            tmem_wait_ld16(o);
+#pragma unroll
+            for (int h = 0; h < 16; ++h) o[h] *= alpha[h];
+            tmem_st16(t_o + lane_addr + obuf * 16, o);
+            tmem_wait_st();
+          }
         }
-        float* rm = red_max + (it & 1) * 64;
-        if (lane < 16) {
-          float mine = mx[0];
-#pragma unroll
-          for (int h = 1; h < 16; ++h) if (lane == h) mine = mx[h];
-          rm[wq * 16 + lane] = mine;
-        }
-        if (!wg_sync(&bars->wg, wg_phase)) { set_abort(bars); ok = false; ++it; break; }
-        float alpha[16];
+        // P buffer sb was last read by the PV of tile tcnt-2
+        if (tcnt >= 2 && !mbar_wait(&bars->pv_done[w][sb], ((tcnt - 2) >> 1) & 1)) set_abort(bars);
         uint32_t pk[8];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          const float tmax = fmaxf(fmaxf(rm[h], rm[16 + h]), fmaxf(rm[32 + h], rm[48 + h]));
-          const float m_new = fmaxf(m_run[h], tmax);
-          const bool none = (m_new == -INFINITY);
-          alpha[h] = none ? 1.f : ex2(m_run[h] - m_new);
-          const float p = none ? 0.f : ex2(v[h] - m_new);
-          l_part[h] = l_part[h] * alpha[h] + p;
-          m_run[h] = m_new;
-          v[h] = p;
+        for (int h = 0; h < 16; h += 2) {
+          const float p0 = ex2(v[h] - m_ref[h]);
+          const float p1 = ex2(v[h + 1] - m_ref[h + 1]);
+          l_part[h] += p0;
+          l_part[h + 1] += p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[h >> 1] = *reinterpret_cast<uint32_t*>(&b2);
         }
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * h], v[2 * h + 1]);
-          pk[h] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        uint8_t* pbuf = sP + sb * C::kPBuf;
+        uint8_t* pbuf = sP + (w * 2 + sb) * C::kPBuf;
         const uint32_t poff = (kl >> 3) * 256 + (kl & 7) * 16;
         *reinterpret_cast<uint4*>(pbuf + poff) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4*>(pbuf + poff + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) { mbar_arrive(&bars->p_full[sb]); mbar_arrive(&bars->s_empty[sb]); }
-        // ---- correction: fold this tile's P.V into the register accumulator
-        if (!mbar_wait(&bars->o_full[sb], (it >> 1) & 1)) { set_abort(bars); ok = false; ++it; break; }
-        tc_fence_after();
-        float ov[16];
-        tmem_ld16(tmem + lane_addr + 32 + sb * 16, ov);
-        tmem_wait_ld16(ov);
-#pragma unroll
-        for (int h = 0; h < 16; ++h) o_acc[h] = fmaf(o_acc[h], alpha[h], ov[h]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->o_empty[sb]);
+        if (lane == 0) { mbar_arrive(&bars->p_full[w][sb]); mbar_arrive(&bars->s_empty[w][sb]); }
       }
-      if (!ok) break;
-      // ---- row sums over the 128 key lanes, then the normalised output
+      if (stop) break;
+      // ---- unit done: wait for its last PV, reduce the row sums, write out
+      bool ab = (nt > 0) && !mbar_wait(&bars->pv_done[w][(tcnt - 1) & 1], ((tcnt - 1) >> 1) & 1);
+      if (ab) set_abort(bars);
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(t_o + lane_addr + obuf * 16, o);
+      tmem_wait_ld16(o);
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], o);
+        for (int s2 = 16; s2 > 0; s2 >>= 1) l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], s2);
       }
       if (lane < 16) {
         float mine = l_part[0];
 #pragma unroll
         for (int h = 1; h < 16; ++h) if (lane == h) mine = l_part[h];
-        red_l[wq * 16 + lane] = mine;
+        red_w[wq * 16 + lane] = mine;
       }
-      if (!wg_sync(&bars->wg, wg_phase)) { set_abort(bars); break; }
+      ab = ab || aborted(bars);
+      if (bar_red_or(bar_id, 128, ab)) { stop = true; break; }
       if (kl < D) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float l = red_l[h] + red_l[16 + h] + red_l[32 + h] + red_l[48 + h];
-          const float o = (l > 0.f) ? o_acc[h] / l : 0.f;
+          const float l = red_w[h] + red_w[16 + h] + red_w[32 + h] + red_w[48 + h];
+          const float r = (l > 0.f) ? o[h] / l : 0.f;
           const int64_t idx = (x.row * h_q + static_cast<int64_t>(x.g) * G + h) * D + kl;
-          if (OUT_F32) reinterpret_cast<float*>(out)[idx] = o;
-          else reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(o);
+          if (OUT_F32) reinterpret_cast<float*>(out)[idx] = r;
+          else reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(r);
         }
       }
-      if (!wg_sync(&bars->wg, wg_phase)) { set_abort(bars); break; }   // red_l is reused by the next unit
+      tc_fence_before();
+      named_bar_sync(bar_id, 128);           // red_w and this O buffer are free again
+      if (lane == 0) mbar_arrive(&bars->o_free[w][obuf]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 64);
+  if (warp == 1) tmem_dealloc(tmem, 128);
 }
 
 }  // namespace sparse
@@ -390,7 +476,7 @@ static cudaError_t launch_sparse_t(const void* Q, const void* K, const void* V, 
   if (e != cudaSuccess) return e;
   const int64_t units = static_cast<int64_t>(h_kv) * total;
   if (units == 0) return cudaSuccess;
-  const int64_t grid = std::min<int64_t>(units, num_sms());
+  const int64_t grid = std::min<int64_t>((units + 1) / 2, num_sms());
   kern<<<static_cast<unsigned>(grid), sparse::kThreads, C::kSmem, st>>>(mQ, mK, mV, idx, cu, batch, total, h_q,
                                                                         h_kv, n_sel, scale, out);
   return cudaGetLastError();
