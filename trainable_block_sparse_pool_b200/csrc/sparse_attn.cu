@@ -100,6 +100,48 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Number of valid (>= 0) entries of a block list, with independent vector
+// loads (lists hold their valid entries first, then -1 padding).
+__device__ __forceinline__ int count_valid(const int32_t* I, int n_sel) {
+  int nv = 0;
+  if ((n_sel & 3) == 0 && (reinterpret_cast<uintptr_t>(I) & 15) == 0) {
+    const int4* I4 = reinterpret_cast<const int4*>(I);
+#pragma unroll 8
+    for (int i = 0; i < n_sel / 4; ++i) {
+      const int4 v = __ldg(I4 + i);
+      nv += (v.x >= 0) + (v.y >= 0) + (v.z >= 0) + (v.w >= 0);
+    }
+  } else {
+    for (int i = 0; i < n_sel; ++i) nv += (__ldg(I + i) >= 0);
+  }
+  return nv;
+}
+
+// Block list entries in registers: lane l of a warp holds entries
+// base + 2*(l + 32*r) + half for r = 0, 1 (tiles j = l + 32 r), so tile j's
+// block is shfl(reg[j >> 5], j & 31).  Lists longer than 128 entries are
+// read from global memory instead.
+struct WarpList {
+  int r0, r1;
+};
+__device__ __forceinline__ WarpList load_warp_list(const int32_t* I, int nvalid, int half, int lane) {
+  WarpList L;
+  const int e0 = 2 * lane + half, e1 = 2 * (lane + 32) + half;
+  L.r0 = (e0 < nvalid) ? __ldg(I + e0) : -1;
+  L.r1 = (e1 < nvalid) ? __ldg(I + e1) : -1;
+  return L;
+}
+__device__ __forceinline__ int warp_list_get(const WarpList& L, const int32_t* I, int nvalid, int n_sel, int j,
+                                             int half) {
+  if (n_sel <= 128) {
+    const int v0 = __shfl_sync(0xffffffffu, L.r0, j & 31);
+    const int v1 = __shfl_sync(0xffffffffu, L.r1, j & 31);
+    return (j < 32) ? v0 : v1;
+  }
+  const int e = 2 * j + half;
+  return (e < nvalid) ? __ldg(I + e) : -1;
+}
+
 struct Unit {
   int g, t, seq_start, nvalid;
   int64_t row;
@@ -115,9 +157,7 @@ __device__ __forceinline__ Unit get_unit(int64_t u, const int32_t* cu, int batch
   x.seq_start = cu[s];
   x.t = static_cast<int>(x.row - x.seq_start);
   x.I = block_idx + u * n_sel;
-  int nv = 0;
-  while (nv < n_sel && x.I[nv] >= 0) ++nv;
-  x.nvalid = nv;
+  x.nvalid = count_valid(x.I, n_sel);
   return x;
 }
 
@@ -171,53 +211,73 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
-      int it = 0;
-      int ucnt[kNumWG] = {0, 0};
-      bool ok = true;
-      for (int64_t k0 = 0; ok && k0 < my_units; k0 += kNumWG) {
-        Unit x[kNumWG];
-        int nt[kNumWG];
-        for (int w = 0; w < kNumWG; ++w) {
-          nt[w] = 0;
-          if (k0 + w >= my_units) continue;
-          x[w] = get_unit(blockIdx.x + (k0 + w) * gridDim.x, cu, batch, total, block_idx, n_sel);
-          nt[w] = ntiles_of(x[w]);
-          const int qb = ucnt[w] & 1;
-          if (!mbar_wait(&bars->q_empty[w][qb], ((ucnt[w] >> 1) & 1) ^ 1)) { set_abort(bars); ok = false; break; }
-          mbar_arrive_expect_tx(&bars->q_full[w][qb], C::KCH * G * 128);
-          for (int ch = 0; ch < C::KCH; ++ch)
-            tma_load_4d(sQ + (w * 2 + qb) * C::kQBuf + ch * 2048, &tmQ, &bars->q_full[w][qb], ch * 64, 0, x[w].g,
-                        static_cast<int>(x[w].row));
-          ++ucnt[w];
-        }
-        const int nmax = max(nt[0], nt[1]);
-        for (int j = 0; ok && j < nmax; ++j) {
-          for (int w = 0; w < kNumWG; ++w) {
-            if (j >= nt[w]) continue;
-            const int st = it % C::kStages;
-            if (!mbar_wait(&bars->kv_empty[st], ((it / C::kStages) & 1) ^ 1) || aborted(bars)) {
-              set_abort(bars); ok = false; break;
-            }
-            const int b0 = x[w].I[2 * j];
-            const int b1 = (2 * j + 1 < x[w].nvalid) ? x[w].I[2 * j + 1] : b0;   // odd count: reload, masked
-            uint8_t* dK = sKV + st * C::kStageBytes;
-            uint8_t* dV = dK + C::kKBytes;
-            mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
-            for (int ch = 0; ch < C::KCH; ++ch) {
-              tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
-              tma_load_3d(dK + ch * C::kChunk + C::kHalf, &tmK, &bars->kv_full[st], ch * 64, x[w].g,
-                          x[w].seq_start + 64 * b1);
-              tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
-              tma_load_3d(dV + ch * C::kChunk + C::kHalf, &tmV, &bars->kv_full[st], ch * 64, x[w].g,
-                          x[w].seq_start + 64 * b1);
-            }
-            ++it;
+    // The whole warp walks the units (their block lists live in its
+    // registers); lane 0 waits and issues the copies.
+    if (lane == 0) { tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV); }
+    int it = 0;
+    int ucnt[kNumWG] = {0, 0};
+    bool ok = true;
+    for (int64_t k0 = 0; ok && k0 < my_units; k0 += kNumWG) {
+      Unit x[kNumWG];
+      WarpList Le[kNumWG], Lo[kNumWG];
+      int nt[kNumWG];
+      for (int w = 0; w < kNumWG; ++w) {
+        nt[w] = 0;
+        if (k0 + w >= my_units) continue;
+        x[w] = get_unit(blockIdx.x + (k0 + w) * gridDim.x, cu, batch, total, block_idx, n_sel);
+        nt[w] = ntiles_of(x[w]);
+        Le[w] = load_warp_list(x[w].I, x[w].nvalid, 0, lane);
+        Lo[w] = load_warp_list(x[w].I, x[w].nvalid, 1, lane);
+        const int qb = ucnt[w] & 1;
+        int good = 1;
+        if (lane == 0) {
+          good = mbar_wait(&bars->q_empty[w][qb], ((ucnt[w] >> 1) & 1) ^ 1);
+          if (good) {
+            mbar_arrive_expect_tx(&bars->q_full[w][qb], C::KCH * G * 128);
+            for (int ch = 0; ch < C::KCH; ++ch)
+              tma_load_4d(sQ + (w * 2 + qb) * C::kQBuf + ch * 2048, &tmQ, &bars->q_full[w][qb], ch * 64, 0,
+                          x[w].g, static_cast<int>(x[w].row));
+          } else {
+            set_abort(bars);
           }
         }
+        if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+        ++ucnt[w];
       }
-      // wait for every copy still in flight before the CTA may exit
+      const int nmax = max(nt[0], nt[1]);
+      for (int j = 0; ok && j < nmax; ++j) {
+        for (int w = 0; w < kNumWG; ++w) {
+          if (j >= nt[w]) continue;
+          const int b0 = warp_list_get(Le[w], x[w].I, x[w].nvalid, n_sel, j, 0);
+          int b1 = warp_list_get(Lo[w], x[w].I, x[w].nvalid, n_sel, j, 1);
+          if (b1 < 0) b1 = b0;   // odd count: reload the first block, masked by the softmax
+          const int st = it % C::kStages;
+          int good = 1;
+          if (lane == 0) {
+            good = mbar_wait(&bars->kv_empty[st], ((it / C::kStages) & 1) ^ 1) && !aborted(bars);
+            if (good) {
+              uint8_t* dK = sKV + st * C::kStageBytes;
+              uint8_t* dV = dK + C::kKBytes;
+              mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
+              for (int ch = 0; ch < C::KCH; ++ch) {
+                tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
+                tma_load_3d(dK + ch * C::kChunk + C::kHalf, &tmK, &bars->kv_full[st], ch * 64, x[w].g,
+                            x[w].seq_start + 64 * b1);
+                tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
+                tma_load_3d(dV + ch * C::kChunk + C::kHalf, &tmV, &bars->kv_full[st], ch * 64, x[w].g,
+                            x[w].seq_start + 64 * b1);
+              }
+            } else {
+              set_abort(bars);
+            }
+          }
+          if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+          ++it;
+        }
+      }
+    }
+    // wait for every copy still in flight before the CTA may exit
+    if (lane == 0) {
       for (int i = max(0, it - C::kStages); i < it; ++i)
         mbar_wait(&bars->kv_full[i % C::kStages], (i / C::kStages) & 1);
       for (int w = 0; w < kNumWG; ++w)
@@ -316,6 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       const Unit x = get_unit(blockIdx.x + k * gridDim.x, cu, batch, total, block_idx, n_sel);
       const int nt = ntiles_of(x);
       const int obuf = ucnt & 1;
+      const int half = kl >> 6;              // this warp's keys come from the pair's first or second block
+      const WarpList L = load_warp_list(x.I, x.nvalid, half, lane);
       float m_ref[16], l_part[16];
 #pragma unroll
       for (int h = 0; h < 16; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
@@ -327,8 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         float v[16];
         tmem_ld16(t_s + lane_addr + sb * 16, v);
         tmem_wait_ld16(v);
-        const int bsel = 2 * j + (kl >> 6);
-        const int blk = (bsel < x.nvalid) ? x.I[bsel] : -1;
+        const int blk = warp_list_get(L, x.I, x.nvalid, n_sel, j, half);
         const int pos = 64 * blk + (kl & 63);
         const bool valid = (blk >= 0) && (pos <= x.t);
         bool exceed = false;
