@@ -164,6 +164,30 @@ int infllm2_select_blocks(const void* Q, const void* K_c1, const void* K_c2,
                           void* workspace, size_t workspace_bytes, int32_t* block_idx,
                           float* s_shared_out, const infllm2_params* p, void* stream);
 
+/* Allocation-free variant of infllm2_select_blocks.  The paper has no
+ * counterpart: this is a convenience of this library for callers that cannot
+ * allocate device memory when they select blocks (code running inside a
+ * custom allocator or memory pool, plugins whose host owns every device
+ * allocation, paths that must not call cudaMalloc because it can
+ * synchronise the device).  Same arguments and results as
+ * infllm2_select_blocks, without a workspace: S_shared is kept in a
+ * fixed array of INFLLM2_NOALLOC_SCRATCH_BYTES in the library's device
+ * memory, held on every GPU that loads the library until the process exits.
+ *   - Problems whose S_shared (h_kv * total * ld floats, ld =
+ *     infllm2_scores_ld) exceeds the array return
+ *     INFLLM2_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   - The first call on a device looks up the array's device address for
+ *     that device (cudaGetSymbolAddress); make that first call before
+ *     capturing the stream into a graph.
+ *   - Every call uses the same array: calls whose kernels can overlap on the
+ *     GPU race on it.  It keeps the last call's scores; none of it needs to
+ *     start at zero.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine. */
+#define INFLLM2_NOALLOC_SCRATCH_BYTES (64u << 20)
+int infllm2_select_blocks_noalloc(const void* Q, const void* K_c1, const void* K_c2,
+                                  const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
+                                  int32_t* block_idx, const infllm2_params* p, void* stream);
+
 /* ---------------------------------------------------------------------
  * Step 4: block-sparse causal attention ([blog] "对齐计算图": selected and
  * sliding attention merged into one sparse attention with a single output;

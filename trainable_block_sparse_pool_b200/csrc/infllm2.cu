@@ -265,3 +265,6 @@ int infllm2_debug_wait_timeout(uint64_t limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// Allocation-free variant of infllm2_select_blocks (fixed device scratch).
+#include "noalloc.cu"
