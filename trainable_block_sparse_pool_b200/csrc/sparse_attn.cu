@@ -20,10 +20,12 @@
 //    round trip through the PV product.
 //  * The rescale decision is one `bar.red.or` over the warpgroup.
 //  * Two softmax warpgroups work on alternating units of the CTA, so one
-//    group's waits overlap the other's work; the TMA producer and the MMA
-//    issuer interleave the two units' tiles.
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer / TMEM owner,
-// warps 2-5 softmax group 0, warps 6-9 softmax group 1.  Persistent CTAs,
+//    group's waits overlap the other's work; the TMA producer and the QK
+//    issuer interleave the two units' tiles, and each group has its own PV
+//    issuer, so no issuer blocks on another group's progress.
+// Warp roles: warp 0 TMA producer, warp 1 QK issuer / TMEM owner,
+// warps 2-5 softmax group 0, warps 6-9 softmax group 1, warps 10-11 issue
+// the PV products of groups 0 and 1.  Persistent CTAs,
 // one per SM, take units round-robin (consecutive CTAs work on consecutive
 // tokens of one group, so the group's init/local blocks stay hot in L2).
 #include "sm100.cuh"
@@ -33,7 +35,7 @@ namespace infllm2 {
 namespace sparse {
 
 constexpr int kNumWG = 2;
-constexpr int kThreads = 64 + 128 * kNumWG;
+constexpr int kThreads = 64 + 128 * kNumWG + 32 * kNumWG;   // producer, QK, softmax groups, PV issuers
 constexpr int kPairKeys = 128;       // keys per tile (two 64-key blocks)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.f;      // raise m_ref only past this margin (log2 units)
@@ -63,7 +65,7 @@ struct Bars {
   uint64_t p_full[kNumWG][2];
   uint64_t pv_done[kNumWG][2];
   uint64_t o_free[kNumWG][2];
-  uint64_t mma_done;
+  uint64_t mma_done[1 + kNumWG];
   uint32_t tmem_base;
   int abort;
 };
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         mbar_init(&bars->pv_done[w][i], 1);
         mbar_init(&bars->o_free[w][i], 4);
       }
-    mbar_init(&bars->mma_done, 1);
+    for (int i = 0; i < 1 + kNumWG; ++i) mbar_init(&bars->mma_done[i], 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -284,47 +286,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         for (int i = max(0, ucnt[w] - 2); i < ucnt[w]; ++i) mbar_wait(&bars->q_full[w][i & 1], (i >> 1) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ QK issuer
+    // Walks the stream in order: a QK product goes out as soon as its K/V
+    // stage has landed and its group's S buffer is free.
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 16, 0, 0);
-      const uint32_t idO = idesc_bf16_f32(128, 16, 1, 1);
-      const uint32_t lboV = (D == 128) ? C::kChunk : 0u;   // d = 64: rows 64-127 of O^T repeat 0-63
       int it = 0;
       int tcnt[kNumWG] = {0, 0}, ucnt[kNumWG] = {0, 0};
       bool ok = true;
-      // the PV product waiting for the softmax of its tile
-      struct Pend { int w, tile, st, obuf; bool first, valid; } pend = {0, 0, 0, 0, false, false};
-      auto issue_pv = [&](const Pend& q) -> bool {
-        const int pb = q.tile & 1;
-        if (!mbar_wait(&bars->p_full[q.w][pb], (q.tile >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(sKV + q.st * C::kStageBytes + C::kKBytes);
-        const uint32_t p_base = smem_u32(sP + (q.w * 2 + pb) * C::kPBuf);
-        const uint32_t o_addr = tmem + q.w * 64 + 32 + q.obuf * 16;
-#pragma unroll
-        for (int k = 0; k < kPairKeys / 16; ++k) {
-          const uint64_t a = make_sdesc(v_base + k * 2048, lboV, 1024, kLayoutSW128);
-          const uint64_t b = make_sdesc(p_base + k * 512, 256, 128, kLayoutNone);
-          umma_bf16(o_addr, a, b, idO, (q.first && k == 0) ? 0u : 1u);
-        }
-        umma_commit(&bars->kv_empty[q.st]);
-        umma_commit(&bars->pv_done[q.w][pb]);
-        return true;
-      };
       for (int64_t k0 = 0; ok && k0 < my_units; k0 += kNumWG) {
-        int nt[kNumWG], qb[kNumWG], ob[kNumWG];
+        int nt[kNumWG], qb[kNumWG];
         for (int w = 0; w < kNumWG; ++w) {
           nt[w] = 0;
           if (k0 + w >= my_units) continue;
           const Unit x = get_unit(blockIdx.x + (k0 + w) * gridDim.x, cu, batch, total, block_idx, n_sel);
           nt[w] = ntiles_of(x);
           qb[w] = ucnt[w] & 1;
-          ob[w] = ucnt[w] & 1;
-          if (!mbar_wait(&bars->q_full[w][qb[w]], (ucnt[w] >> 1) & 1) ||
-              !mbar_wait(&bars->o_free[w][ob[w]], ((ucnt[w] >> 1) & 1) ^ 1)) {
-            set_abort(bars); ok = false; break;
-          }
-          if (nt[w] == 0) umma_commit(&bars->q_empty[w][qb[w]]);   // an empty block list: Q is free at once
+          if (!mbar_wait(&bars->q_full[w][qb[w]], (ucnt[w] >> 1) & 1)) { set_abort(bars); ok = false; break; }
+          if (nt[w] == 0) umma_commit(&bars->q_empty[w][qb[w]]);   // empty list: Q is free at once
           ++ucnt[w];
         }
         const int nmax = max(nt[0], nt[1]);
@@ -348,19 +327,71 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
             }
             umma_commit(&bars->s_full[w][sb]);
             if (j == nt[w] - 1) umma_commit(&bars->q_empty[w][qb[w]]);
-            if (pend.valid && !issue_pv(pend)) { set_abort(bars); ok = false; break; }
-            pend = {w, tcnt[w], st, ob[w], j == 0, true};
             ++tcnt[w];
             ++it;
           }
         }
       }
-      if (ok && pend.valid && !issue_pv(pend)) set_abort(bars);
-      umma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0);
+      umma_commit(&bars->mma_done[0]);
+      mbar_wait(&bars->mma_done[0], 0);
+    }
+  } else if (warp >= 2 + 4 * kNumWG) {
+    // ------------------------------------------------------------ PV issuers
+    // One warp per softmax group: the group's PV products in order, each as
+    // soon as its P is in shared memory.  The stream is replayed to find
+    // which K/V stage each tile occupies.
+    const int pw = warp - (2 + 4 * kNumWG);
+    if (lane == 0) {
+      const uint32_t idO = idesc_bf16_f32(128, 16, 1, 1);
+      const uint32_t lboV = (D == 128) ? C::kChunk : 0u;   // d = 64: rows 64-127 of O^T repeat 0-63
+      int it = 0, tcnt = 0, ucnt = 0;
+      bool ok = true;
+      for (int64_t k0 = 0; ok && k0 < my_units; k0 += kNumWG) {
+        int nt[kNumWG];
+        for (int w = 0; w < kNumWG; ++w) {
+          nt[w] = 0;
+          if (k0 + w >= my_units) continue;
+          const Unit x = get_unit(blockIdx.x + (k0 + w) * gridDim.x, cu, batch, total, block_idx, n_sel);
+          nt[w] = ntiles_of(x);
+        }
+        const bool mine = (k0 + pw < my_units);
+        const int obuf = ucnt & 1;
+        if (mine && nt[pw] > 0 &&
+            !mbar_wait(&bars->o_free[pw][obuf], ((ucnt >> 1) & 1) ^ 1)) { set_abort(bars); ok = false; break; }
+        const int nmax = max(nt[0], nt[1]);
+        for (int j = 0; ok && j < nmax; ++j) {
+          for (int w = 0; w < kNumWG; ++w) {
+            if (j >= nt[w]) continue;
+            if (w == pw) {
+              const int st = it % C::kStages;
+              const int pb = tcnt & 1;
+              if (!mbar_wait(&bars->p_full[pw][pb], (tcnt >> 1) & 1) || aborted(bars)) {
+                set_abort(bars); ok = false; break;
+              }
+              tc_fence_after();
+              const uint32_t v_base = smem_u32(sKV + st * C::kStageBytes + C::kKBytes);
+              const uint32_t p_base = smem_u32(sP + (pw * 2 + pb) * C::kPBuf);
+              const uint32_t o_addr = tmem + pw * 64 + 32 + obuf * 16;
+#pragma unroll
+              for (int k = 0; k < kPairKeys / 16; ++k) {
+                const uint64_t a = make_sdesc(v_base + k * 2048, lboV, 1024, kLayoutSW128);
+                const uint64_t b = make_sdesc(p_base + k * 512, 256, 128, kLayoutNone);
+                umma_bf16(o_addr, a, b, idO, (j == 0 && k == 0) ? 0u : 1u);
+              }
+              umma_commit(&bars->kv_empty[st]);
+              umma_commit(&bars->pv_done[pw][pb]);
+              ++tcnt;
+            }
+            ++it;
+          }
+        }
+        if (mine) ++ucnt;
+      }
+      umma_commit(&bars->mma_done[1 + pw]);
+      mbar_wait(&bars->mma_done[1 + pw], 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax groups
+    // ------------------------------------------------------------ softmax groups (warps 2 .. 2+4*kNumWG-1)
     const int w = (warp - 2) >> 2;           // softmax group
     const int wq = warp & 3;                 // TMEM lane quadrant of this warp
     const int kl = wq * 32 + lane;           // key lane (softmax) / d row (output)
@@ -389,6 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         float v[16];
         tmem_ld16(t_s + lane_addr + sb * 16, v);
         tmem_wait_ld16(v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_empty[w][sb]);   // S is in registers: the buffer is free
         const int blk = warp_list_get(L, x.I, x.nvalid, n_sel, j, half);
         const int pos = 64 * blk + (kl & 63);
         const bool valid = (blk >= 0) && (pos <= x.t);
@@ -462,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) { mbar_arrive(&bars->p_full[w][sb]); mbar_arrive(&bars->s_empty[w][sb]); }
+        if (lane == 0) mbar_arrive(&bars->p_full[w][sb]);
       }
       if (stop) break;
       // ---- unit done: wait for its last PV, reduce the row sums, write out
