@@ -76,8 +76,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = smem + C::kQBytes;
-  float* lse2 = reinterpret_cast<float*>(sK + kStages * C::kStageBytes);
-  Bars* bars = reinterpret_cast<Bars*>(lse2 + 256);
+  float* nlse = reinterpret_cast<float*>(sK + kStages * C::kStageBytes);   // -LSE (log2 units) per Q row
+  Bars* bars = reinterpret_cast<Bars*>(nlse + 256);
   __shared__ int red[32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -196,26 +196,31 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
       const int buf = it & 1;
       if (!mbar_wait(&bars->tfull[buf], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
       tc_fence_after();
-#pragma unroll 1
-      for (int cc = 0; cc < 128; cc += 16) {
-        float v[16];
-        tmem_ld16(tmem + lane_addr + buf * 256 + hh * 128 + cc, v);
-        tmem_wait_ld16(v);
+      const uint32_t tcol = tmem + lane_addr + buf * 256 + hh * 128;
+      float va[32], vb[32];
+      tmem_ld32(tcol, va);
+      tmem_wait_ld32(va);
+#pragma unroll
+      for (int cc = 0; cc < 128; cc += 32) {
+        float (&v)[32] = ((cc >> 5) & 1) ? vb : va;
+        float (&vn)[32] = ((cc >> 5) & 1) ? va : vb;
+        if (cc + 32 < 128) tmem_ld32(tcol + cc + 32, vn);
+        const int m0 = it * kKeysPerTile + cc;
         float mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int m = it * kKeysPerTile + cc + i;
-          v[i] = (m < n2) ? v[i] * c : -INFINITY;
+        for (int i = 0; i < 32; ++i) {
+          v[i] = (m0 + i < n2) ? v[i] * c : -INFINITY;
           mx = fmaxf(mx, v[i]);
         }
         const float m_new = fmaxf(m_run, mx);
         if (m_new != -INFINITY) {
           float acc = 0.f;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc += ex2(v[i] - m_new);
+          for (int i = 0; i < 32; ++i) acc += ex2(v[i] - m_new);
           l_run = l_run * ex2(m_run - m_new) + acc;
           m_run = m_new;
         }
+        if (cc + 32 < 128) tmem_wait_ld32(vn);
       }
       tc_fence_before();
       __syncwarp();
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
       float mm = -INFINITY, ll = 0.f;
       if (t < len) {
         const __nv_bfloat16* qp = Q + (static_cast<int64_t>(row0 + t) * h_q + g * G + h) * D;
-        for (int j = 0; j < n1; ++j) {
+        for (int j = 0; j < n1 && c1_off + j < total_c1; ++j) {
           const __nv_bfloat16* kp = Kc1 + (static_cast<int64_t>(g) * total_c1 + c1_off + j) * D;
           float dot = 0.f;
           for (int e = 0; e < D; ++e) dot += __bfloat162float(qp[e]) * __bfloat162float(kp[e]);
@@ -243,33 +248,53 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
       }
       lse = (n1 > 0) ? mm + log2f(ll) : INFINITY;
     }
-    lse2[r] = lse;
-    named_bar_sync(1, kEpiThreads);
 
     // phase B: this thread owns key j; columns hh*128 .. +128 are tokens
     // hh*TQ/2 .. (hh+1)*TQ/2 - 1, G heads each
+    nlse[r] = -lse;                     // stored negated: exp2(s*c - lse) = ex2(fma(s, c, nlse))
+    named_bar_sync(2, kEpiThreads);
+    const int tt0 = t0 + hh * (TQ / 2);
+    float* srow0 = S + (static_cast<int64_t>(g) * total + row0 + tt0) * ld;
     for (; ok && it < nA + nB; ++it) {
       const int buf = it & 1;
       const int kt = it - nA;
       if (!mbar_wait(&bars->tfull[buf], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
       tc_fence_after();
       const int j = kt * kKeysPerTile + q4 * 32 + lane;
-      float acc = 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < 128; cc += 16) {
-        float v[16];
-        tmem_ld16(tmem + lane_addr + buf * 256 + hh * 128 + cc, v);
-        tmem_wait_ld16(v);
+      const int need = 16 * j + 31;     // window j is visible to tokens at or after this position
+      // software-pipelined over four 32-column chunks: the load of chunk
+      // c+1 is in flight while chunk c is computed
+      const uint32_t tcol = tmem + lane_addr + buf * 256 + hh * 128;
+      float va[32], vb[32];
+      tmem_ld32(tcol, va);
+      tmem_wait_ld32(va);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc += ex2(fmaf(v[i], c, -lse2[hh * 128 + cc + i]));
-          if ((i % G) == G - 1) {       // last head of a token: store its group sum
-            const int tt = t0 + (hh * 128 + cc + i) / G;
-            if (tt < len && j < visible_windows_dev(tt, 32, 16))
-              S[(static_cast<int64_t>(g) * total + row0 + tt) * ld + j] = acc;
-            acc = 0.f;
-          }
+      for (int cc = 0; cc < 128; cc += 32) {
+        float (&v)[32] = ((cc >> 5) & 1) ? vb : va;
+        float (&vn)[32] = ((cc >> 5) & 1) ? va : vb;
+        if (cc + 32 < 128) tmem_ld32(tcol + cc + 32, vn);
+        const float4* l4 = reinterpret_cast<const float4*>(nlse + hh * 128 + cc);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 L = l4[q];
+          v[4 * q + 0] = ex2(fmaf(v[4 * q + 0], c, L.x));
+          v[4 * q + 1] = ex2(fmaf(v[4 * q + 1], c, L.y));
+          v[4 * q + 2] = ex2(fmaf(v[4 * q + 2], c, L.z));
+          v[4 * q + 3] = ex2(fmaf(v[4 * q + 3], c, L.w));
         }
+        // group sums: tree over each token's G head columns
+#pragma unroll
+        for (int w = 1; w < G; w <<= 1) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2 * w) v[i] += v[i + w];
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += G) {
+          const int tl = (cc + i) / G;          // token index within this half
+          const int tt = tt0 + tl;
+          if (tt < len && tt >= need) srow0[static_cast<int64_t>(tl) * ld + j] = v[i];
+        }
+        if (cc + 32 < 128) tmem_wait_ld32(vn);
       }
       tc_fence_before();
       __syncwarp();
