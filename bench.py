@@ -83,6 +83,19 @@ def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
     return w
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of x over all ranks (the job's time is its slowest
+    rank's).  Single process: x itself."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     def __init__(self):
@@ -172,6 +185,82 @@ def oracle_sample(w, data, seconds: float):
     return n / total_s, rows, t_pool + t_rows
 
 
+# ---------------------------------------------------------------- decode
+def decode_bytes_per_step(prefix: int, steps: int, batch: int, h_kv: int, d: int) -> float:
+    """Algorithmic HBM bytes of one decode step (averaged over the timed
+    steps): the visible pooled keys of both kinds and the K/V rows of the
+    visible selected keys, per sequence and kv group."""
+    tot = 0.0
+    for i in range(steps):
+        t = prefix + i
+        n1 = (t - 31) // 16 + 1
+        n2 = (t - 127) // 64 + 1
+        b_t = t // 64
+        keys = (min(96, b_t + 1) - 1) * 64 + (t % 64) + 1
+        tot += batch * h_kv * (n1 * d * 2 + n2 * d * 2 + keys * 2 * d * 2)
+    return tot / steps
+
+
+def bench_decode(T, gen, torch, dev, graph_steps: int = 64, reps: int = 3):
+    """µs per decode step of the 16 x 131072 workload, steps replayed from a
+    CUDA graph of `graph_steps` consecutive steps (inputs staged on device)."""
+    w = gen.WORKLOADS["decode_16x128k"]
+    prefix, steps, batch = w.seqlen, graph_steps, w.batch
+    cap = prefix + steps
+    p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+    k_cache = torch.empty(batch, cap, w.h_kv, w.d, dtype=torch.bfloat16, device=dev)
+    v_cache = torch.empty_like(k_cache)
+    q_all = torch.empty(steps, batch, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
+    kn_all = torch.empty(steps, batch, w.h_kv, w.d, dtype=torch.bfloat16, device=dev)
+    vn_all = torch.empty_like(kn_all)
+    for b in range(batch):
+        one = gen.make_decode_sequence(w, b, prefix, steps)
+        k_cache[b] = one["K"].to(dev)
+        v_cache[b] = one["V"].to(dev)
+        q_all[:, b] = one["q_steps"].to(dev)
+        kn_all[:, b] = one["K"][prefix:].to(dev)
+        vn_all[:, b] = one["V"][prefix:].to(dev)
+    kc1 = torch.empty(batch, w.h_kv, T.window_count(cap, 32, 16), w.d, dtype=torch.bfloat16, device=dev)
+    kc2 = torch.empty(batch, w.h_kv, T.window_count(cap, 128, 64), w.d, dtype=torch.bfloat16, device=dev)
+    seq_len = torch.full((batch,), prefix, dtype=torch.int32, device=dev)
+    st = T.make_decode_state(k_cache, v_cache, kc1, kc2, seq_len, w.h_q)
+    ws = torch.empty(T.infllm2_decode_workspace_bytes(st, p), dtype=torch.uint8, device=dev)
+    out = torch.empty(batch, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
+    T.infllm2_decode_build_caches(st, p)
+    stream = torch.cuda.Stream()
+    prefix_t = torch.full((batch,), prefix, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    # one eager pass (warm-up, and the first call on the device)
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            T.infllm2_decode_step(st, q_all[i], kn_all[i], vn_all[i], out, ws, p, stream)
+        seq_len.copy_(prefix_t)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            T.infllm2_decode_step(st, q_all[i], kn_all[i], vn_all[i], out, ws, p, stream)
+    times = []
+    for _ in range(reps + 1):
+        seq_len.copy_(prefix_t)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    status = T.infllm2_get_device_status()
+    ms = statistics.median(times[1:])
+    us = 1e3 * ms / steps
+    byts = decode_bytes_per_step(prefix, steps, batch, w.h_kv, w.d)
+    del g
+    return {"workload": w.name, "us_per_step": us, "graph_steps": steps, "batch": batch, "cache": prefix,
+            "launches_per_step": 6, "bytes_per_step": byts, "achieved_GB/s": byts / (us / 1e6) / 1e9,
+            "device_status": status}
+
+
 # ---------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -183,6 +272,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -272,10 +362,7 @@ def main():
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
     per_kernel = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, nm in enumerate(kernels)}
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     tokens = w.seqlen * world
     value = tokens / (ms_per_step / 1e3)
@@ -301,11 +388,7 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / args.steps
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
         h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
         d2h = outh.numel() * outh.element_size()
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -359,6 +442,12 @@ def main():
         "clocks": clk,
         "device_status": status,
     }
+    if not args.no_decode:
+        dd = bench_decode(T, gen, torch, dev)
+        dd["peak_GB/s"] = hbm
+        dd["frac"] = dd["achieved_GB/s"] / hbm
+        dd["bound"] = "hbm"
+        line["decode"] = dd
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",

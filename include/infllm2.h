@@ -207,6 +207,45 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V,
                        const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
                        void* out, int32_t out_dtype, const infllm2_params* p, void* stream);
 
+/* ---------------------------------------------------------------------
+ * Step 5: one decode step per sequence (dtcms article §二.2.b: the sparse
+ * pattern serves prefill and decode alike).  The caller owns the state:
+ *   k_cache, v_cache  bf16 [batch, capacity, h_kv, d]
+ *   k_c1              bf16 [batch, h_kv, cap_c1, d], cap_c1 = infllm2_window_count(capacity, 32, 16)
+ *   k_c2              bf16 [batch, h_kv, cap_c2, d], cap_c2 = infllm2_window_count(capacity, 128, 64)
+ *   seq_len           int32 [batch] on the device: tokens already cached.
+ * infllm2_decode_step appends k_new / v_new ([batch, h_kv, d]) at position
+ * t = seq_len[b], pools the stage-1 window ending at t when 16 divides t+1
+ * (t+1 >= 32) and the coarse window ending at t when 64 divides t+1
+ * (t+1 >= 128), then computes for the query q ([batch, h_q, d]) exactly
+ * row t of the prefill path (scores, max-pool, selection, sparse attention
+ * over keys <= t) and writes out ([batch, h_q, d] bf16); finally
+ * seq_len[b] += 1.  t must be < capacity (else the device status records
+ * INFLLM2_ERR_DEVICE_BOUNDS and the sequence is skipped).  The step is a
+ * fixed sequence of kernel launches with no host synchronisation, so it can
+ * be captured in a CUDA graph.  workspace: infllm2_decode_workspace_bytes.
+ * infllm2_decode_build_caches pools the seq_len[b] tokens already in the
+ * cache into k_c1 / k_c2 (for a prefix written by the caller).
+ * ------------------------------------------------------------------- */
+typedef struct {
+  void* k_cache;
+  void* v_cache;
+  void* k_c1;
+  void* k_c2;
+  int32_t* seq_len;
+  int32_t batch;
+  int32_t capacity;
+  int32_t h_q;
+  int32_t h_kv;
+  int32_t d;
+} infllm2_decode_state;
+
+size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infllm2_params* p);
+int infllm2_decode_build_caches(const infllm2_decode_state* st, const infllm2_params* p, void* stream);
+int infllm2_decode_step(const infllm2_decode_state* st, const void* q, const void* k_new, const void* v_new,
+                        void* out, void* workspace, size_t workspace_bytes, const infllm2_params* p,
+                        void* stream);
+
 /* Device status word (per device).  Returns INFLLM2_OK or the first
  * INFLLM2_ERR_DEVICE_* recorded by a kernel since the last clear.
  * Synchronises the device. */

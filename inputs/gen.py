@@ -138,19 +138,17 @@ def make_decode(w: Workload, prefix: Optional[int] = None, steps: Optional[int] 
     decode steps append, one per step.  q_steps is [steps, batch, h_q, d].
     The block offset of a new token continues the block structure (a fresh
     offset starts with every new 64-token block).  Sequence s uses its own
-    seed, so one sequence can be regenerated alone."""
+    seed (draw order: step queries, K noise, mu, V), so one sequence can be
+    regenerated alone."""
     prefix = w.seqlen if prefix is None else prefix
     steps = w.decode_steps if steps is None else steps
     batch = w.batch if batch is None else batch
-    n = prefix + steps
     Ks, Vs, Qs = [], [], []
     for s in range(batch):
-        rng = np.random.Generator(np.random.PCG64(w.seed * 100 + s))
-        q = rng.standard_normal((n, w.h_q, w.d), dtype=np.float32)
-        Qs.append(to_bf16(q[prefix:]))
-        del q
-        Ks.append(to_bf16(_keys(rng, [n], w.h_kv, w.d, w.block_offset_std)))
-        Vs.append(to_bf16(rng.standard_normal((n, w.h_kv, w.d), dtype=np.float32)))
+        one = make_decode_sequence(w, s, prefix, steps)
+        Qs.append(one["q_steps"])
+        Ks.append(one["K"])
+        Vs.append(one["V"])
     return {
         "K": torch.stack(Ks),                       # [batch, n, h_kv, d]
         "V": torch.stack(Vs),
@@ -164,9 +162,8 @@ def make_decode_sequence(w: Workload, s: int, prefix: int, steps: int) -> dict:
     """One sequence of :func:`make_decode` (same values), without the others."""
     n = prefix + steps
     rng = np.random.Generator(np.random.PCG64(w.seed * 100 + s))
-    q = rng.standard_normal((n, w.h_q, w.d), dtype=np.float32)
-    Q = to_bf16(q[prefix:])
-    del q
+    # only the decoded tokens need queries (the prefix's queries are never used)
+    Q = to_bf16(rng.standard_normal((steps, w.h_q, w.d), dtype=np.float32))
     K = to_bf16(_keys(rng, [n], w.h_kv, w.d, w.block_offset_std))
     V = to_bf16(rng.standard_normal((n, w.h_kv, w.d), dtype=np.float32))
     return {"K": K, "V": V, "q_steps": Q}

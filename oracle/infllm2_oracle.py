@@ -291,6 +291,33 @@ class Sequence1:
         return attend(self.q_group(t, g), self.K[:, g, :], self.V[:, g, :], t, dense_keys(t), self.scale)
 
 
+def decode_row(K_seq: np.ndarray, V_seq: np.ndarray, q_t: np.ndarray, p: Params):
+    """One decode step: the new token at position t = len(K_seq) - 1 is row t
+    of the prefill rule on the extended sequence ([news] §二.2.b: the sparse
+    pattern serves prefill and decode alike), so this calls the pinned prefill
+    functions.  K_seq, V_seq: [t+1, h_kv, d] including the new token;
+    q_t: [h_q, d].  Returns (selected blocks [h_kv, |I|], output [h_q, d],
+    scores per group, the pooled keys K_C1, K_C2)."""
+    t = K_seq.shape[0] - 1
+    h_q, d = q_t.shape
+    h_kv = K_seq.shape[1]
+    G = h_q // h_kv
+    scale = p.softmax_scale(d)
+    Kc1 = pool_keys(K_seq, p.c1_len, p.c1_stride)
+    Kc2 = pool_keys(K_seq, p.c2_len, p.c2_stride)
+    sel = np.empty((h_kv, p.n_sel), dtype=np.int64)
+    out = np.empty((h_q, d))
+    scores = []
+    for g in range(h_kv):
+        qg = q_t[g * G:(g + 1) * G]
+        S = shared_scores(qg, Kc1[g], Kc2[g], t, p, scale)
+        scores.append(S)
+        sel[g] = select_blocks(S, t, p)
+        keys = sparse_keys(t, sel[g], p.block)
+        out[g * G:(g + 1) * G] = attend(qg, K_seq[:, g, :], V_seq[:, g, :], t, keys, scale)
+    return sel, out, scores, Kc1, Kc2
+
+
 def lse_rows_comparable(t: int, p: Params) -> bool:
     """Rows whose scores are defined by the approximation proper (at least one
     C2 window visible).  Earlier rows use the exact fallback; they never reach

@@ -1,0 +1,123 @@
+"""GPU parity of the decode step (append, incremental pooled caches, one-row
+selection and sparse attention) against the oracle's decode row, which is the
+pinned prefill rule applied to the sequence extended by the new token."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from inputs import gen
+from oracle import infllm2_oracle as O
+from tests import harness as H
+import trainable_block_sparse_pool_b200 as T
+
+pytestmark = pytest.mark.gpu
+
+
+class DecodeRun:
+    def __init__(self, w, prefix, steps, batch):
+        self.w = w
+        self.data = gen.make_decode(w, prefix=prefix, steps=steps, batch=batch)
+        self.p = H.lib_params(w)
+        dev = torch.device("cuda")
+        cap = prefix + steps
+        self.k_cache = torch.zeros(batch, cap, w.h_kv, w.d, dtype=torch.bfloat16, device=dev)
+        self.v_cache = torch.zeros_like(self.k_cache)
+        self.k_cache[:, :prefix] = self.data["K"][:, :prefix].to(dev)
+        self.v_cache[:, :prefix] = self.data["V"][:, :prefix].to(dev)
+        self.kc1 = torch.zeros(batch, w.h_kv, max(1, T.window_count(cap, 32, 16)), w.d, dtype=torch.bfloat16, device=dev)
+        self.kc2 = torch.zeros(batch, w.h_kv, max(1, T.window_count(cap, 128, 64)), w.d, dtype=torch.bfloat16, device=dev)
+        self.seq_len = torch.full((batch,), prefix, dtype=torch.int32, device=dev)
+        self.st = T.make_decode_state(self.k_cache, self.v_cache, self.kc1, self.kc2, self.seq_len, w.h_q)
+        self.ws = torch.empty(T.infllm2_decode_workspace_bytes(self.st, self.p), dtype=torch.uint8, device=dev)
+        self.out = torch.empty(batch, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
+        self.prefix, self.steps, self.batch = prefix, steps, batch
+        T.infllm2_decode_build_caches(self.st, self.p)
+
+    def step(self, i):
+        dev = torch.device("cuda")
+        t = self.prefix + i
+        q = self.data["q_steps"][i].to(dev)
+        kn = self.data["K"][:, t].contiguous().to(dev)
+        vn = self.data["V"][:, t].contiguous().to(dev)
+        T.infllm2_decode_step(self.st, q, kn, vn, self.out, self.ws, self.p)
+
+
+def _check_step(run, i, seqs, op):
+    torch.cuda.synchronize()
+    out = run.out.float().cpu().numpy()
+    t = run.prefix + i
+    errs, checked = [], 0
+    for b in seqs:
+        K = O.to_f64(run.data["K"][b, :t + 1])
+        V = O.to_f64(run.data["V"][b, :t + 1])
+        q = O.to_f64(run.data["q_steps"][i, b])
+        sel, ref, scores, _, _ = O.decode_row(K, V, q, op)
+        # skip groups whose top-k is decided by a near tie (gap <= 1e-4)
+        for g in range(run.w.h_kv):
+            if O.topk_gap(scores[g], t, op) <= H.GAP_MIN:
+                continue
+            G = run.w.group
+            errs.append(np.abs(out[b, g * G:(g + 1) * G] - ref[g * G:(g + 1) * G]).ravel())
+            checked += 1
+    return errs, checked
+
+
+def _run_case(w, prefix, steps, batch, check_every=1, seqs=None):
+    run = DecodeRun(w, prefix, steps, batch)
+    op = H.oracle_params(w)
+    seqs = list(range(batch)) if seqs is None else seqs
+    errs, checked = [], 0
+    for i in range(steps):
+        run.step(i)
+        if i % check_every == 0 or i == steps - 1:
+            e, c = _check_step(run, i, seqs, op)
+            errs += e
+            checked += c
+    assert checked > 0
+    e = np.concatenate(errs)
+    assert e.max() <= H.ATT_MAX_ABS and e.mean() <= H.ATT_MEAN_ABS, (e.max(), e.mean())
+    # the pooled caches after the steps equal the oracle's pooling of the whole sequence
+    torch.cuda.synchronize()
+    assert run.seq_len.cpu().tolist() == [prefix + steps] * batch
+    n = prefix + steps
+    for b in seqs:
+        K = O.to_f64(run.data["K"][b, :n])
+        c1 = O.pool_keys(K, 32, 16)
+        c2 = O.pool_keys(K, 128, 64)
+        np.testing.assert_array_equal(run.kc1[b, :, :c1.shape[1]].float().cpu().numpy(), c1)
+        np.testing.assert_array_equal(run.kc2[b, :, :c2.shape[1]].float().cpu().numpy(), c2)
+    assert T.infllm2_get_device_status() == 0
+
+
+def test_decode_small_d128_g16():
+    # prefixes straddle the interesting boundaries: no coarse window yet,
+    # fewer candidates than top_k, and a full selection
+    w = dataclasses.replace(gen.WORKLOADS["prefill_32k"], name="decode_small", n_local=4, top_k=6, seed=41)
+    _run_case(w, prefix=100, steps=70, batch=1)
+    _run_case(dataclasses.replace(w, seed=42), prefix=1500, steps=40, batch=3)
+
+
+def test_decode_tiny_d64_g4():
+    w = dataclasses.replace(gen.WORKLOADS["tiny_1k"], name="decode_tiny", seed=43)
+    _run_case(w, prefix=900, steps=130, batch=2, check_every=3)
+
+
+def test_decode_16x128k_sampled():
+    # the benchmark's decode workload: 16 sequences x 131072-token cache;
+    # the oracle checks two sequences on the first and a later step
+    w = gen.WORKLOADS["decode_16x128k"]
+    run = DecodeRun(w, prefix=w.seqlen, steps=4, batch=w.batch)
+    op = H.oracle_params(w)
+    errs, checked = [], 0
+    for i in range(4):
+        run.step(i)
+        if i in (0, 3):
+            e, c = _check_step(run, i, [0, 11], op)
+            errs += e
+            checked += c
+    assert checked > 0
+    e = np.concatenate(errs)
+    assert e.max() <= H.ATT_MAX_ABS and e.mean() <= H.ATT_MEAN_ABS, (e.max(), e.mean())
+    assert T.infllm2_get_device_status() == 0

@@ -22,7 +22,8 @@ __all__ = [
     "infllm2_compress_k", "infllm2_shared_scores", "infllm2_topk_blocks", "infllm2_select_blocks",
     "infllm2_select_workspace_bytes", "infllm2_scores_ld", "infllm2_sparse_attn", "infllm2_dense_attn",
     "infllm2_get_device_status", "infllm2_clear_device_status", "infllm2_debug_wait_timeout",
-    "OUT_BF16", "OUT_F32",
+    "DecodeState", "make_decode_state", "infllm2_decode_workspace_bytes", "infllm2_decode_build_caches",
+    "infllm2_decode_step", "OUT_BF16", "OUT_F32",
 ]
 
 OUT_BF16 = 0
@@ -51,6 +52,14 @@ class Varlen(ctypes.Structure):
     _fields_ = [
         ("cu_seqlens", ctypes.c_void_p), ("batch", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
         ("total", ctypes.c_int64), ("total_c1", ctypes.c_int64), ("total_c2", ctypes.c_int64),
+    ]
+
+
+class DecodeState(ctypes.Structure):
+    _fields_ = [
+        ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("k_c1", ctypes.c_void_p),
+        ("k_c2", ctypes.c_void_p), ("seq_len", ctypes.c_void_p), ("batch", ctypes.c_int32),
+        ("capacity", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32), ("d", ctypes.c_int32),
     ]
 
 
@@ -84,6 +93,10 @@ def lib() -> ctypes.CDLL:
         "infllm2_get_device_status": (ctypes.c_int, []),
         "infllm2_clear_device_status": (ctypes.c_int, []),
         "infllm2_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
+        "infllm2_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(DecodeState), pp]),
+        "infllm2_decode_build_caches": (ctypes.c_int, [ctypes.POINTER(DecodeState), pp, _P]),
+        "infllm2_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P, ctypes.c_size_t, pp,
+                                                _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -215,3 +228,34 @@ def infllm2_clear_device_status() -> None:
 
 def infllm2_debug_wait_timeout(limit_ns: int, stream=None) -> None:
     _check("infllm2_debug_wait_timeout", lib().infllm2_debug_wait_timeout(limit_ns, _stream(stream)))
+
+
+def make_decode_state(k_cache: torch.Tensor, v_cache: torch.Tensor, k_c1: torch.Tensor, k_c2: torch.Tensor,
+                      seq_len: torch.Tensor, h_q: int) -> DecodeState:
+    """Decode state over caller-owned device tensors: caches [batch, capacity,
+    h_kv, d], pooled caches [batch, h_kv, cap, d], seq_len int32 [batch]."""
+    st = DecodeState()
+    st.k_cache, st.v_cache = _ptr(k_cache), _ptr(v_cache)
+    st.k_c1, st.k_c2, st.seq_len = _ptr(k_c1), _ptr(k_c2), _ptr(seq_len)
+    st.batch, st.capacity, st.h_kv, st.d = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2], k_cache.shape[3]
+    st.h_q = h_q
+    st._keep = (k_cache, v_cache, k_c1, k_c2, seq_len)  # noqa: SLF001
+    return st
+
+
+def infllm2_decode_workspace_bytes(st: DecodeState, params: Optional[Params] = None) -> int:
+    return int(lib().infllm2_decode_workspace_bytes(ctypes.byref(st), ctypes.byref(params or default_params())))
+
+
+def infllm2_decode_build_caches(st: DecodeState, params: Optional[Params] = None, stream=None) -> None:
+    rc = lib().infllm2_decode_build_caches(ctypes.byref(st), ctypes.byref(params or default_params()), _stream(stream))
+    _check("infllm2_decode_build_caches", rc)
+
+
+def infllm2_decode_step(st: DecodeState, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                        out: torch.Tensor, workspace: torch.Tensor, params: Optional[Params] = None,
+                        stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().infllm2_decode_step(ctypes.byref(st), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(workspace),
+                                   ws_bytes, ctypes.byref(params or default_params()), _stream(stream))
+    _check("infllm2_decode_step", rc)

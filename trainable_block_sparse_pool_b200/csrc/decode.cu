@@ -1,2 +1,537 @@
-// decode step (to come)
+// Step 5: one decode step — a new token per sequence against a KV cache,
+// with the pooled key caches kept current (InfLLM-V2 keeps the sparse
+// pattern for decoding too: dtcms article §二.2.b, "prefill 与 decode 全链路";
+// the pages' end-to-end decode measurement at |I| = 96).
+//
+// The new token of sequence b sits at position t = seq_len[b]; the step is
+// row t of the prefill rule applied to the sequence extended by one token:
+//   A  append k, v at t; if a stage-1 window ends at t (t+1 >= 32,
+//      (t+1) % 16 == 0) pool it into K_c1, likewise a coarse window
+//      (t+1 >= 128, (t+1) % 64 == 0) into K_c2 — exact mean, one bf16 rounding
+//   B  per-head log-sum-exp over the visible coarse windows, split over CTAs
+//   C  S over the visible stage-1 windows (head-group sum fused) and the
+//      max-pool to block scores, split over CTAs (each CTA keeps one window
+//      of halo so blocks never straddle CTAs)
+//   D  top-k selection per (sequence, kv group)
+//   E  split-KV block-sparse attention: the prefill sparse kernel in its
+//      partial-output mode (sparse_attn.cu)
+//   F  combine the splits, write the output, advance seq_len
+// All of it is HBM-bound (the pooled keys and the selected K/V are read
+// once); the tiny contractions of B and C (16 heads against 8 windows per
+// instruction) use warp-level mma.sync, which is far from being the limit.
 #include "sm100.cuh"
+
+namespace infllm2 {
+
+namespace dec {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kLseWin = 128;   // coarse windows per LSE CTA
+constexpr int kScoreWin = 256; // stage-1 windows per score CTA (64 blocks)
+
+// D = A(16x16, bf16, row) * B(16x8, bf16, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The contraction over d uses a fixed permutation of d inside each pair of
+// 16-wide k steps, so a thread's operands are one 16-byte load: for
+// k-step 2p+e, thread (gid, tig) covers d = 32p + 8 tig + 4e + {0,1} (as
+// logical k 2tig, 2tig+1) and + {2,3} (as k 2tig+8, 2tig+9).  A and B use
+// the same map, so the sum is unchanged.
+template <int D>
+struct QFrag {
+  uint4 lo[D / 32], hi[D / 32];   // heads gid and gid + 8
+};
+
+template <int D>
+__device__ __forceinline__ void load_qfrag(QFrag<D>& f, const __nv_bfloat16* q_heads /* [16][D] */, int lane,
+                                           int G) {
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int p = 0; p < D / 32; ++p) {
+    const int off = 32 * p + 8 * tig;
+    f.lo[p] = (gid < G) ? *reinterpret_cast<const uint4*>(q_heads + gid * D + off) : make_uint4(0, 0, 0, 0);
+    f.hi[p] = (gid + 8 < G) ? *reinterpret_cast<const uint4*>(q_heads + (gid + 8) * D + off) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Scores of 16 heads against the 8 keys rows[gid] (a row pointer per lane
+// group, nullptr = zero row).  c[0..1]: head gid, keys 2tig, 2tig+1;
+// c[2..3]: head gid+8.
+template <int D>
+__device__ __forceinline__ void scores_16x8(float (&c)[4], const QFrag<D>& f, const __nv_bfloat16* row, int lane) {
+  const int tig = lane & 3;
+  c[0] = c[1] = c[2] = c[3] = 0.f;
+#pragma unroll
+  for (int p = 0; p < D / 32; ++p) {
+    const uint4 kv = row ? *reinterpret_cast<const uint4*>(row + 32 * p + 8 * tig) : make_uint4(0, 0, 0, 0);
+    const uint32_t a0[4] = {f.lo[p].x, f.hi[p].x, f.lo[p].y, f.hi[p].y};
+    mma16816(c, a0, kv.x, kv.y);
+    const uint32_t a1[4] = {f.lo[p].z, f.hi[p].z, f.lo[p].w, f.hi[p].w};
+    mma16816(c, a1, kv.z, kv.w);
+  }
+}
+
+// ---------------------------------------------------------------- A: append + pool
+template <int D>
+__global__ void __launch_bounds__(128) append_kernel(const __nv_bfloat16* __restrict__ k_new,
+                                                     const __nv_bfloat16* __restrict__ v_new,
+                                                     __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
+                                                     __nv_bfloat16* __restrict__ kc1, __nv_bfloat16* __restrict__ kc2,
+                                                     const int32_t* __restrict__ seq_len, int capacity, int h_kv,
+                                                     int cap_c1, int cap_c2) {
+  constexpr int SL = D / 8;
+  constexpr int NRG = 128 / SL;                 // row groups of the 128 threads
+  __shared__ double part[NRG][D];
+  const int b = blockIdx.x / h_kv, g = blockIdx.x % h_kv;
+  const int t = seq_len[b];
+  if (t < 0 || t >= capacity) {
+    if (threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const int64_t seq0 = static_cast<int64_t>(b) * capacity;
+  const __nv_bfloat16* kn = k_new + (static_cast<int64_t>(b) * h_kv + g) * D;
+  const __nv_bfloat16* vn = v_new + (static_cast<int64_t>(b) * h_kv + g) * D;
+  if (threadIdx.x < SL) {
+    reinterpret_cast<uint4*>(kc + ((seq0 + t) * h_kv + g) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(kn)[threadIdx.x];
+    reinterpret_cast<uint4*>(vc + ((seq0 + t) * h_kv + g) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(vn)[threadIdx.x];
+  }
+  // a window [t-len+1, t] completes at this step: pool it (rows before t come
+  // from the cache, row t from k_new)
+  for (int which = 0; which < 2; ++which) {
+    const int len = which ? 128 : 32, stride = which ? 64 : 16;
+    if (t + 1 < len || (t + 1 - len) % stride != 0) continue;
+    const int j = (t + 1 - len) / stride;
+    if (j >= (which ? cap_c2 : cap_c1)) {
+      if (threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    // 128 threads: slice sl = tid % SL, row group rg = tid / SL (8 groups for D=128)
+    const int sl = threadIdx.x % SL, rg = threadIdx.x / SL;
+    double acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    for (int r = rg; r < len; r += NRG) {
+      const int u = t - len + 1 + r;
+      const __nv_bfloat16* src = (u == t) ? kn : kc + ((seq0 + u) * h_kv + g) * D;
+      const uint4 raw = reinterpret_cast<const uint4*>(src)[sl];
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(p2[i]);
+        acc[2 * i] += static_cast<double>(f.x);
+        acc[2 * i + 1] += static_cast<double>(f.y);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[rg][sl * 8 + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < SL) {
+      uint16_t o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        double s = 0.0;
+        for (int q = 0; q < NRG; ++q) s += part[q][threadIdx.x * 8 + i];
+        o[i] = f64_to_bf16_rne(s / len);
+      }
+      uint4 v;
+      v.x = o[0] | (static_cast<uint32_t>(o[1]) << 16);
+      v.y = o[2] | (static_cast<uint32_t>(o[3]) << 16);
+      v.z = o[4] | (static_cast<uint32_t>(o[5]) << 16);
+      v.w = o[6] | (static_cast<uint32_t>(o[7]) << 16);
+      __nv_bfloat16* dst = (which ? kc2 : kc1) +
+                           ((static_cast<int64_t>(b) * h_kv + g) * (which ? cap_c2 : cap_c1) + j) * D;
+      reinterpret_cast<uint4*>(dst)[threadIdx.x] = v;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- B: coarse LSE partials
+// grid (batch*h_kv, nsplit2), 4 warps.  part2[(bg*nsplit2 + c)*16 + h] = (max, sum) in log2 units.
+template <int D>
+__global__ void __launch_bounds__(128) lse_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc2,
+                                                  const int32_t* __restrict__ seq_len, int h_q, int h_kv, int cap_c2,
+                                                  float scale, float2* __restrict__ part2) {
+  const int bg = blockIdx.x, c = blockIdx.y;
+  const int b = bg / h_kv, g = bg % h_kv;
+  const int G = h_q / h_kv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  __shared__ float2 red[4][16];
+  const int t = seq_len[b];
+  const int n2 = visible_windows_dev(t, 128, 64);
+  QFrag<D> f;
+  load_qfrag<D>(f, q + (static_cast<int64_t>(b) * h_q + g * G) * D, lane, G);
+  const float cs = scale * kLog2e;
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // heads gid, gid+8
+  const __nv_bfloat16* base = kc2 + static_cast<int64_t>(bg) * cap_c2 * D;
+  for (int nt = warp; nt < kLseWin / 8; nt += 4) {
+    const int w0 = c * kLseWin + nt * 8;
+    if (w0 >= n2) break;
+    const int wr = w0 + gid;
+    float sc[4];
+    scores_16x8<D>(sc, f, (wr < n2) ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float x0 = (w0 + 2 * tig < n2) ? sc[2 * r] * cs : -INFINITY;
+      float x1 = (w0 + 2 * tig + 1 < n2) ? sc[2 * r + 1] * cs : -INFINITY;
+      const float mn = fmaxf(m[r], fmaxf(x0, x1));
+      if (mn != -INFINITY) {
+        l[r] = l[r] * ex2(m[r] - mn) + ex2(x0 - mn) + ex2(x1 - mn);
+        m[r] = mn;
+      }
+    }
+  }
+  // combine over the 4 lanes of a head row, then over warps
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[r], o);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[r], o);
+      const float mn = fmaxf(m[r], mo);
+      if (mn != -INFINITY) {
+        l[r] = l[r] * ex2(m[r] - mn) + lo * ex2(mo - mn);
+        m[r] = mn;
+      }
+    }
+  }
+  if (tig == 0) {
+    red[warp][gid] = make_float2(m[0], l[0]);
+    red[warp][gid + 8] = make_float2(m[1], l[1]);
+  }
+  __syncthreads();
+  if (threadIdx.x < 16) {
+    float mm = -INFINITY, ll = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float2 v = red[w][threadIdx.x];
+      const float mn = fmaxf(mm, v.x);
+      if (mn != -INFINITY) {
+        ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
+        mm = mn;
+      }
+    }
+    part2[(static_cast<int64_t>(bg) * gridDim.y + c) * 16 + threadIdx.x] = make_float2(mm, ll);
+  }
+}
+
+// ---------------------------------------------------------------- C: scores + max-pool
+// grid (batch*h_kv, nsplit1), 8 warps; windows [256c - 1, 256c + 255) -> blocks [64c, 64c + 64)
+template <int D>
+__global__ void __launch_bounds__(256) score_pool_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
+    const float2* __restrict__ part2, int nsplit2, int h_q, int h_kv, int cap_c1, int nblk_cap, float scale,
+    float* __restrict__ bscore) {
+  const int bg = blockIdx.x, c = blockIdx.y;
+  const int b = bg / h_kv, g = bg % h_kv;
+  const int G = h_q / h_kv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  __shared__ float nlse[16];
+  __shared__ float sw[kScoreWin + 8];
+  const int t = seq_len[b];
+  const int n1 = visible_windows_dev(t, 32, 16);
+  const int n2 = visible_windows_dev(t, 128, 64);
+  const int j0 = c * kScoreWin - 1;
+  if (j0 + 1 >= n1 && c > 0) return;            // no visible window here
+  const float cs = scale * kLog2e;
+  const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
+  const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
+  if (threadIdx.x < 16) {
+    const int h = threadIdx.x;
+    float mm = -INFINITY, ll = 0.f;
+    if (h < G) {
+      if (n2 > 0) {
+        for (int k = 0; k < nsplit2; ++k) {
+          const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + k) * 16 + h];
+          const float mn = fmaxf(mm, v.x);
+          if (mn != -INFINITY) {
+            ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
+            mm = mn;
+          }
+        }
+      } else {
+        // no coarse window yet (t < 127): exact log-sum-exp over the visible stage-1 windows
+        for (int j = 0; j < n1 && j < cap_c1; ++j) {
+          float dot = 0.f;
+          for (int e = 0; e < D; ++e)
+            dot += __bfloat162float(qh[h * D + e]) * __bfloat162float(base[static_cast<int64_t>(j) * D + e]);
+          const float x = dot * cs;
+          const float mn = fmaxf(mm, x);
+          ll = ll * ex2(mm - mn) + ex2(x - mn);
+          mm = mn;
+        }
+      }
+    }
+    nlse[h] = (h < G && ll > 0.f) ? -(mm + log2f(ll)) : -INFINITY;
+  }
+  __syncthreads();
+  QFrag<D> f;
+  load_qfrag<D>(f, qh, lane, G);
+  const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
+  for (int nt = warp; nt * 8 < kScoreWin + 1; nt += 8) {
+    const int w0 = j0 + nt * 8;
+    const int wr = w0 + gid;
+    float sc[4];
+    scores_16x8<D>(sc, f, (wr >= 0 && wr < n1) ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+    // head-group sum for keys 2tig and 2tig+1: two heads here, the other 14 on the lanes with the same tig
+    float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
+    float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      e0 += __shfl_xor_sync(0xffffffffu, e0, o);
+      e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+    }
+    if (gid == 0) {
+      const int i0 = nt * 8 + 2 * tig;
+      if (i0 < kScoreWin + 8) sw[i0] = (w0 + 2 * tig >= 0 && w0 + 2 * tig < n1) ? e0 : -INFINITY;
+      if (i0 + 1 < kScoreWin + 8) sw[i0 + 1] = (w0 + 2 * tig + 1 >= 0 && w0 + 2 * tig + 1 < n1) ? e1 : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // block scores: block blk = 64c + i takes windows 4 blk - 1 .. 4 blk + 3 = sw[4i .. 4i + 4]
+  if (threadIdx.x < kScoreWin / 4) {
+    const int i = threadIdx.x;
+    const int blk = c * (kScoreWin / 4) + i;
+    if (blk < nblk_cap) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int q4 = 0; q4 < 5; ++q4) m = fmaxf(m, sw[4 * i + q4]);
+      bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- D: top-k per (sequence, group)
+__global__ void __launch_bounds__(32) select_kernel(const float* __restrict__ bscore, const int32_t* __restrict__ seq_len,
+                                                    int h_kv, int nblk_cap, int cand_cap, int n_init, int n_local,
+                                                    int top_k, int n_sel, int32_t* __restrict__ idx) {
+  extern __shared__ uint32_t dsel_smem[];
+  uint32_t* keys = dsel_smem;
+  int* hist = reinterpret_cast<int*>(keys + cand_cap);
+  const int bg = blockIdx.x, lane = threadIdx.x;
+  const int b = bg / h_kv;
+  const int t = seq_len[b];
+  const int b_t = t / 64;
+  int32_t* out = idx + static_cast<int64_t>(bg) * n_sel;
+  const int init_hi = min(n_init, b_t + 1);
+  const int loc_lo = max(0, b_t - n_local + 1);
+  const int ncand = max(0, loc_lo - init_hi);
+  if (ncand <= top_k) {
+    for (int i = lane; i < n_sel; i += 32) out[i] = (i <= b_t) ? i : -1;
+    return;
+  }
+  if (ncand > cand_cap || init_hi + ncand > nblk_cap) {
+    if (lane == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const float* row = bscore + static_cast<int64_t>(bg) * nblk_cap;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int i = lane; i < ncand; i += 32) {
+    const uint32_t k = __float_as_uint(fmaxf(row[init_hi + i], 0.f));
+    keys[i] = k;
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+  sel::warp_select_write(keys, hist, ncand, init_hi, init_hi, loc_lo, b_t, top_k, n_sel, kmin, kmax, out, lane);
+}
+
+// ---------------------------------------------------------------- F: combine + advance
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int nsplit, int h_q, int h_kv,
+                                                      __nv_bfloat16* __restrict__ out, int32_t* __restrict__ seq_len) {
+  const int bg = blockIdx.x;
+  const int b = bg / h_kv, g = bg % h_kv;
+  const int G = h_q / h_kv;
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int h = i / D, dd = i % D;
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part[((static_cast<int64_t>(bg) * nsplit + s) * G + h) * (D + 2) + D]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < nsplit; ++s) {
+        const float* p = part + ((static_cast<int64_t>(bg) * nsplit + s) * G + h) * (D + 2);
+        const float m = p[D];
+        if (m == -INFINITY) continue;
+        const float w = ex2(m - M);
+        L += p[D + 1] * w;
+        O += p[dd] * w;
+      }
+    }
+    out[(static_cast<int64_t>(b) * h_q + g * G + h) * D + dd] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+  }
+  __syncthreads();
+  if (g == 0 && threadIdx.x == 0) seq_len[b] = seq_len[b] + 1;
+}
+
+// ---------------------------------------------------------------- pooled caches of a prefix
+// grid (ceil(capacity/512), batch, h_kv): the compress algorithm on the
+// decode cache layout, for the seq_len[b] tokens already in the cache.
+template <int D>
+__global__ void __launch_bounds__(256) build_caches_kernel(const __nv_bfloat16* __restrict__ kc,
+                                                           const int32_t* __restrict__ seq_len, int capacity, int h_kv,
+                                                           __nv_bfloat16* __restrict__ kc1, int cap_c1,
+                                                           __nv_bfloat16* __restrict__ kc2, int cap_c2) {
+  constexpr int SL = D / 8;
+  constexpr int NCH = 512 / 16 + 8;
+  __shared__ double csum[NCH][D];
+  const int b = blockIdx.y, g = blockIdx.z;
+  const int len = min(seq_len[b], capacity);
+  const int t0 = blockIdx.x * 512;
+  if (t0 >= len) return;
+  const int64_t seq0 = static_cast<int64_t>(b) * capacity;
+  for (int item = threadIdx.x; item < NCH * SL; item += 256) {
+    const int ch = item / SL, sl = item % SL;
+    double acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    for (int r = 0; r < 16; ++r) {
+      const int t = t0 + ch * 16 + r;
+      if (t < len) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(kc + ((seq0 + t) * h_kv + g) * D + sl * 8);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f2 = __bfloat1622float2(p2[i]);
+          acc[2 * i] += static_cast<double>(f2.x);
+          acc[2 * i + 1] += static_cast<double>(f2.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) csum[ch][sl * 8 + i] = acc[i];
+  }
+  __syncthreads();
+  const int n_c1 = window_count_dev(len, 32, 16), n_c2 = window_count_dev(len, 128, 64);
+  for (int item = threadIdx.x; item < 40 * SL; item += 256) {
+    const bool is2 = item >= 32 * SL;
+    const int w = is2 ? (item - 32 * SL) / SL : item / SL;
+    const int sl = item % SL;
+    const int j = is2 ? t0 / 64 + w : t0 / 16 + w;
+    if (j >= (is2 ? n_c2 : n_c1) || j >= (is2 ? cap_c2 : cap_c1)) continue;
+    uint16_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      double a = 0.0;
+      if (is2) {
+        for (int q4 = 0; q4 < 8; ++q4) a += csum[4 * w + q4][sl * 8 + i];
+        o[i] = f64_to_bf16_rne(a * (1.0 / 128.0));
+      } else {
+        a = csum[w][sl * 8 + i] + csum[w + 1][sl * 8 + i];
+        o[i] = f64_to_bf16_rne(a * (1.0 / 32.0));
+      }
+    }
+    uint4 v;
+    v.x = o[0] | (static_cast<uint32_t>(o[1]) << 16);
+    v.y = o[2] | (static_cast<uint32_t>(o[3]) << 16);
+    v.z = o[4] | (static_cast<uint32_t>(o[5]) << 16);
+    v.w = o[6] | (static_cast<uint32_t>(o[7]) << 16);
+    __nv_bfloat16* dst = (is2 ? kc2 : kc1) + ((static_cast<int64_t>(b) * h_kv + g) * (is2 ? cap_c2 : cap_c1) + j) * D;
+    reinterpret_cast<uint4*>(dst)[sl] = v;
+  }
+}
+
+}  // namespace dec
+
+// ---------------------------------------------------------------- host side
+struct DecodePlan {
+  int cap_c1, cap_c2, nblk_cap, cand_cap, nsplit2, nsplit1, nsplit, bps, n_sel;
+  size_t off_part2, off_bscore, off_idx, off_part, bytes;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_sel, int sms) {
+  DecodePlan p{};
+  p.n_sel = n_sel;
+  p.cap_c1 = static_cast<int>(infllm2_window_count(capacity, 32, 16));
+  p.cap_c2 = static_cast<int>(infllm2_window_count(capacity, 128, 64));
+  p.nblk_cap = (capacity + 63) / 64;
+  p.cand_cap = (p.nblk_cap + 31) & ~31;
+  p.nsplit2 = std::max(1, (p.cap_c2 + dec::kLseWin - 1) / dec::kLseWin);
+  p.nsplit1 = std::max(1, (p.cap_c1 + dec::kScoreWin) / dec::kScoreWin);
+  const int bg = batch * h_kv;
+  const int target = std::max(1, (4 * sms + bg - 1) / bg);           // about four units per SM
+  int bps = std::max(2, (n_sel + target - 1) / target);
+  bps = (bps + 1) & ~1;                                               // whole pairs of blocks
+  p.bps = bps;
+  p.nsplit = std::max(1, (n_sel + bps - 1) / bps);
+  const int G = h_q / h_kv;
+  size_t off = 0;
+  p.off_part2 = off; off = align256(off + static_cast<size_t>(bg) * p.nsplit2 * 16 * sizeof(float2));
+  p.off_bscore = off; off = align256(off + static_cast<size_t>(bg) * p.nblk_cap * sizeof(float));
+  p.off_idx = off; off = align256(off + static_cast<size_t>(bg) * n_sel * sizeof(int32_t));
+  p.off_part = off; off = align256(off + static_cast<size_t>(bg) * p.nsplit * G * (d + 2) * sizeof(float));
+  p.bytes = off;
+  return p;
+}
+
+cudaError_t launch_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* idx,
+                                 const int32_t* seq_len, int batch, int capacity, int h_q, int h_kv, int d,
+                                 int n_sel, int nsplit, int bps, float scale, float* part, cudaStream_t st,
+                                 bool* map_fail);
+
+template <int D>
+static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, const void* k_new, const void* v_new,
+                                 void* out, void* ws, const DecodePlan& P, int n_init, int n_local, int top_k,
+                                 float scale, cudaStream_t st, bool* map_fail) {
+  using bf = __nv_bfloat16;
+  const int bg = s->batch * s->h_kv;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float2* part2 = reinterpret_cast<float2*>(w + P.off_part2);
+  float* bscore = reinterpret_cast<float*>(w + P.off_bscore);
+  int32_t* idx = reinterpret_cast<int32_t*>(w + P.off_idx);
+  float* part = reinterpret_cast<float*>(w + P.off_part);
+  dec::append_kernel<D><<<bg, 128, 0, st>>>(static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
+                                            static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache),
+                                            static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2), s->seq_len,
+                                            s->capacity, s->h_kv, P.cap_c1, P.cap_c2);
+  dec::lse_kernel<D><<<dim3(bg, P.nsplit2), 128, 0, st>>>(static_cast<const bf*>(q), static_cast<const bf*>(s->k_c2),
+                                                          s->seq_len, s->h_q, s->h_kv, P.cap_c2, scale, part2);
+  dec::score_pool_kernel<D><<<dim3(bg, P.nsplit1), 256, 0, st>>>(
+      static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->h_q, s->h_kv,
+      P.cap_c1, P.nblk_cap, scale, bscore);
+  const size_t sel_smem = (static_cast<size_t>(P.cand_cap) + sel::kHistBins) * 4;
+  cudaError_t e = cudaFuncSetAttribute(dec::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sel_smem));
+  if (e != cudaSuccess) return e;
+  dec::select_kernel<<<bg, 32, sel_smem, st>>>(bscore, s->seq_len, s->h_kv, P.nblk_cap, P.cand_cap, n_init, n_local,
+                                               top_k, P.n_sel, idx);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_sparse_decode(q, s->k_cache, s->v_cache, idx, s->seq_len, s->batch, s->capacity, s->h_q, s->h_kv, D,
+                           P.n_sel, P.nsplit, P.bps, scale, part, st, map_fail);
+  if (e != cudaSuccess) return e;
+  dec::combine_kernel<D><<<bg, 256, 0, st>>>(part, P.nsplit, s->h_q, s->h_kv, static_cast<bf*>(out), s->seq_len);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_step(const infllm2_decode_state* s, const void* q, const void* k_new, const void* v_new,
+                               void* out, void* ws, const DecodePlan& P, int n_init, int n_local, int top_k,
+                               float scale, cudaStream_t st, bool* map_fail) {
+  if (s->d == 128) return decode_step_t<128>(s, q, k_new, v_new, out, ws, P, n_init, n_local, top_k, scale, st, map_fail);
+  return decode_step_t<64>(s, q, k_new, v_new, out, ws, P, n_init, n_local, top_k, scale, st, map_fail);
+}
+
+cudaError_t launch_decode_build_caches(const infllm2_decode_state* s, const DecodePlan& P, cudaStream_t st) {
+  dim3 grid((s->capacity + 511) / 512, s->batch, s->h_kv);
+  using bf = __nv_bfloat16;
+  if (s->d == 128)
+    dec::build_caches_kernel<128><<<grid, 256, 0, st>>>(static_cast<const bf*>(s->k_cache), s->seq_len, s->capacity,
+                                                        s->h_kv, static_cast<bf*>(s->k_c1), P.cap_c1,
+                                                        static_cast<bf*>(s->k_c2), P.cap_c2);
+  else
+    dec::build_caches_kernel<64><<<grid, 256, 0, st>>>(static_cast<const bf*>(s->k_cache), s->seq_len, s->capacity,
+                                                       s->h_kv, static_cast<bf*>(s->k_c1), P.cap_c1,
+                                                       static_cast<bf*>(s->k_c2), P.cap_c2);
+  return cudaGetLastError();
+}
+
+}  // namespace infllm2

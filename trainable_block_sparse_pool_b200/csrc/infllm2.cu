@@ -240,6 +240,47 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V, const infllm
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
 
+static int check_decode_state(const infllm2_decode_state* s) {
+  if (!s || !s->k_cache || !s->v_cache || !s->k_c1 || !s->k_c2 || !s->seq_len) return INFLLM2_ERR_INVALID_ARG;
+  if (!aligned16(s->k_cache) || !aligned16(s->v_cache) || !aligned16(s->k_c1) || !aligned16(s->k_c2))
+    return INFLLM2_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->batch > 65535 || s->capacity < 1) return INFLLM2_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s->batch) * s->capacity > INT32_MAX) return INFLLM2_ERR_UNSUPPORTED;
+  return check_heads(s->h_q, s->h_kv, s->d);
+}
+
+size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infllm2_params* p) {
+  if (check_decode_state(st) || check_params(p)) return 0;
+  return decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d, p->n_init + p->n_local + p->top_k,
+                     num_sms()).bytes;
+}
+
+int infllm2_decode_build_caches(const infllm2_decode_state* st, const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_decode_state(st)) || (r = check_params(p))) return r;
+  const DecodePlan P = decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d,
+                                   p->n_init + p->n_local + p->top_k, num_sms());
+  cudaError_t e = launch_decode_build_caches(st, P, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_decode_step(const infllm2_decode_state* st, const void* q, const void* k_new, const void* v_new,
+                        void* out, void* workspace, size_t workspace_bytes, const infllm2_params* p, void* stream) {
+  int r;
+  if ((r = check_decode_state(st)) || (r = check_params(p))) return r;
+  if (!q || !k_new || !v_new || !out || !workspace || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned16(out) || !aligned16(workspace))
+    return INFLLM2_ERR_INVALID_ARG;
+  const DecodePlan P = decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d,
+                                   p->n_init + p->n_local + p->top_k, num_sms());
+  if (workspace_bytes < P.bytes) return INFLLM2_ERR_WORKSPACE_TOO_SMALL;
+  bool map_fail = false;
+  cudaError_t e = launch_decode_step(st, q, k_new, v_new, out, workspace, P, p->n_init, p->n_local, p->top_k,
+                                     softmax_scale(p, st->d), static_cast<cudaStream_t>(stream), &map_fail);
+  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
 int infllm2_get_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e);

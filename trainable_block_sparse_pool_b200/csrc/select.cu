@@ -47,51 +47,14 @@ __device__ __forceinline__ float block_score(const float* __restrict__ row, int 
   return m;
 }
 
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, int64_t ld,
-                                                   const int32_t* __restrict__ cu, int batch, int64_t total,
-                                                   int h_kv, int n_init, int n_local, int top_k, int n_sel,
-                                                   int cand_cap, int32_t* __restrict__ out_idx) {
-  extern __shared__ uint32_t sel_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
-  uint32_t* keys = sel_smem + warp * (cand_cap + kHistBins);
-  int* hist = reinterpret_cast<int*>(keys + cand_cap);
-
-  const int64_t unit = static_cast<int64_t>(blockIdx.x) * wpb + warp;
-  if (unit >= static_cast<int64_t>(h_kv) * total) return;
-  const int g = static_cast<int>(unit / total);
-  const int64_t row = unit - static_cast<int64_t>(g) * total;
-  const int s = find_sequence(cu, batch, row);
-  const int t = static_cast<int>(row - cu[s]);
-  const int b_t = t / 64;
-  int32_t* out = out_idx + unit * n_sel;
-
-  const int init_hi = min(n_init, b_t + 1);          // INIT  = [0, init_hi)
-  const int loc_lo = max(0, b_t - n_local + 1);      // LOCAL = [loc_lo, b_t]
-  const int cand_lo = init_hi;
-  const int ncand = max(0, loc_lo - init_hi);        // CAND  = [init_hi, loc_lo)
-
-  if (ncand <= top_k) {
-    // every causal block is taken
-    for (int i = lane; i < n_sel; i += 32) out[i] = (i <= b_t) ? i : -1;
-    return;
-  }
-  if (ncand > cand_cap) {  // host sizes cand_cap from max_seqlen; never expected
-    if (lane == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
-    return;
-  }
-
-  // 1. block scores of the candidates
-  const float* srow = S + (static_cast<int64_t>(g) * total + row) * ld;
-  const int n1 = visible_windows_dev(t, 32, 16);
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = lane; i < ncand; i += 32) {
-    const float sc = fmaxf(block_score(srow, cand_lo + i, n1), 0.f);
-    const uint32_t k = __float_as_uint(sc);
-    keys[i] = k;
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
-  }
+// Writes the selected block list of one query row, given the candidates'
+// keys (bit patterns of non-negative scores, candidate i is block
+// cand_lo + i) in this warp's shared memory, each lane's partial min / max of
+// the keys (reduced over the warp here), and the init / local
+// ranges.  Shared by the prefill and decode selections.
+__device__ __noinline__ void warp_select_write(uint32_t* keys, int* hist, int ncand, int cand_lo, int init_hi,
+                                               int loc_lo, int b_t, int top_k, int n_sel, uint32_t kmin,
+                                               uint32_t kmax, int32_t* out, int lane) {
   kmin = warp_min_u32(kmin);
   kmax = warp_max_u32(kmax);
   __syncwarp();
@@ -169,6 +132,54 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
   for (int i = lane; i < nloc; i += 32) out[pos + i] = loc_lo + i;
   pos += nloc;
   for (int i = pos + lane; i < n_sel; i += 32) out[i] = -1;
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, int64_t ld,
+                                                   const int32_t* __restrict__ cu, int batch, int64_t total,
+                                                   int h_kv, int n_init, int n_local, int top_k, int n_sel,
+                                                   int cand_cap, int32_t* __restrict__ out_idx) {
+  extern __shared__ uint32_t sel_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  uint32_t* keys = sel_smem + warp * (cand_cap + kHistBins);
+  int* hist = reinterpret_cast<int*>(keys + cand_cap);
+
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * wpb + warp;
+  if (unit >= static_cast<int64_t>(h_kv) * total) return;
+  const int g = static_cast<int>(unit / total);
+  const int64_t row = unit - static_cast<int64_t>(g) * total;
+  const int s = find_sequence(cu, batch, row);
+  const int t = static_cast<int>(row - cu[s]);
+  const int b_t = t / 64;
+  int32_t* out = out_idx + unit * n_sel;
+
+  const int init_hi = min(n_init, b_t + 1);          // INIT  = [0, init_hi)
+  const int loc_lo = max(0, b_t - n_local + 1);      // LOCAL = [loc_lo, b_t]
+  const int cand_lo = init_hi;
+  const int ncand = max(0, loc_lo - init_hi);        // CAND  = [init_hi, loc_lo)
+
+  if (ncand <= top_k) {
+    // every causal block is taken
+    for (int i = lane; i < n_sel; i += 32) out[i] = (i <= b_t) ? i : -1;
+    return;
+  }
+  if (ncand > cand_cap) {  // host sizes cand_cap from max_seqlen; never expected
+    if (lane == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    return;
+  }
+
+  // 1. block scores of the candidates
+  const float* srow = S + (static_cast<int64_t>(g) * total + row) * ld;
+  const int n1 = visible_windows_dev(t, 32, 16);
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int i = lane; i < ncand; i += 32) {
+    const float sc = fmaxf(block_score(srow, cand_lo + i, n1), 0.f);
+    const uint32_t k = __float_as_uint(sc);
+    keys[i] = k;
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+  warp_select_write(keys, hist, ncand, cand_lo, init_hi, loc_lo, b_t, top_k, n_sel, kmin, kmax, out, lane);
 }
 
 }  // namespace sel
