@@ -246,9 +246,10 @@ def bench_decode(T, gen, torch, dev, graph_steps: int = 64, reps: int = 3):
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        g.replay()
-        b.record(stream)
+        with torch.cuda.stream(stream):          # replay and both events on the same stream
+            a.record(stream)
+            g.replay()
+            b.record(stream)
         b.synchronize()
         times.append(a.elapsed_time(b))
     status = T.infllm2_get_device_status()
@@ -273,6 +274,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
+    ap.add_argument("--decode-steps", type=int, default=64)
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -311,6 +314,12 @@ def main():
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
     T.lib()
+
+    if args.decode_only:
+        dd = bench_decode(T, gen, torch, dev, graph_steps=args.decode_steps)
+        if rank == 0:
+            print(json.dumps({"decode": dd}), flush=True)
+        return
 
     data = gen.make_prefill(w)
     p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
@@ -443,7 +452,7 @@ def main():
         "device_status": status,
     }
     if not args.no_decode:
-        dd = bench_decode(T, gen, torch, dev)
+        dd = bench_decode(T, gen, torch, dev, graph_steps=args.decode_steps)
         dd["peak_GB/s"] = hbm
         dd["frac"] = dd["achieved_GB/s"] / hbm
         dd["bound"] = "hbm"
