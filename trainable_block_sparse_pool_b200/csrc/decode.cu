@@ -77,6 +77,27 @@ __device__ __forceinline__ void scores_16x8(float (&c)[4], const QFrag<D>& f, co
   }
 }
 
+// Same product as scores_16x8, with the key row already loaded into
+// registers (so a warp can issue every load it needs before the first MMA).
+template <int D>
+__device__ __forceinline__ void load_krow(uint4 (&kv)[D / 32], const __nv_bfloat16* row, int lane) {
+  const int tig = lane & 3;
+#pragma unroll
+  for (int p = 0; p < D / 32; ++p)
+    kv[p] = row ? *reinterpret_cast<const uint4*>(row + 32 * p + 8 * tig) : make_uint4(0, 0, 0, 0);
+}
+template <int D>
+__device__ __forceinline__ void scores_16x8_reg(float (&c)[4], const QFrag<D>& f, const uint4 (&kv)[D / 32]) {
+  c[0] = c[1] = c[2] = c[3] = 0.f;
+#pragma unroll
+  for (int p = 0; p < D / 32; ++p) {
+    const uint32_t a0[4] = {f.lo[p].x, f.hi[p].x, f.lo[p].y, f.hi[p].y};
+    mma16816(c, a0, kv[p].x, kv[p].y);
+    const uint32_t a1[4] = {f.lo[p].z, f.hi[p].z, f.lo[p].w, f.hi[p].w};
+    mma16816(c, a1, kv[p].z, kv[p].w);
+  }
+}
+
 // ---------------------------------------------------------------- A: append + pool
 template <int D>
 __global__ void __launch_bounds__(128) append_kernel(const __nv_bfloat16* __restrict__ k_new,
@@ -172,12 +193,20 @@ __global__ void __launch_bounds__(128) lse_kernel(const __nv_bfloat16* __restric
   const float cs = scale * kLog2e;
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // heads gid, gid+8
   const __nv_bfloat16* base = kc2 + static_cast<int64_t>(bg) * cap_c2 * D;
-  for (int nt = warp; nt < kLseWin / 8; nt += 4) {
+  constexpr int kMaxNt = kLseWin / 8 / 4;
+  uint4 kv[kMaxNt][D / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxNt; ++i) {
+    const int wr = c * kLseWin + (warp + 4 * i) * 8 + gid;
+    load_krow<D>(kv[i], (wr < n2) ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+  }
+#pragma unroll
+  for (int i = 0; i < kMaxNt; ++i) {
+    const int nt = warp + 4 * i;
     const int w0 = c * kLseWin + nt * 8;
     if (w0 >= n2) break;
-    const int wr = w0 + gid;
     float sc[4];
-    scores_16x8<D>(sc, f, (wr < n2) ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+    scores_16x8_reg<D>(sc, f, kv[i]);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       float x0 = (w0 + 2 * tig < n2) ? sc[2 * r] * cs : -INFINITY;
@@ -276,11 +305,23 @@ __global__ void __launch_bounds__(256) score_pool_kernel(
   QFrag<D> f;
   load_qfrag<D>(f, qh, lane, G);
   const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
-  for (int nt = warp; nt * 8 < kScoreWin + 1; nt += 8) {
+  // this warp's n-tiles are nt = warp + 8 i (i < 5): issue every load first
+  constexpr int kMaxNt = (kScoreWin / 8 + 1 + 7) / 8;
+  uint4 kv[kMaxNt][D / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxNt; ++i) {
+    const int nt = warp + 8 * i;
+    const int wr = j0 + nt * 8 + gid;
+    const bool ok = (nt * 8 < kScoreWin + 1) && wr >= 0 && wr < n1;
+    load_krow<D>(kv[i], ok ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+  }
+#pragma unroll
+  for (int i = 0; i < kMaxNt; ++i) {
+    const int nt = warp + 8 * i;
+    if (nt * 8 >= kScoreWin + 1) break;
     const int w0 = j0 + nt * 8;
-    const int wr = w0 + gid;
     float sc[4];
-    scores_16x8<D>(sc, f, (wr >= 0 && wr < n1) ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+    scores_16x8_reg<D>(sc, f, kv[i]);
     // head-group sum for keys 2tig and 2tig+1: two heads here, the other 14 on the lanes with the same tig
     float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
     float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
@@ -310,13 +351,23 @@ __global__ void __launch_bounds__(256) score_pool_kernel(
 }
 
 // ---------------------------------------------------------------- D: top-k per (sequence, group)
-__global__ void __launch_bounds__(32) select_kernel(const float* __restrict__ bscore, const int32_t* __restrict__ seq_len,
-                                                    int h_kv, int nblk_cap, int cand_cap, int n_init, int n_local,
-                                                    int top_k, int n_sel, int32_t* __restrict__ idx) {
+// One CTA of kSelThreads per (sequence, kv group): the same exact radix
+// select as the prefill top-k (8-bit digits of score - min, ties to the
+// lower block), but the candidates are spread over all threads, so the
+// latency of a single row is short.
+constexpr int kSelThreads = 256;
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ bscore,
+                                                             const int32_t* __restrict__ seq_len, int h_kv,
+                                                             int nblk_cap, int cand_cap, int n_init, int n_local,
+                                                             int top_k, int n_sel, int32_t* __restrict__ idx) {
   extern __shared__ uint32_t dsel_smem[];
-  uint32_t* keys = dsel_smem;
-  int* hist = reinterpret_cast<int*>(keys + cand_cap);
-  const int bg = blockIdx.x, lane = threadIdx.x;
+  uint32_t* keys = dsel_smem;                                   // [cand_cap]
+  __shared__ int hist[256];
+  __shared__ uint32_t s_red[2][kSelThreads / 32];
+  __shared__ int s_digit, s_above, s_wsum[kSelThreads / 32], s_wsum2[kSelThreads / 32];
+  const int bg = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = kSelThreads / 32;
   const int b = bg / h_kv;
   const int t = seq_len[b];
   const int b_t = t / 64;
@@ -325,50 +376,163 @@ __global__ void __launch_bounds__(32) select_kernel(const float* __restrict__ bs
   const int loc_lo = max(0, b_t - n_local + 1);
   const int ncand = max(0, loc_lo - init_hi);
   if (ncand <= top_k) {
-    for (int i = lane; i < n_sel; i += 32) out[i] = (i <= b_t) ? i : -1;
+    for (int i = tid; i < n_sel; i += kSelThreads) out[i] = (i <= b_t) ? i : -1;
     return;
   }
   if (ncand > cand_cap || init_hi + ncand > nblk_cap) {
-    if (lane == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    if (tid == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
     return;
   }
   const float* row = bscore + static_cast<int64_t>(bg) * nblk_cap;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = lane; i < ncand; i += 32) {
+  for (int i = tid; i < ncand; i += kSelThreads) {
     const uint32_t k = __float_as_uint(fmaxf(row[init_hi + i], 0.f));
     keys[i] = k;
     kmin = min(kmin, k);
     kmax = max(kmax, k);
   }
-  sel::warp_select_write(keys, hist, ncand, init_hi, init_hi, loc_lo, b_t, top_k, n_sel, kmin, kmax, out, lane);
+  kmin = sel::warp_min_u32(kmin);
+  kmax = sel::warp_max_u32(kmax);
+  if (lane == 0) { s_red[0][warp] = kmin; s_red[1][warp] = kmax; }
+  __syncthreads();
+  kmin = 0xffffffffu; kmax = 0u;
+  for (int w = 0; w < NW; ++w) { kmin = min(kmin, s_red[0][w]); kmax = max(kmax, s_red[1][w]); }
+  const uint32_t range = kmax - kmin;
+  int hi = range ? 32 - __clz(range) : 0;
+  uint32_t prefix = 0;
+  int k_rem = top_k;
+  while (hi > 0) {
+    const int shift = max(0, hi - 8);
+    const int nb = 1 << (hi - shift);
+    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    const uint64_t want = static_cast<uint64_t>(prefix) >> hi;
+    for (int i = tid; i < ncand; i += kSelThreads) {
+      const uint32_t u = keys[i] - kmin;
+      if ((static_cast<uint64_t>(u) >> hi) == want) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int lsum = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) lsum += (lane * 8 + q < nb) ? hist[lane * 8 + q] : 0;
+      int suf = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += v;
+      }
+      int above = suf - lsum;
+      int digit = -1, above_digit = 0;
+      if (above < k_rem && suf >= k_rem) {
+        for (int q = 7; q >= 0; --q) {
+          const int bb = lane * 8 + q;
+          const int hh = (bb < nb) ? hist[bb] : 0;
+          if (above + hh >= k_rem) { digit = bb; above_digit = above; break; }
+          above += hh;
+        }
+      }
+      if (digit >= 0) { s_digit = digit; s_above = above_digit; }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(s_digit) << shift;
+    k_rem -= s_above;
+    hi = shift;
+    __syncthreads();
+  }
+  const uint32_t T = kmin + prefix;
+  // ordered output: INIT, chosen candidates ascending, LOCAL, padding
+  for (int i = tid; i < init_hi; i += kSelThreads) out[i] = i;
+  int pos = init_hi, eq_seen = 0;
+  for (int base = 0; base < ncand; base += kSelThreads) {
+    const int i = base + tid;
+    const bool valid = i < ncand;
+    const uint32_t k = valid ? keys[i] : 0u;
+    const bool gt = valid && k > T, eq = valid && k == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) s_wsum[warp] = __popc(eqm);
+    __syncthreads();
+    int eq_before = eq_seen;
+    for (int w = 0; w < warp; ++w) eq_before += s_wsum[w];
+    int eq_tot = 0;
+    for (int w = 0; w < NW; ++w) eq_tot += s_wsum[w];
+    const bool take = gt || (eq && eq_before + __popc(eqm & lanemask_lt()) < k_rem);
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (lane == 0) s_wsum2[warp] = __popc(tm);
+    __syncthreads();
+    int take_before = pos;
+    for (int w = 0; w < warp; ++w) take_before += s_wsum2[w];
+    int take_tot = 0;
+    for (int w = 0; w < NW; ++w) take_tot += s_wsum2[w];
+    if (take) out[take_before + __popc(tm & lanemask_lt())] = init_hi + i;
+    pos += take_tot;
+    eq_seen += eq_tot;
+    __syncthreads();
+  }
+  const int nloc = b_t - loc_lo + 1;
+  for (int i = tid; i < nloc; i += kSelThreads) out[pos + i] = loc_lo + i;
+  pos += nloc;
+  for (int i = pos + tid; i < n_sel; i += kSelThreads) out[i] = -1;
 }
 
 // ---------------------------------------------------------------- F: combine + advance
+// grid (batch*h_kv, G), D threads: one (sequence, group, head) per CTA.  The
+// split weights 2^(m_s - M) are computed once in shared memory, then each
+// thread folds its column of d over the splits (coalesced across threads).
 template <int D>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int nsplit, int h_q, int h_kv,
-                                                      __nv_bfloat16* __restrict__ out, int32_t* __restrict__ seq_len) {
-  const int bg = blockIdx.x;
+__global__ void __launch_bounds__(D) combine_kernel(const float* __restrict__ part, int nsplit, int h_q, int h_kv,
+                                                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ seq_len) {
+  extern __shared__ float cw[];           // [nsplit] weights
+  __shared__ float red[D / 32];
+  __shared__ float s_M, s_L;
+  const int bg = blockIdx.x, h = blockIdx.y;
   const int b = bg / h_kv, g = bg % h_kv;
-  const int G = h_q / h_kv;
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int h = i / D, dd = i % D;
+  const int G = gridDim.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* base = part + (static_cast<int64_t>(bg) * nsplit * G + h) * (D + 2);
+  const int64_t sstride = static_cast<int64_t>(G) * (D + 2);
+  float m = -INFINITY;
+  for (int s2 = tid; s2 < nsplit; s2 += D) m = fmaxf(m, base[s2 * sstride + D]);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (tid == 0) {
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part[((static_cast<int64_t>(bg) * nsplit + s) * G + h) * (D + 2) + D]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < nsplit; ++s) {
-        const float* p = part + ((static_cast<int64_t>(bg) * nsplit + s) * G + h) * (D + 2);
-        const float m = p[D];
-        if (m == -INFINITY) continue;
-        const float w = ex2(m - M);
-        L += p[D + 1] * w;
-        O += p[dd] * w;
-      }
-    }
-    out[(static_cast<int64_t>(b) * h_q + g * G + h) * D + dd] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    s_M = M;
   }
   __syncthreads();
-  if (g == 0 && threadIdx.x == 0) seq_len[b] = seq_len[b] + 1;
+  const float M = s_M;
+  float l = 0.f;
+  for (int s2 = tid; s2 < nsplit; s2 += D) {
+    const float ms = base[s2 * sstride + D];
+    const float wgt = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
+    cw[s2] = wgt;
+    l += base[s2 * sstride + D + 1] * wgt;
+  }
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = l;
+  __syncthreads();
+  if (tid == 0) {
+    float L = 0.f;
+    for (int w = 0; w < D / 32; ++w) L += red[w];
+    s_L = L;
+  }
+  __syncthreads();
+  float o = 0.f;
+  for (int s2 = 0; s2 < nsplit; ++s2) {
+    const float wgt = cw[s2];
+    if (wgt != 0.f) o += base[s2 * sstride + tid] * wgt;
+  }
+  const float L = s_L;
+  out[(static_cast<int64_t>(b) * h_q + g * G + h) * D + tid] = __float2bfloat16_rn(L > 0.f ? o / L : 0.f);
+}
+
+// seq_len[b] += 1 once every kernel of the step has read it
+__global__ void advance_kernel(int32_t* __restrict__ seq_len, int batch) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < batch) seq_len[b] = seq_len[b] + 1;
 }
 
 // ---------------------------------------------------------------- pooled caches of a prefix
@@ -498,18 +662,20 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
   dec::score_pool_kernel<D><<<dim3(bg, P.nsplit1), 256, 0, st>>>(
       static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->h_q, s->h_kv,
       P.cap_c1, P.nblk_cap, scale, bscore);
-  const size_t sel_smem = (static_cast<size_t>(P.cand_cap) + sel::kHistBins) * 4;
+  const size_t sel_smem = static_cast<size_t>(P.cand_cap) * 4;
   cudaError_t e = cudaFuncSetAttribute(dec::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sel_smem));
   if (e != cudaSuccess) return e;
-  dec::select_kernel<<<bg, 32, sel_smem, st>>>(bscore, s->seq_len, s->h_kv, P.nblk_cap, P.cand_cap, n_init, n_local,
-                                               top_k, P.n_sel, idx);
+  dec::select_kernel<<<bg, dec::kSelThreads, sel_smem, st>>>(bscore, s->seq_len, s->h_kv, P.nblk_cap, P.cand_cap,
+                                                             n_init, n_local, top_k, P.n_sel, idx);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_sparse_decode(q, s->k_cache, s->v_cache, idx, s->seq_len, s->batch, s->capacity, s->h_q, s->h_kv, D,
                            P.n_sel, P.nsplit, P.bps, scale, part, st, map_fail);
   if (e != cudaSuccess) return e;
-  dec::combine_kernel<D><<<bg, 256, 0, st>>>(part, P.nsplit, s->h_q, s->h_kv, static_cast<bf*>(out), s->seq_len);
+  dec::combine_kernel<D><<<dim3(bg, s->h_q / s->h_kv), D, P.nsplit * sizeof(float), st>>>(
+      part, P.nsplit, s->h_q, s->h_kv, static_cast<bf*>(out), s->seq_len);
+  dec::advance_kernel<<<(s->batch + 127) / 128, 128, 0, st>>>(s->seq_len, s->batch);
   return cudaGetLastError();
 }
 

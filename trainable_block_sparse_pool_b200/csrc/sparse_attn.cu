@@ -35,7 +35,8 @@ namespace infllm2 {
 namespace sparse {
 
 constexpr int kNumWG = 2;
-constexpr int kThreads = 64 + 128 * kNumWG + 32 * kNumWG;   // producer, QK, softmax groups, PV issuers
+constexpr int kThreads = 64 + 128 * kNumWG + 32 * kNumWG + 32;   // K producer, QK, softmax groups, PV issuers, V producer
+constexpr int kVWarp = 2 + 5 * kNumWG;   // the V producer
 constexpr int kPairKeys = 128;       // keys per tile (two 64-key blocks)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.f;      // raise m_ref only past this margin (log2 units)
@@ -46,7 +47,7 @@ struct Cfg {
   static constexpr uint32_t kChunk = kPairKeys * 128;         // 16 KB: 128 keys x 64 dims
   static constexpr uint32_t kHalf = 64 * 128;                 // one block inside a chunk
   static constexpr uint32_t kKBytes = kChunk * KCH;
-  static constexpr uint32_t kStageBytes = 2 * kKBytes;        // K then V
+  static constexpr uint32_t kStageBytes = 2 * kKBytes;        // one K slot plus one V slot
   static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr uint32_t kQBuf = 2048 * KCH;               // 16 head rows x d
   static constexpr uint32_t kPBuf = kPairKeys * 16 * 2;       // 4 KB
@@ -56,8 +57,10 @@ struct Cfg {
 };
 
 struct Bars {
-  uint64_t kv_full[8];
-  uint64_t kv_empty[8];
+  uint64_t k_full[8];     // K ring: filled by the K producer, freed when the QK product completes
+  uint64_t k_empty[8];
+  uint64_t v_full[8];     // V ring: filled by the V producer, freed when the PV product completes
+  uint64_t v_empty[8];
   uint64_t q_full[kNumWG][2];
   uint64_t q_empty[kNumWG][2];
   uint64_t s_full[kNumWG][2];
@@ -210,6 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem;
+  uint8_t* sKr = sKV;                                                  // K ring [kStages][kKBytes]
+  uint8_t* sVr = sKV + C::kStages * C::kKBytes;                        // V ring [kStages][kKBytes]
   uint8_t* sQ = sKV + C::kStages * C::kStageBytes;                    // [wg][2]
   uint8_t* sP = sQ + kNumWG * 2 * C::kQBuf;                           // [wg][2]
   float* red = reinterpret_cast<float*>(sP + kNumWG * 2 * C::kPBuf);  // [wg][4][16]
@@ -224,7 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);   // head rows past G stay zero
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
+    }
     for (int w = 0; w < kNumWG; ++w)
       for (int i = 0; i < 2; ++i) {
         mbar_init(&bars->q_full[w][i], 1);
@@ -246,11 +256,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
   const uint32_t tmem = bars->tmem_base;
   // TMEM columns of group w: S buffers at w*64 + {0,16}, O buffers at w*64 + {32,48}
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // The whole warp walks the units (their block lists live in its
-    // registers); lane 0 waits and issues the copies.
-    if (lane == 0) { tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV); }
+  if (warp == 0 || warp == kVWarp) {
+    // ------------------------------------------------------------ producers
+    // Warp 0 loads Q and the K ring, warp kVWarp the V ring; both walk the
+    // same stream of tiles.  The whole warp walks the units (their block
+    // lists live in its registers); lane 0 waits and issues the copies.
+    const bool isV = (warp == kVWarp);
+    const CUtensorMap* tm = isV ? &tmV : &tmK;
+    uint8_t* ring = isV ? sVr : sKr;
+    uint64_t* full = isV ? bars->v_full : bars->k_full;
+    uint64_t* empty = isV ? bars->v_empty : bars->k_empty;
+    if (lane == 0) { tma_prefetch_desc(&tmQ); tma_prefetch_desc(tm); }
     int it = 0;
     int ucnt[kNumWG] = {0, 0};
     bool ok = true;
@@ -265,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         nt[w] = ntiles_of(x[w]);
         Le[w] = load_warp_list(x[w].I, x[w].nvalid, 0, lane);
         Lo[w] = load_warp_list(x[w].I, x[w].nvalid, 1, lane);
+        if (isV) continue;
         const int qb = ucnt[w] & 1;
         int good = 1;
         if (lane == 0) {
@@ -291,17 +308,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
           const int st = it % C::kStages;
           int good = 1;
           if (lane == 0) {
-            good = mbar_wait(&bars->kv_empty[st], ((it / C::kStages) & 1) ^ 1) && !aborted(bars);
+            good = mbar_wait(&empty[st], ((it / C::kStages) & 1) ^ 1) && !aborted(bars);
             if (good) {
-              uint8_t* dK = sKV + st * C::kStageBytes;
-              uint8_t* dV = dK + C::kKBytes;
-              mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
+              uint8_t* dst = ring + st * C::kKBytes;
+              mbar_arrive_expect_tx(&full[st], C::kKBytes);
               for (int ch = 0; ch < C::KCH; ++ch) {
-                tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
-                tma_load_3d(dK + ch * C::kChunk + C::kHalf, &tmK, &bars->kv_full[st], ch * 64, x[w].g,
-                            x[w].seq_start + 64 * b1);
-                tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
-                tma_load_3d(dV + ch * C::kChunk + C::kHalf, &tmV, &bars->kv_full[st], ch * 64, x[w].g,
+                tma_load_3d(dst + ch * C::kChunk, tm, &full[st], ch * 64, x[w].g, x[w].seq_start + 64 * b0);
+                tma_load_3d(dst + ch * C::kChunk + C::kHalf, tm, &full[st], ch * 64, x[w].g,
                             x[w].seq_start + 64 * b1);
               }
             } else {
@@ -315,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     }
     // wait for every copy still in flight before the CTA may exit
     if (lane == 0) {
-      for (int i = max(0, it - C::kStages); i < it; ++i)
-        mbar_wait(&bars->kv_full[i % C::kStages], (i / C::kStages) & 1);
-      for (int w = 0; w < kNumWG; ++w)
-        for (int i = max(0, ucnt[w] - 2); i < ucnt[w]; ++i) mbar_wait(&bars->q_full[w][i & 1], (i >> 1) & 1);
+      for (int i = max(0, it - C::kStages); i < it; ++i) mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
+      if (!isV)
+        for (int w = 0; w < kNumWG; ++w)
+          for (int i = max(0, ucnt[w] - 2); i < ucnt[w]; ++i) mbar_wait(&bars->q_full[w][i & 1], (i >> 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
@@ -347,12 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
             if (j >= nt[w]) continue;
             const int st = it % C::kStages;
             const int sb = tcnt[w] & 1;
-            if (!mbar_wait(&bars->kv_full[st], (it / C::kStages) & 1) ||
+            if (!mbar_wait(&bars->k_full[st], (it / C::kStages) & 1) ||
                 !mbar_wait(&bars->s_empty[w][sb], ((tcnt[w] >> 1) & 1) ^ 1) || aborted(bars)) {
               set_abort(bars); ok = false; break;
             }
             tc_fence_after();
-            const uint32_t k_base = smem_u32(sKV + st * C::kStageBytes);
+            const uint32_t k_base = smem_u32(sKr + st * C::kKBytes);
             const uint32_t q_base = smem_u32(sQ + (w * 2 + qb[w]) * C::kQBuf);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
@@ -361,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
               umma_bf16(tmem + w * 64 + sb * 16, a, b, idS, k > 0);
             }
             umma_commit(&bars->s_full[w][sb]);
+            umma_commit(&bars->k_empty[st]);        // K slot free once this product completes
             if (j == nt[w] - 1) umma_commit(&bars->q_empty[w][qb[w]]);
             ++tcnt[w];
             ++it;
@@ -370,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       umma_commit(&bars->mma_done[0]);
       mbar_wait(&bars->mma_done[0], 0);
     }
-  } else if (warp >= 2 + 4 * kNumWG) {
+  } else if (warp >= 2 + 4 * kNumWG && warp < kVWarp) {
     // ------------------------------------------------------------ PV issuers
     // One warp per softmax group: the group's PV products in order, each as
     // soon as its P is in shared memory.  The stream is replayed to find
@@ -400,11 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
             if (w == pw) {
               const int st = it % C::kStages;
               const int pb = tcnt & 1;
-              if (!mbar_wait(&bars->p_full[pw][pb], (tcnt >> 1) & 1) || aborted(bars)) {
+              if (!mbar_wait(&bars->p_full[pw][pb], (tcnt >> 1) & 1) ||
+                  !mbar_wait(&bars->v_full[st], (it / C::kStages) & 1) || aborted(bars)) {
                 set_abort(bars); ok = false; break;
               }
               tc_fence_after();
-              const uint32_t v_base = smem_u32(sKV + st * C::kStageBytes + C::kKBytes);
+              const uint32_t v_base = smem_u32(sVr + st * C::kKBytes);
               const uint32_t p_base = smem_u32(sP + (pw * 2 + pb) * C::kPBuf);
               const uint32_t o_addr = tmem + pw * 64 + 32 + obuf * 16;
 #pragma unroll
@@ -413,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
                 const uint64_t b = make_sdesc(p_base + k * 512, 256, 128, kLayoutNone);
                 umma_bf16(o_addr, a, b, idO, (j == 0 && k == 0) ? 0u : 1u);
               }
-              umma_commit(&bars->kv_empty[st]);
+              umma_commit(&bars->v_empty[st]);
               umma_commit(&bars->pv_done[pw][pb]);
               ++tcnt;
             }
