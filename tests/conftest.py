@@ -24,3 +24,16 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _fresh_device_status(request):
+    """The library's device status word is sticky (the first error wins), so
+    every GPU test starts from a cleared word: one failing test must not
+    fail the ones after it."""
+    if "gpu" in request.keywords:
+        import torch
+        import trainable_block_sparse_pool_b200 as T
+        torch.cuda.synchronize()
+        T.infllm2_clear_device_status()
+    yield

@@ -26,6 +26,10 @@ class DecodeRun:
         self.v_cache = torch.zeros_like(self.k_cache)
         self.k_cache[:, :prefix] = self.data["K"][:, :prefix].to(dev)
         self.v_cache[:, :prefix] = self.data["V"][:, :prefix].to(dev)
+        # rows past the prefix are not written yet: NaN there must never
+        # reach an output (they are appended one per step)
+        self.k_cache[:, prefix:] = float("nan")
+        self.v_cache[:, prefix:] = float("nan")
         self.kc1 = torch.zeros(batch, w.h_kv, max(1, T.window_count(cap, 32, 16)), w.d, dtype=torch.bfloat16, device=dev)
         self.kc2 = torch.zeros(batch, w.h_kv, max(1, T.window_count(cap, 128, 64)), w.d, dtype=torch.bfloat16, device=dev)
         self.seq_len = torch.full((batch,), prefix, dtype=torch.int32, device=dev)

@@ -13,12 +13,13 @@
 //      max-pool to block scores, split over CTAs (each CTA keeps one window
 //      of halo so blocks never straddle CTAs)
 //   D  top-k selection per (sequence, kv group)
-//   E  split-KV block-sparse attention: the prefill sparse kernel in its
-//      partial-output mode (sparse_attn.cu)
+//   E  split-KV block-sparse attention over the selected blocks, one
+//      partial (unnormalised O, max, sum) per split
 //   F  combine the splits, write the output, advance seq_len
 // All of it is HBM-bound (the pooled keys and the selected K/V are read
-// once); the tiny contractions of B and C (16 heads against 8 windows per
-// instruction) use warp-level mma.sync, which is far from being the limit.
+// once); the small contractions of B, C and E (16 heads against 8 keys or
+// windows per instruction) use warp-level mma.sync, which is far from being
+// the limit.
 #include "sm100.cuh"
 
 namespace infllm2 {
@@ -273,6 +274,17 @@ __global__ void __launch_bounds__(256) score_pool_kernel(
   const float cs = scale * kLog2e;
   const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
   const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
+  // this warp's n-tiles are nt = warp + 8 i (i < 5): issue every load first
+  constexpr int kMaxNt = (kScoreWin / 8 + 1 + 7) / 8;
+  uint4 kv[kMaxNt][D / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxNt; ++i) {
+    const int nt = warp + 8 * i;
+    const int wr = j0 + nt * 8 + gid;
+    const bool ok = (nt * 8 < kScoreWin + 1) && wr >= 0 && wr < n1;
+    load_krow<D>(kv[i], ok ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+  }
+  // the per-head LSE (coarse partials combined) while the loads are in flight
   if (threadIdx.x < 16) {
     const int h = threadIdx.x;
     float mm = -INFINITY, ll = 0.f;
@@ -301,20 +313,10 @@ __global__ void __launch_bounds__(256) score_pool_kernel(
     }
     nlse[h] = (h < G && ll > 0.f) ? -(mm + log2f(ll)) : -INFINITY;
   }
-  __syncthreads();
   QFrag<D> f;
   load_qfrag<D>(f, qh, lane, G);
+  __syncthreads();
   const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
-  // this warp's n-tiles are nt = warp + 8 i (i < 5): issue every load first
-  constexpr int kMaxNt = (kScoreWin / 8 + 1 + 7) / 8;
-  uint4 kv[kMaxNt][D / 32];
-#pragma unroll
-  for (int i = 0; i < kMaxNt; ++i) {
-    const int nt = warp + 8 * i;
-    const int wr = j0 + nt * 8 + gid;
-    const bool ok = (nt * 8 < kScoreWin + 1) && wr >= 0 && wr < n1;
-    load_krow<D>(kv[i], ok ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
-  }
 #pragma unroll
   for (int i = 0; i < kMaxNt; ++i) {
     const int nt = warp + 8 * i;
@@ -475,6 +477,262 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   for (int i = pos + tid; i < n_sel; i += kSelThreads) out[i] = -1;
 }
 
+// ---------------------------------------------------------------- E: split-KV sparse attention
+// grid (batch*h_kv, nsplit), kAttWarps warps.  CTA (bg, sp) covers the
+// entries [sp*bps, sp*bps + bps) of the block list of (sequence b, group g);
+// each entry is two 32-key chunks, and warp w takes chunks w, w + kAttWarps, ...
+// Per chunk the warp stages K and V (cp.async, 16 B pieces, 16-byte
+// chunks of a key row XOR-swizzled by the row index so ldmatrix is free of
+// bank conflicts), then
+//   S[16 heads, 32 keys] = Q . K^T     (mma.sync m16n8k16, K via ldmatrix)
+//   online softmax in log2 units (running max m, sum l per head)
+//   O[16, D] += P . V                  (P re-used from the S fragments,
+//                                        V via ldmatrix.trans)
+// The next chunk's K is issued as soon as S is done and its V as soon as
+// the PV product is done, so every warp keeps a copy in flight.  The warps'
+// (m, l, O) are merged in shared memory and written as one partial
+// (unnormalised O, m, l) per CTA for the combine kernel.
+// Keys past t (and chunks of invalid or not-yet-visible blocks) are never
+// read: their staging rows are zero-filled and their scores are -inf.
+constexpr int kAttWarps = 4;
+constexpr int kChunkKeys = 32;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(full ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D>
+struct AttCfg {
+  static constexpr int CH = D / 8;                            // 16-byte pieces per key row
+  static constexpr uint32_t kTile = kChunkKeys * D * 2;       // one K or V chunk
+  static constexpr uint32_t kSmem = kAttWarps * 2 * kTile;    // per-warp K and V buffers
+  static_assert(kAttWarps * 16 * (D + 2) * 4 <= kSmem, "merge area fits in the staging buffers");
+};
+
+template <int D>
+__global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ seq_len, int capacity, int h_q, int h_kv, int n_sel,
+    int bps, float scale, float* __restrict__ part) {
+  using C = AttCfg<D>;
+  extern __shared__ __align__(128) uint8_t att_smem[];
+  const int bg = blockIdx.x, sp = blockIdx.y, nsplit = gridDim.y;
+  const int b = bg / h_kv, g = bg % h_kv;
+  const int G = h_q / h_kv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  // the new token's position; keys 0..t are visible (t is clamped into the
+  // cache, so no address below can leave it)
+  const int t = min(seq_len[b], capacity - 1);
+  const int32_t* list = idx + static_cast<int64_t>(bg) * n_sel + static_cast<int64_t>(sp) * bps;
+  const int nb = max(0, min(bps, n_sel - sp * bps));
+  const int nmine = (2 * nb > warp) ? (2 * nb - 1 - warp) / kAttWarps + 1 : 0;
+  const int64_t kstride = static_cast<int64_t>(h_kv) * D;    // elements from one key row to the next
+  const int64_t row0 = (static_cast<int64_t>(b) * capacity * h_kv + g) * D;
+  const uint32_t sK = smem_u32(att_smem) + warp * 2 * C::kTile;
+  const uint32_t sV = sK + C::kTile;
+
+  // Q of the group's 16 heads (rows >= G are zero) as m16n8k16 A fragments
+  uint32_t qa[D / 16][4];
+  {
+    const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int d0 = 16 * kk + 2 * tig;
+      qa[kk][0] = (gid < G) ? *reinterpret_cast<const uint32_t*>(qh + gid * D + d0) : 0u;
+      qa[kk][1] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qh + (gid + 8) * D + d0) : 0u;
+      qa[kk][2] = (gid < G) ? *reinterpret_cast<const uint32_t*>(qh + gid * D + d0 + 8) : 0u;
+      qa[kk][3] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qh + (gid + 8) * D + d0 + 8) : 0u;
+    }
+  }
+
+  // first key of the warp's i-th chunk, or -1 when it has no visible key
+  auto chunk_key0 = [&](int i) -> int {
+    if (i >= nmine) return -1;
+    const int ch = warp + kAttWarps * i;
+    const int blk = list[ch >> 1];
+    const int k0 = 64 * blk + kChunkKeys * (ch & 1);
+    return (blk >= 0 && blk <= t / 64 && k0 <= t) ? k0 : -1;
+  };
+  auto stage = [&](uint32_t dst, const __nv_bfloat16* cache, int k0) {
+    if (k0 >= 0) {
+#pragma unroll
+      for (int j = 0; j < kChunkKeys * C::CH / 32; ++j) {
+        const int pc = lane + 32 * j;
+        const int r = pc / C::CH, c = pc % C::CH;
+        const bool ok = k0 + r <= t;
+        const __nv_bfloat16* src = cache + row0 + static_cast<int64_t>(ok ? k0 + r : k0) * kstride + c * 8;
+        cp_async16(dst + r * (D * 2) + ((c ^ (r & 7)) << 4), src, ok);
+      }
+    }
+    cp_async_commit();
+  };
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads gid, gid + 8
+  const float cs = scale * kLog2e;
+
+  int k0 = chunk_key0(0);
+  stage(sK, kc, k0);
+  stage(sV, vc, k0);
+  for (int i = 0; i < nmine; ++i) {
+    const int k0n = chunk_key0(i + 1);
+    cp_async_wait1();                        // K of chunk i (its V may still be in flight)
+    __syncwarp();
+    float s[4][4];
+    if (k0 >= 0) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+      for (int p = 0; p < D / 32; ++p) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = 8 * j + (lane & 7), c = 4 * p + (lane >> 3);
+          uint32_t kb[4];
+          ldsm_x4(kb, sK + r * (D * 2) + ((c ^ (r & 7)) << 4));
+          mma16816(s[j], qa[2 * p], kb[0], kb[1]);
+          mma16816(s[j], qa[2 * p + 1], kb[2], kb[3]);
+        }
+      }
+    }
+    __syncwarp();                            // every lane is done with this K buffer
+    stage(sK, kc, k0n);
+    if (k0 >= 0) {
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool ok = k0 + 8 * j + 2 * tig + e <= t;
+          s[j][e] = ok ? s[j][e] * cs : -INFINITY;
+          s[j][2 + e] = ok ? s[j][2 + e] * cs : -INFINITY;
+          mx0 = fmaxf(mx0, s[j][e]);
+          mx1 = fmaxf(mx1, s[j][2 + e]);
+        }
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      // k0 <= t, so key k0 is visible and both maxima are finite
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float a0 = ex2(m0 - mn0), a1 = ex2(m1 - mn1);    // m = -inf: 0
+      m0 = mn0;
+      m1 = mn1;
+      float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          s[j][e] = ex2(s[j][e] - mn0);
+          s[j][2 + e] = ex2(s[j][2 + e] - mn1);
+          ps0 += s[j][e];
+          ps1 += s[j][2 + e];
+        }
+      }
+      l0 = l0 * a0 + ps0;
+      l1 = l1 * a1 + ps1;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o[n][0] *= a0;
+        o[n][1] *= a0;
+        o[n][2] *= a1;
+        o[n][3] *= a1;
+      }
+    }
+    cp_async_wait1();                        // V of chunk i (the next K may still be in flight)
+    __syncwarp();
+    if (k0 >= 0) {
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const uint32_t pa[4] = {pack_bf16(s[2 * s2][0], s[2 * s2][1]), pack_bf16(s[2 * s2][2], s[2 * s2][3]),
+                                pack_bf16(s[2 * s2 + 1][0], s[2 * s2 + 1][1]),
+                                pack_bf16(s[2 * s2 + 1][2], s[2 * s2 + 1][3])};
+#pragma unroll
+        for (int n = 0; n < D / 8; n += 2) {
+          const int r = 16 * s2 + (lane & 7) + ((lane >> 3) & 1) * 8, c = n + (lane >> 4);
+          uint32_t vb[4];
+          ldsm_x4_t(vb, sV + r * (D * 2) + ((c ^ (r & 7)) << 4));
+          mma16816(o[n], pa, vb[0], vb[1]);
+          mma16816(o[n + 1], pa, vb[2], vb[3]);
+        }
+      }
+    }
+    __syncwarp();                            // every lane is done with this V buffer
+    stage(sV, vc, k0n);
+    k0 = k0n;
+  }
+  cp_async_wait0();
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+  // merge the warps: [warp][16 heads][D + 2] in the (now idle) staging buffers
+  __syncthreads();
+  float* mw = reinterpret_cast<float*>(att_smem);
+  {
+    float* r0 = mw + (warp * 16 + gid) * (D + 2);
+    float* r1 = mw + (warp * 16 + gid + 8) * (D + 2);
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      r0[8 * n + 2 * tig] = o[n][0];
+      r0[8 * n + 2 * tig + 1] = o[n][1];
+      r1[8 * n + 2 * tig] = o[n][2];
+      r1[8 * n + 2 * tig + 1] = o[n][3];
+    }
+    if (tig == 0) {
+      r0[D] = m0;
+      r0[D + 1] = l0;
+      r1[D] = m1;
+      r1[D + 1] = l1;
+    }
+  }
+  __syncthreads();
+  float* dst = part + (static_cast<int64_t>(bg) * nsplit + sp) * G * (D + 2);
+  for (int e = threadIdx.x; e < G * (D + 1); e += 32 * kAttWarps) {
+    const int h = e / (D + 1), d = e - h * (D + 1);   // d == D: the row sum
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, mw[(w * 16 + h) * (D + 2) + D]);
+    float acc = 0.f;
+    const int col = (d < D) ? d : D + 1;
+#pragma unroll
+    for (int w = 0; w < kAttWarps; ++w) {
+      const float mwh = mw[(w * 16 + h) * (D + 2) + D];
+      if (mwh != -INFINITY) acc += mw[(w * 16 + h) * (D + 2) + col] * ex2(mwh - M);
+    }
+    if (d < D) {
+      dst[h * (D + 2) + d] = acc;
+    } else {
+      dst[h * (D + 2) + D] = M;
+      dst[h * (D + 2) + D + 1] = acc;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- F: combine + advance
 // grid (batch*h_kv, G), D threads: one (sequence, group, head) per CTA.  The
 // split weights 2^(m_s - M) are computed once in shared memory, then each
@@ -527,12 +785,9 @@ __global__ void __launch_bounds__(D) combine_kernel(const float* __restrict__ pa
   }
   const float L = s_L;
   out[(static_cast<int64_t>(b) * h_q + g * G + h) * D + tid] = __float2bfloat16_rn(L > 0.f ? o / L : 0.f);
-}
-
-// seq_len[b] += 1 once every kernel of the step has read it
-__global__ void advance_kernel(int32_t* __restrict__ seq_len, int batch) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < batch) seq_len[b] = seq_len[b] + 1;
+  // advance the sequence: nothing in this kernel reads seq_len, and every
+  // kernel before it in the step has finished
+  if (g == 0 && h == 0 && tid == 0) seq_len[b] = seq_len[b] + 1;
 }
 
 // ---------------------------------------------------------------- pooled caches of a prefix
@@ -622,11 +877,10 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   p.nsplit2 = std::max(1, (p.cap_c2 + dec::kLseWin - 1) / dec::kLseWin);
   p.nsplit1 = std::max(1, (p.cap_c1 + dec::kScoreWin) / dec::kScoreWin);
   const int bg = batch * h_kv;
-  const int target = std::max(1, (4 * sms + bg - 1) / bg);           // about four units per SM
-  int bps = std::max(2, (n_sel + target - 1) / target);
-  bps = (bps + 1) & ~1;                                               // whole pairs of blocks
-  p.bps = bps;
-  p.nsplit = std::max(1, (n_sel + bps - 1) / bps);
+  // attention splits: about three CTAs of the attention kernel per SM
+  const int per_bg = std::max(1, (3 * sms) / std::max(1, bg));
+  p.bps = std::max(1, (n_sel + per_bg - 1) / per_bg);
+  p.nsplit = std::max(1, (n_sel + p.bps - 1) / p.bps);
   const int G = h_q / h_kv;
   size_t off = 0;
   p.off_part2 = off; off = align256(off + static_cast<size_t>(bg) * p.nsplit2 * 16 * sizeof(float2));
@@ -637,16 +891,13 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   return p;
 }
 
-cudaError_t launch_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* idx,
-                                 const int32_t* seq_len, int batch, int capacity, int h_q, int h_kv, int d,
-                                 int n_sel, int nsplit, int bps, float scale, float* part, cudaStream_t st,
-                                 bool* map_fail);
 
 template <int D>
 static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, const void* k_new, const void* v_new,
                                  void* out, void* ws, const DecodePlan& P, int n_init, int n_local, int top_k,
                                  float scale, cudaStream_t st, bool* map_fail) {
   using bf = __nv_bfloat16;
+  *map_fail = false;                       // the decode step builds no tensor maps
   const int bg = s->batch * s->h_kv;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float2* part2 = reinterpret_cast<float2*>(w + P.off_part2);
@@ -668,14 +919,14 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
   if (e != cudaSuccess) return e;
   dec::select_kernel<<<bg, dec::kSelThreads, sel_smem, st>>>(bscore, s->seq_len, s->h_kv, P.nblk_cap, P.cand_cap,
                                                              n_init, n_local, top_k, P.n_sel, idx);
-  e = cudaGetLastError();
+  e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(dec::AttCfg<D>::kSmem));
   if (e != cudaSuccess) return e;
-  e = launch_sparse_decode(q, s->k_cache, s->v_cache, idx, s->seq_len, s->batch, s->capacity, s->h_q, s->h_kv, D,
-                           P.n_sel, P.nsplit, P.bps, scale, part, st, map_fail);
-  if (e != cudaSuccess) return e;
+  dec::attend_kernel<D><<<dim3(bg, P.nsplit), 32 * dec::kAttWarps, dec::AttCfg<D>::kSmem, st>>>(
+      static_cast<const bf*>(q), static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache), idx,
+      s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps, scale, part);
   dec::combine_kernel<D><<<dim3(bg, s->h_q / s->h_kv), D, P.nsplit * sizeof(float), st>>>(
       part, P.nsplit, s->h_q, s->h_kv, static_cast<bf*>(out), s->seq_len);
-  dec::advance_kernel<<<(s->batch + 127) / 128, 128, 0, st>>>(s->seq_len, s->batch);
   return cudaGetLastError();
 }
 

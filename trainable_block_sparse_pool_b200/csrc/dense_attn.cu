@@ -192,8 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
 #pragma unroll 1
       for (int cc = 0; cc < kKeys; cc += 16) {
         float v[16];
-        tmem_ld16(s_addr + cc, v);
-        tmem_wait_ld16(v);
+        tmem_load16(s_addr + cc, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) if (kbase + cc + i <= t) mx = fmaxf(mx, v[i] * c);
       }
@@ -204,8 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
 #pragma unroll 1
       for (int cc = 0; cc < kKeys; cc += 16) {
         float v[16];
-        tmem_ld16(s_addr + cc, v);
-        tmem_wait_ld16(v);
+        tmem_load16(s_addr + cc, v);
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
@@ -235,8 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
 #pragma unroll
       for (int cc = 0; cc < D; cc += 16) {
         float v[16];
-        tmem_ld16(tmem + lane_addr + C::kOCol + pb * D + cc, v);
-        tmem_wait_ld16(v);
+        tmem_load16(tmem + lane_addr + C::kOCol + pb * D + cc, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) o_acc[cc + i] = fmaf(o_acc[cc + i], alpha, v[i]);
       }

@@ -95,15 +95,6 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
-      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Number of valid (>= 0) entries of a block list, with independent vector
 // loads (lists hold their valid entries first, then -1 padding).
@@ -153,58 +144,36 @@ struct Unit {
   const int32_t* I;
 };
 
-// Where the units come from.  Prefill: unit u = (kv group, packed row),
-// u = g * total + row, its list is block_idx[g, row, :].  Decode (seq_len
-// non-null): unit u = ((b * h_kv + g) * nsplit + sp), one split of the
-// block list of the new token of sequence b; the product is a partial
-// (unnormalised O, reference maximum, row sum) for the combine kernel.
+// Unit u = (kv group, packed row), u = g * total + row; its list is
+// block_idx[g, row, :].
 struct SparseArgs {
   const int32_t* block_idx;
   const int32_t* cu;
   int batch;
-  int64_t total;       // prefill: packed rows; decode: batch (rows of q)
+  int64_t total;       // packed rows
   int h_q, h_kv, n_sel;
   float scale;
   void* out;
-  const int32_t* seq_len;
-  int capacity, nsplit, bps;
-  float* part;         // decode: [units][G][D + 2]
 };
 
-template <bool DEC>
-__device__ __forceinline__ int64_t num_units(const SparseArgs& a) {
-  return DEC ? static_cast<int64_t>(a.batch) * a.h_kv * a.nsplit : static_cast<int64_t>(a.h_kv) * a.total;
-}
+__device__ __forceinline__ int64_t num_units(const SparseArgs& a) { return static_cast<int64_t>(a.h_kv) * a.total; }
 
-template <bool DEC>
 __device__ __forceinline__ Unit get_unit(int64_t u, const SparseArgs& a) {
   Unit x;
-  if (DEC) {
-    const int sp = static_cast<int>(u % a.nsplit);
-    const int bg = static_cast<int>(u / a.nsplit);
-    const int b = bg / a.h_kv;
-    x.g = bg - b * a.h_kv;
-    x.row = b;
-    x.t = a.seq_len[b];
-    x.seq_start = b * a.capacity;
-    x.I = a.block_idx + static_cast<int64_t>(bg) * a.n_sel + sp * a.bps;
-    x.nlist = max(0, min(a.bps, a.n_sel - sp * a.bps));
-  } else {
-    x.g = static_cast<int>(u / a.total);
-    x.row = u - static_cast<int64_t>(x.g) * a.total;
-    const int s = find_sequence(a.cu, a.batch, x.row);
-    x.seq_start = a.cu[s];
-    x.t = static_cast<int>(x.row - x.seq_start);
-    x.I = a.block_idx + u * a.n_sel;
-    x.nlist = a.n_sel;
-  }
+  x.g = static_cast<int>(u / a.total);
+  x.row = u - static_cast<int64_t>(x.g) * a.total;
+  const int s = find_sequence(a.cu, a.batch, x.row);
+  x.seq_start = a.cu[s];
+  x.t = static_cast<int>(x.row - x.seq_start);
+  x.I = a.block_idx + u * a.n_sel;
+  x.nlist = a.n_sel;
   x.nvalid = count_valid(x.I, x.nlist);
   return x;
 }
 
 __device__ __forceinline__ int ntiles_of(const Unit& x) { return (x.nvalid + 1) >> 1; }
 
-template <int D, int G, bool OUT_F32, bool DEC>
+template <int D, int G, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const SparseArgs args) {
@@ -221,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
   Bars* bars = reinterpret_cast<Bars*>(red + kNumWG * 4 * 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n_units = num_units<DEC>(args);
+  const int64_t n_units = num_units(args);
   // units of this CTA: u_k = blockIdx.x + k * gridDim.x; unit k goes to group k & 1
   const int64_t my_units = (n_units > blockIdx.x) ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
@@ -277,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       for (int w = 0; w < kNumWG; ++w) {
         nt[w] = 0;
         if (k0 + w >= my_units) continue;
-        x[w] = get_unit<DEC>(blockIdx.x + (k0 + w) * gridDim.x, args);
+        x[w] = get_unit(blockIdx.x + (k0 + w) * gridDim.x, args);
         nt[w] = ntiles_of(x[w]);
         Le[w] = load_warp_list(x[w].I, x[w].nvalid, 0, lane);
         Lo[w] = load_warp_list(x[w].I, x[w].nvalid, 1, lane);
@@ -347,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         for (int w = 0; w < kNumWG; ++w) {
           nt[w] = 0;
           if (k0 + w >= my_units) continue;
-          const Unit x = get_unit<DEC>(blockIdx.x + (k0 + w) * gridDim.x, args);
+          const Unit x = get_unit(blockIdx.x + (k0 + w) * gridDim.x, args);
           nt[w] = ntiles_of(x);
           qb[w] = ucnt[w] & 1;
           if (!mbar_wait(&bars->q_full[w][qb[w]], (ucnt[w] >> 1) & 1)) { set_abort(bars); ok = false; break; }
@@ -400,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         for (int w = 0; w < kNumWG; ++w) {
           nt[w] = 0;
           if (k0 + w >= my_units) continue;
-          const Unit x = get_unit<DEC>(blockIdx.x + (k0 + w) * gridDim.x, args);
+          const Unit x = get_unit(blockIdx.x + (k0 + w) * gridDim.x, args);
           nt[w] = ntiles_of(x);
         }
         const bool mine = (k0 + pw < my_units);
@@ -454,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     int tcnt = 0, ucnt = 0;
     bool stop = false;
     for (int64_t k = w; !stop && k < my_units; k += kNumWG, ++ucnt) {
-      const Unit x = get_unit<DEC>(blockIdx.x + k * gridDim.x, args);
+      const Unit x = get_unit(blockIdx.x + k * gridDim.x, args);
       const int nt = ntiles_of(x);
       const int obuf = ucnt & 1;
       const int half = kl >> 6;              // this warp's keys come from the pair's first or second block
@@ -468,8 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         if (ab) set_abort(bars);
         tc_fence_after();
         float v[16];
-        tmem_ld16(t_s + lane_addr + sb * 16, v);
-        tmem_wait_ld16(v);
+        tmem_load16(t_s + lane_addr + sb * 16, v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_empty[w][sb]);   // S is in registers: the buffer is free
@@ -519,12 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
             if (!okw) set_abort(bars);
             tc_fence_after();
             float o[16];
-            tmem_ld16(t_o + lane_addr + obuf * 16, o);
-            tmem_wait_ld16(o);
+            tmem_load16(t_o + lane_addr + obuf * 16, o);
 #pragma unroll
             for (int h = 0; h < 16; ++h) o[h] *= alpha[h];
-            tmem_st16(t_o + lane_addr + obuf * 16, o);
-            tmem_wait_st();
+            tmem_store16(t_o + lane_addr + obuf * 16, o);
           }
         }
         // P buffer sb was last read by the PV of tile tcnt-2
@@ -554,8 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       if (ab) set_abort(bars);
       tc_fence_after();
       float o[16];
-      tmem_ld16(t_o + lane_addr + obuf * 16, o);
-      tmem_wait_ld16(o);
+      tmem_load16(t_o + lane_addr + obuf * 16, o);
       if (nt == 0) {                         // empty list: no PV wrote this buffer
 #pragma unroll
         for (int h = 0; h < 16; ++h) o[h] = 0.f;
@@ -573,22 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       }
       ab = ab || aborted(bars);
       if (bar_red_or(bar_id, 128, ab)) { stop = true; break; }
-      if (DEC) {
-        // split-KV partial: unnormalised O, the reference maximum (log2
-        // units) and the row sum, per head
-        float* part = args.part + (blockIdx.x + k * gridDim.x) * static_cast<int64_t>(G) * (D + 2);
-        if (kl < D) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) part[h * (D + 2) + kl] = o[h];
-        }
-        if (kl < G) {
-          float mr = m_ref[0];
-#pragma unroll
-          for (int h = 1; h < 16; ++h) if (kl == h) mr = m_ref[h];
-          part[kl * (D + 2) + D] = (nt > 0) ? mr : -INFINITY;
-          part[kl * (D + 2) + D + 1] = red_w[kl] + red_w[16 + kl] + red_w[32 + kl] + red_w[48 + kl];
-        }
-      } else if (kl < D) {
+      if (kl < D) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float l = red_w[h] + red_w[16 + h] + red_w[32 + h] + red_w[48 + h];
@@ -616,29 +566,29 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dim
                const uint32_t* box);
 int num_sms();
 
-template <int D, int G, bool F32, bool DEC>
-static cudaError_t launch_sparse_t(const void* Q, const void* K, const void* V, int64_t q_rows, int64_t kv_rows,
+template <int D, int G, bool F32>
+static cudaError_t launch_sparse_t(const void* Q, const void* K, const void* V, int64_t rows,
                                    const sparse::SparseArgs& args, cudaStream_t st, bool* map_fail) {
   using C = sparse::Cfg<D>;
   const int h_q = args.h_q, h_kv = args.h_kv;
   CUtensorMap mQ, mK, mV;
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)G, (uint64_t)h_kv, (uint64_t)q_rows};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)G, (uint64_t)h_kv, (uint64_t)rows};
     const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)G * D * 2, (uint64_t)h_q * D * 2};
     const uint32_t box[4] = {64, (uint32_t)G, 1, 1};
     if (!make_tmap(&mQ, Q, 4, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
   }
   {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)h_kv, (uint64_t)kv_rows};
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)h_kv, (uint64_t)rows};
     const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)h_kv * D * 2};
     const uint32_t box[3] = {64, 1, 64};
     if (!make_tmap(&mK, K, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
     if (!make_tmap(&mV, V, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
   }
-  auto kern = sparse::sparse_attn_kernel<D, G, F32, DEC>;
+  auto kern = sparse::sparse_attn_kernel<D, G, F32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  const int64_t units = DEC ? static_cast<int64_t>(args.batch) * h_kv * args.nsplit : static_cast<int64_t>(h_kv) * args.total;
+  const int64_t units = static_cast<int64_t>(h_kv) * args.total;
   if (units == 0) return cudaSuccess;
   const int64_t grid = std::min<int64_t>((units + 1) / 2, num_sms());
   kern<<<static_cast<unsigned>(grid), sparse::kThreads, C::kSmem, st>>>(mQ, mK, mV, args);
@@ -650,12 +600,12 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
                                void* out, bool out_f32, cudaStream_t st, bool* map_fail) {
   sparse::SparseArgs a{};
   a.block_idx = idx; a.cu = cu; a.batch = batch; a.total = total; a.h_q = h_q; a.h_kv = h_kv; a.n_sel = n_sel;
-  a.scale = scale; a.out = out; a.seq_len = nullptr;
+  a.scale = scale; a.out = out;
   const int G = h_q / h_kv;
-#define INFLLM2_SPARSE_CASE(DD, GG)                                                                       \
-  if (d == DD && G == GG)                                                                                \
-    return out_f32 ? launch_sparse_t<DD, GG, true, false>(Q, K, V, total, total, a, st, map_fail)        \
-                   : launch_sparse_t<DD, GG, false, false>(Q, K, V, total, total, a, st, map_fail);
+#define INFLLM2_SPARSE_CASE(DD, GG)                                                            \
+  if (d == DD && G == GG)                                                                     \
+    return out_f32 ? launch_sparse_t<DD, GG, true>(Q, K, V, total, a, st, map_fail)           \
+                   : launch_sparse_t<DD, GG, false>(Q, K, V, total, a, st, map_fail);
   INFLLM2_SPARSE_CASE(128, 16)
   INFLLM2_SPARSE_CASE(128, 8)
   INFLLM2_SPARSE_CASE(128, 4)
@@ -667,33 +617,6 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
   INFLLM2_SPARSE_CASE(64, 2)
   INFLLM2_SPARSE_CASE(64, 1)
 #undef INFLLM2_SPARSE_CASE
-  return cudaErrorInvalidValue;
-}
-
-// Split-KV decode attention: partials for the combine kernel.
-cudaError_t launch_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* idx,
-                                 const int32_t* seq_len, int batch, int capacity, int h_q, int h_kv, int d,
-                                 int n_sel, int nsplit, int bps, float scale, float* part, cudaStream_t st,
-                                 bool* map_fail) {
-  sparse::SparseArgs a{};
-  a.block_idx = idx; a.cu = nullptr; a.batch = batch; a.total = batch; a.h_q = h_q; a.h_kv = h_kv;
-  a.n_sel = n_sel; a.scale = scale; a.out = nullptr; a.seq_len = seq_len; a.capacity = capacity;
-  a.nsplit = nsplit; a.bps = bps; a.part = part;
-  const int G = h_q / h_kv;
-  const int64_t kv_rows = static_cast<int64_t>(batch) * capacity;
-#define INFLLM2_SPARSE_DEC_CASE(DD, GG) \
-  if (d == DD && G == GG) return launch_sparse_t<DD, GG, false, true>(q, k_cache, v_cache, batch, kv_rows, a, st, map_fail);
-  INFLLM2_SPARSE_DEC_CASE(128, 16)
-  INFLLM2_SPARSE_DEC_CASE(128, 8)
-  INFLLM2_SPARSE_DEC_CASE(128, 4)
-  INFLLM2_SPARSE_DEC_CASE(128, 2)
-  INFLLM2_SPARSE_DEC_CASE(128, 1)
-  INFLLM2_SPARSE_DEC_CASE(64, 16)
-  INFLLM2_SPARSE_DEC_CASE(64, 8)
-  INFLLM2_SPARSE_DEC_CASE(64, 4)
-  INFLLM2_SPARSE_DEC_CASE(64, 2)
-  INFLLM2_SPARSE_DEC_CASE(64, 1)
-#undef INFLLM2_SPARSE_DEC_CASE
   return cudaErrorInvalidValue;
 }
 
