@@ -201,11 +201,12 @@ def decode_bytes_per_step(prefix: int, steps: int, batch: int, h_kv: int, d: int
     return tot / steps
 
 
-def bench_decode(T, gen, torch, dev, graph_steps: int = 64, reps: int = 3):
+def bench_decode(T, gen, torch, dev, graph_steps: int = 64, reps: int = 3, batch: int = 0):
     """µs per decode step of the 16 x 131072 workload, steps replayed from a
-    CUDA graph of `graph_steps` consecutive steps (inputs staged on device)."""
+    CUDA graph of `graph_steps` consecutive steps (inputs staged on device).
+    `batch` > 0 runs fewer sequences (a smaller case for profiling)."""
     w = gen.WORKLOADS["decode_16x128k"]
-    prefix, steps, batch = w.seqlen, graph_steps, w.batch
+    prefix, steps, batch = w.seqlen, graph_steps, (batch or w.batch)
     cap = prefix + steps
     p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
     k_cache = torch.empty(batch, cap, w.h_kv, w.d, dtype=torch.bfloat16, device=dev)
@@ -276,6 +277,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
     ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--decode-batch", type=int, default=0, help="sequences of the decode case (0: the workload's 16)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -316,7 +318,7 @@ def main():
     T.lib()
 
     if args.decode_only:
-        dd = bench_decode(T, gen, torch, dev, graph_steps=args.decode_steps)
+        dd = bench_decode(T, gen, torch, dev, graph_steps=args.decode_steps, batch=args.decode_batch)
         if rank == 0:
             print(json.dumps({"decode": dd}), flush=True)
         return

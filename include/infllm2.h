@@ -221,11 +221,16 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V,
  * row t of the prefill path (scores, max-pool, selection, sparse attention
  * over keys <= t) and writes out ([batch, h_q, d] bf16); finally
  * seq_len[b] += 1.  t must be < capacity (else the device status records
- * INFLLM2_ERR_DEVICE_BOUNDS and the sequence is skipped).  The step is a
- * fixed sequence of kernel launches with no host synchronisation, so it can
- * be captured in a CUDA graph.  workspace: infllm2_decode_workspace_bytes.
- * infllm2_decode_build_caches pools the seq_len[b] tokens already in the
- * cache into k_c1 / k_c2 (for a prefix written by the caller).
+ * INFLLM2_ERR_DEVICE_BOUNDS and that sequence's step is skipped: no output,
+ * seq_len[b] unchanged).  The step is three kernel launches with no host
+ * synchronisation, so it can be captured in a CUDA graph.  workspace:
+ * infllm2_decode_workspace_bytes (device, caller-owned, no alignment beyond
+ * 16 bytes, contents need no initialisation and carry nothing from one step
+ * to the next; one workspace must not serve two steps in flight at once).
+ * Capacities above 2.6M tokens (more than 40960 candidate blocks) are
+ * INFLLM2_ERR_UNSUPPORTED, and infllm2_decode_workspace_bytes returns 0 for
+ * them.  infllm2_decode_build_caches pools the seq_len[b] tokens already in
+ * the cache into k_c1 / k_c2 (for a prefix written by the caller).
  * ------------------------------------------------------------------- */
 typedef struct {
   void* k_cache;

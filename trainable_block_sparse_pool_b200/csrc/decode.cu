@@ -4,22 +4,24 @@
 // the pages' end-to-end decode measurement at |I| = 96).
 //
 // The new token of sequence b sits at position t = seq_len[b]; the step is
-// row t of the prefill rule applied to the sequence extended by one token:
-//   A  append k, v at t; if a stage-1 window ends at t (t+1 >= 32,
+// row t of the prefill rule applied to the sequence extended by one token.
+// Three kernels:
+//   K1 append k, v at t; if a stage-1 window ends at t (t+1 >= 32,
 //      (t+1) % 16 == 0) pool it into K_c1, likewise a coarse window
-//      (t+1 >= 128, (t+1) % 64 == 0) into K_c2 — exact mean, one bf16 rounding
-//   B  per-head log-sum-exp over the visible coarse windows, split over CTAs
-//   C  S over the visible stage-1 windows (head-group sum fused) and the
-//      max-pool to block scores, split over CTAs (each CTA keeps one window
-//      of halo so blocks never straddle CTAs)
-//   D  top-k selection per (sequence, kv group)
-//   E  split-KV block-sparse attention over the selected blocks, one
-//      partial (unnormalised O, max, sum) per split
-//   F  combine the splits, write the output, advance seq_len
+//      (t+1 >= 128, (t+1) % 64 == 0) into K_c2 (exact mean, one bf16
+//      rounding); per-head log-sum-exp partials over the visible coarse
+//      windows, split over CTAs
+//   K2 S over the visible stage-1 windows (head-group sum fused) and the
+//      max-pool to block scores, split over CTAs; the last CTA of each
+//      (sequence, group) selects the blocks
+//   K3 split-KV block-sparse attention over the selected blocks; the last
+//      CTA of each (sequence, group) merges the splits and writes the
+//      output, and the last group of a sequence advances seq_len
+// The "last CTA" hand-offs use a completion counter per (sequence, group)
+// (threadfence, then atomicAdd): no CTA ever waits for another.
 // All of it is HBM-bound (the pooled keys and the selected K/V are read
-// once); the small contractions of B, C and E (16 heads against 8 keys or
-// windows per instruction) use warp-level mma.sync, which is far from being
-// the limit.
+// once); the small contractions (16 heads against 8 keys or windows per
+// instruction) use warp-level mma.sync, which is far from being the limit.
 #include "sm100.cuh"
 
 namespace infllm2 {
@@ -29,6 +31,8 @@ namespace dec {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kLseWin = 128;   // coarse windows per LSE CTA
 constexpr int kScoreWin = 256; // stage-1 windows per score CTA (64 blocks)
+constexpr int kMaxSplits = 256; // attention splits per (sequence, group)
+constexpr float kRescaleLog2 = 8.f; // attention: raise the reference max only past this margin
 
 // D = A(16x16, bf16, row) * B(16x8, bf16, col) + C, fp32 accumulate.
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -99,96 +103,110 @@ __device__ __forceinline__ void scores_16x8_reg(float (&c)[4], const QFrag<D>& f
   }
 }
 
-// ---------------------------------------------------------------- A: append + pool
+// ---------------------------------------------------------------- pooling of the window that ends at t
+// Window [t - len + 1, t] of kv group g: rows before t from the cache, row t
+// from k_new (it may not be in the cache yet).  Exact mean in fp64, one bf16
+// rounding, written to dst.  All 128 threads of the CTA take part; `part` is
+// shared scratch of (128 / (D/8)) x D doubles.
 template <int D>
-__global__ void __launch_bounds__(128) append_kernel(const __nv_bfloat16* __restrict__ k_new,
-                                                     const __nv_bfloat16* __restrict__ v_new,
-                                                     __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
-                                                     __nv_bfloat16* __restrict__ kc1, __nv_bfloat16* __restrict__ kc2,
-                                                     const int32_t* __restrict__ seq_len, int capacity, int h_kv,
-                                                     int cap_c1, int cap_c2) {
+__device__ void pool_window(int len, const __nv_bfloat16* kc, int64_t seq0, int h_kv, int g, int t,
+                            const __nv_bfloat16* kn, __nv_bfloat16* dst, double* part) {
   constexpr int SL = D / 8;
   constexpr int NRG = 128 / SL;                 // row groups of the 128 threads
-  __shared__ double part[NRG][D];
-  const int b = blockIdx.x / h_kv, g = blockIdx.x % h_kv;
-  const int t = seq_len[b];
-  if (t < 0 || t >= capacity) {
-    if (threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
-    return;
+  const int sl = threadIdx.x % SL, rg = threadIdx.x / SL;
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  for (int r = rg; r < len; r += NRG) {
+    const int u = t - len + 1 + r;
+    const __nv_bfloat16* src = (u == t) ? kn : kc + ((seq0 + u) * h_kv + g) * D;
+    const uint4 raw = reinterpret_cast<const uint4*>(src)[sl];
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p2[i]);
+      acc[2 * i] += static_cast<double>(f.x);
+      acc[2 * i + 1] += static_cast<double>(f.y);
+    }
   }
-  const int64_t seq0 = static_cast<int64_t>(b) * capacity;
-  const __nv_bfloat16* kn = k_new + (static_cast<int64_t>(b) * h_kv + g) * D;
-  const __nv_bfloat16* vn = v_new + (static_cast<int64_t>(b) * h_kv + g) * D;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[rg * D + sl * 8 + i] = acc[i];
+  __syncthreads();
   if (threadIdx.x < SL) {
-    reinterpret_cast<uint4*>(kc + ((seq0 + t) * h_kv + g) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(kn)[threadIdx.x];
-    reinterpret_cast<uint4*>(vc + ((seq0 + t) * h_kv + g) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(vn)[threadIdx.x];
+    uint16_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      double s = 0.0;
+      for (int q = 0; q < NRG; ++q) s += part[q * D + threadIdx.x * 8 + i];
+      o[i] = f64_to_bf16_rne(s / len);
+    }
+    uint4 v;
+    v.x = o[0] | (static_cast<uint32_t>(o[1]) << 16);
+    v.y = o[2] | (static_cast<uint32_t>(o[3]) << 16);
+    v.z = o[4] | (static_cast<uint32_t>(o[5]) << 16);
+    v.w = o[6] | (static_cast<uint32_t>(o[7]) << 16);
+    reinterpret_cast<uint4*>(dst)[threadIdx.x] = v;
   }
-  // a window [t-len+1, t] completes at this step: pool it (rows before t come
-  // from the cache, row t from k_new)
-  for (int which = 0; which < 2; ++which) {
-    const int len = which ? 128 : 32, stride = which ? 64 : 16;
-    if (t + 1 < len || (t + 1 - len) % stride != 0) continue;
-    const int j = (t + 1 - len) / stride;
-    if (j >= (which ? cap_c2 : cap_c1)) {
-      if (threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
-      continue;
-    }
-    // 128 threads: slice sl = tid % SL, row group rg = tid / SL (8 groups for D=128)
-    const int sl = threadIdx.x % SL, rg = threadIdx.x / SL;
-    double acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-    for (int r = rg; r < len; r += NRG) {
-      const int u = t - len + 1 + r;
-      const __nv_bfloat16* src = (u == t) ? kn : kc + ((seq0 + u) * h_kv + g) * D;
-      const uint4 raw = reinterpret_cast<const uint4*>(src)[sl];
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(p2[i]);
-        acc[2 * i] += static_cast<double>(f.x);
-        acc[2 * i + 1] += static_cast<double>(f.y);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) part[rg][sl * 8 + i] = acc[i];
-    __syncthreads();
-    if (threadIdx.x < SL) {
-      uint16_t o[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        double s = 0.0;
-        for (int q = 0; q < NRG; ++q) s += part[q][threadIdx.x * 8 + i];
-        o[i] = f64_to_bf16_rne(s / len);
-      }
-      uint4 v;
-      v.x = o[0] | (static_cast<uint32_t>(o[1]) << 16);
-      v.y = o[2] | (static_cast<uint32_t>(o[3]) << 16);
-      v.z = o[4] | (static_cast<uint32_t>(o[5]) << 16);
-      v.w = o[6] | (static_cast<uint32_t>(o[7]) << 16);
-      __nv_bfloat16* dst = (which ? kc2 : kc1) +
-                           ((static_cast<int64_t>(b) * h_kv + g) * (which ? cap_c2 : cap_c1) + j) * D;
-      reinterpret_cast<uint4*>(dst)[threadIdx.x] = v;
-    }
-    __syncthreads();
-  }
+  __syncthreads();                              // part is free again; dst is visible to the CTA
 }
 
-// ---------------------------------------------------------------- B: coarse LSE partials
-// grid (batch*h_kv, nsplit2), 4 warps.  part2[(bg*nsplit2 + c)*16 + h] = (max, sum) in log2 units.
+// ---------------------------------------------------------------- K1: append, pooling, coarse LSE partials
+// grid (batch*h_kv, nsplit2), 4 warps; CTA c covers coarse windows
+// [128c, 128c + 128).
+//  * CTA 0 of (b, g) clears the step's completion counters, appends k, v at
+//    row t and pools the stage-1 window that ends at t, when one does.
+//  * The CTA whose range holds a coarse window ending at t pools it first and
+//    then uses it.
+//  * Every CTA writes (max, sum) in log2 units of its windows' scores, per
+//    head: part2[(bg*nsplit2 + c)*16 + h].
+// Counters (cnt): [0, nbg) score CTAs done per (b, g); [nbg, 2 nbg)
+// attention CTAs done per (b, g); [2 nbg, 2 nbg + batch) groups of b merged.
 template <int D>
-__global__ void __launch_bounds__(128) lse_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc2,
-                                                  const int32_t* __restrict__ seq_len, int h_q, int h_kv, int cap_c2,
-                                                  float scale, float2* __restrict__ part2) {
-  const int bg = blockIdx.x, c = blockIdx.y;
+__global__ void __launch_bounds__(128) lse_append_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
+    const __nv_bfloat16* __restrict__ v_new, __nv_bfloat16* kc, __nv_bfloat16* vc, __nv_bfloat16* kc1,
+    __nv_bfloat16* kc2, const int32_t* __restrict__ seq_len, int capacity, int h_q, int h_kv, int cap_c1, int cap_c2,
+    float scale, float2* __restrict__ part2, unsigned* __restrict__ cnt) {
+  constexpr int SL = D / 8;
+  __shared__ double pool_part[(128 / SL) * D];
+  __shared__ float2 red[4][16];
+  const int bg = blockIdx.x, c = blockIdx.y, nbg = gridDim.x;
   const int b = bg / h_kv, g = bg % h_kv;
   const int G = h_q / h_kv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
-  __shared__ float2 red[4][16];
+  if (c == 0 && threadIdx.x == 0) {
+    cnt[bg] = 0u;
+    cnt[nbg + bg] = 0u;
+    if (g == 0) cnt[2 * nbg + b] = 0u;
+  }
   const int t = seq_len[b];
-  const int n2 = visible_windows_dev(t, 128, 64);
+  if (t < 0 || t >= capacity) {
+    if (c == 0 && g == 0 && threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const int64_t seq0 = static_cast<int64_t>(b) * capacity;
+  const __nv_bfloat16* kn = k_new + (static_cast<int64_t>(b) * h_kv + g) * D;
+  if (c == 0) {
+    if (threadIdx.x < SL) {
+      const __nv_bfloat16* vn = v_new + (static_cast<int64_t>(b) * h_kv + g) * D;
+      reinterpret_cast<uint4*>(kc + ((seq0 + t) * h_kv + g) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(kn)[threadIdx.x];
+      reinterpret_cast<uint4*>(vc + ((seq0 + t) * h_kv + g) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(vn)[threadIdx.x];
+    }
+    if (t + 1 >= 32 && (t + 1 - 32) % 16 == 0) {
+      const int j = (t + 1 - 32) / 16;
+      if (j < cap_c1) pool_window<D>(32, kc, seq0, h_kv, g, t, kn, kc1 + (static_cast<int64_t>(bg) * cap_c1 + j) * D, pool_part);
+      else if (threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    }
+  }
+  if (t + 1 >= 128 && (t + 1 - 128) % 64 == 0) {
+    const int j = (t + 1 - 128) / 64;
+    if (j / kLseWin == c) {
+      if (j < cap_c2) pool_window<D>(128, kc, seq0, h_kv, g, t, kn, kc2 + (static_cast<int64_t>(bg) * cap_c2 + j) * D, pool_part);
+      else if (threadIdx.x == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+    }
+  }
+  const int n2 = min(visible_windows_dev(t, 128, 64), cap_c2);
   QFrag<D> f;
   load_qfrag<D>(f, q + (static_cast<int64_t>(b) * h_q + g * G) * D, lane, G);
   const float cs = scale * kLog2e;
@@ -252,172 +270,107 @@ __global__ void __launch_bounds__(128) lse_kernel(const __nv_bfloat16* __restric
   }
 }
 
-// ---------------------------------------------------------------- C: scores + max-pool
-// grid (batch*h_kv, nsplit1), 8 warps; windows [256c - 1, 256c + 255) -> blocks [64c, 64c + 64)
-template <int D>
-__global__ void __launch_bounds__(256) score_pool_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
-    const float2* __restrict__ part2, int nsplit2, int h_q, int h_kv, int cap_c1, int nblk_cap, float scale,
-    float* __restrict__ bscore) {
-  const int bg = blockIdx.x, c = blockIdx.y;
-  const int b = bg / h_kv, g = bg % h_kv;
-  const int G = h_q / h_kv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  __shared__ float nlse[16];
-  __shared__ float sw[kScoreWin + 8];
-  const int t = seq_len[b];
-  const int n1 = visible_windows_dev(t, 32, 16);
-  const int n2 = visible_windows_dev(t, 128, 64);
-  const int j0 = c * kScoreWin - 1;
-  if (j0 + 1 >= n1 && c > 0) return;            // no visible window here
-  const float cs = scale * kLog2e;
-  const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
-  const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
-  // this warp's n-tiles are nt = warp + 8 i (i < 5): issue every load first
-  constexpr int kMaxNt = (kScoreWin / 8 + 1 + 7) / 8;
-  uint4 kv[kMaxNt][D / 32];
+// ---------------------------------------------------------------- block selection of one (sequence, group)
+// Run by the 256 threads of one CTA.  Candidates are the blocks after the
+// init blocks and before the local run; the top_k largest block scores are
+// found with an exact radix select (8-bit digits of the fp32 bit pattern of
+// score - min; the scores are >= 0, so the bit order is the value order),
+// ties go to the lower block.  Output: init blocks, the chosen candidates
+// ascending, the local run, -1 padding ([top168] §三 third stage, §七).
+constexpr int kSelThreads = 256;
+struct SelScratch {
+  int hist[256];
+  uint32_t red[2][kSelThreads / 32];
+  int wsum[kSelThreads / 32];
+  int digit, above;
+};
+
+// exclusive prefix sum of v over the CTA's threads in index order; *total
+// gets the sum over all threads
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
 #pragma unroll
-  for (int i = 0; i < kMaxNt; ++i) {
-    const int nt = warp + 8 * i;
-    const int wr = j0 + nt * 8 + gid;
-    const bool ok = (nt * 8 < kScoreWin + 1) && wr >= 0 && wr < n1;
-    load_krow<D>(kv[i], ok ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  // the per-head LSE (coarse partials combined) while the loads are in flight
-  if (threadIdx.x < 16) {
-    const int h = threadIdx.x;
-    float mm = -INFINITY, ll = 0.f;
-    if (h < G) {
-      if (n2 > 0) {
-        for (int k = 0; k < nsplit2; ++k) {
-          const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + k) * 16 + h];
-          const float mn = fmaxf(mm, v.x);
-          if (mn != -INFINITY) {
-            ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
-            mm = mn;
-          }
-        }
-      } else {
-        // no coarse window yet (t < 127): exact log-sum-exp over the visible stage-1 windows
-        for (int j = 0; j < n1 && j < cap_c1; ++j) {
-          float dot = 0.f;
-          for (int e = 0; e < D; ++e)
-            dot += __bfloat162float(qh[h * D + e]) * __bfloat162float(base[static_cast<int64_t>(j) * D + e]);
-          const float x = dot * cs;
-          const float mn = fmaxf(mm, x);
-          ll = ll * ex2(mm - mn) + ex2(x - mn);
-          mm = mn;
-        }
-      }
-    }
-    nlse[h] = (h < G && ll > 0.f) ? -(mm + log2f(ll)) : -INFINITY;
-  }
-  QFrag<D> f;
-  load_qfrag<D>(f, qh, lane, G);
+  if (lane == 31) wsum[warp] = x;
   __syncthreads();
-  const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
+  int before = 0, tot = 0;
 #pragma unroll
-  for (int i = 0; i < kMaxNt; ++i) {
-    const int nt = warp + 8 * i;
-    if (nt * 8 >= kScoreWin + 1) break;
-    const int w0 = j0 + nt * 8;
-    float sc[4];
-    scores_16x8_reg<D>(sc, f, kv[i]);
-    // head-group sum for keys 2tig and 2tig+1: two heads here, the other 14 on the lanes with the same tig
-    float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
-    float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      e0 += __shfl_xor_sync(0xffffffffu, e0, o);
-      e1 += __shfl_xor_sync(0xffffffffu, e1, o);
-    }
-    if (gid == 0) {
-      const int i0 = nt * 8 + 2 * tig;
-      if (i0 < kScoreWin + 8) sw[i0] = (w0 + 2 * tig >= 0 && w0 + 2 * tig < n1) ? e0 : -INFINITY;
-      if (i0 + 1 < kScoreWin + 8) sw[i0 + 1] = (w0 + 2 * tig + 1 >= 0 && w0 + 2 * tig + 1 < n1) ? e1 : -INFINITY;
-    }
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    const int s = wsum[w];
+    before += (w < warp) ? s : 0;
+    tot += s;
   }
-  __syncthreads();
-  // block scores: block blk = 64c + i takes windows 4 blk - 1 .. 4 blk + 3 = sw[4i .. 4i + 4]
-  if (threadIdx.x < kScoreWin / 4) {
-    const int i = threadIdx.x;
-    const int blk = c * (kScoreWin / 4) + i;
-    if (blk < nblk_cap) {
-      float m = -INFINITY;
-#pragma unroll
-      for (int q4 = 0; q4 < 5; ++q4) m = fmaxf(m, sw[4 * i + q4]);
-      bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
-    }
-  }
+  __syncthreads();                              // wsum may be reused
+  *total = tot;
+  return before + x - v;
 }
 
-// ---------------------------------------------------------------- D: top-k per (sequence, group)
-// One CTA of kSelThreads per (sequence, kv group): the same exact radix
-// select as the prefill top-k (8-bit digits of score - min, ties to the
-// lower block), but the candidates are spread over all threads, so the
-// latency of a single row is short.
-constexpr int kSelThreads = 256;
-
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ bscore,
-                                                             const int32_t* __restrict__ seq_len, int h_kv,
-                                                             int nblk_cap, int cand_cap, int n_init, int n_local,
-                                                             int top_k, int n_sel, int32_t* __restrict__ idx) {
-  extern __shared__ uint32_t dsel_smem[];
-  uint32_t* keys = dsel_smem;                                   // [cand_cap]
-  __shared__ int hist[256];
-  __shared__ uint32_t s_red[2][kSelThreads / 32];
-  __shared__ int s_digit, s_above, s_wsum[kSelThreads / 32], s_wsum2[kSelThreads / 32];
-  const int bg = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ void select_blocks_cta(const float* row, int t, int n_init, int n_local, int top_k, int n_sel,
+                                  int cand_cap, int32_t* out, uint32_t* keys, SelScratch& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = kSelThreads / 32;
-  const int b = bg / h_kv;
-  const int t = seq_len[b];
   const int b_t = t / 64;
-  int32_t* out = idx + static_cast<int64_t>(bg) * n_sel;
   const int init_hi = min(n_init, b_t + 1);
   const int loc_lo = max(0, b_t - n_local + 1);
   const int ncand = max(0, loc_lo - init_hi);
-  if (ncand <= top_k) {
+  if (ncand <= top_k) {                         // every causal block fits
     for (int i = tid; i < n_sel; i += kSelThreads) out[i] = (i <= b_t) ? i : -1;
     return;
   }
-  if (ncand > cand_cap || init_hi + ncand > nblk_cap) {
+  if (ncand > cand_cap) {
     if (tid == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
     return;
   }
-  const float* row = bscore + static_cast<int64_t>(bg) * nblk_cap;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = tid; i < ncand; i += kSelThreads) {
-    const uint32_t k = __float_as_uint(fmaxf(row[init_hi + i], 0.f));
-    keys[i] = k;
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
+  for (int i0 = 0; i0 < ncand; i0 += 8 * kSelThreads) {        // eight loads in flight per thread
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kSelThreads + tid;
+      v[u] = (i < ncand) ? __ldcg(row + init_hi + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kSelThreads + tid;
+      if (i < ncand) {
+        const uint32_t k = __float_as_uint(fmaxf(v[u], 0.f));
+        keys[i] = k;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
   }
   kmin = sel::warp_min_u32(kmin);
   kmax = sel::warp_max_u32(kmax);
-  if (lane == 0) { s_red[0][warp] = kmin; s_red[1][warp] = kmax; }
+  if (lane == 0) { sh.red[0][warp] = kmin; sh.red[1][warp] = kmax; }
   __syncthreads();
   kmin = 0xffffffffu; kmax = 0u;
-  for (int w = 0; w < NW; ++w) { kmin = min(kmin, s_red[0][w]); kmax = max(kmax, s_red[1][w]); }
+#pragma unroll
+  for (int w = 0; w < NW; ++w) { kmin = min(kmin, sh.red[0][w]); kmax = max(kmax, sh.red[1][w]); }
   const uint32_t range = kmax - kmin;
   int hi = range ? 32 - __clz(range) : 0;
   uint32_t prefix = 0;
-  int k_rem = top_k;
+  int k_rem = top_k;                            // how many of the keys matching prefix are still to take
   while (hi > 0) {
     const int shift = max(0, hi - 8);
     const int nb = 1 << (hi - shift);
-    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+    sh.hist[tid] = 0;
     __syncthreads();
     const uint64_t want = static_cast<uint64_t>(prefix) >> hi;
     for (int i = tid; i < ncand; i += kSelThreads) {
       const uint32_t u = keys[i] - kmin;
-      if ((static_cast<uint64_t>(u) >> hi) == want) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1);
+      if ((static_cast<uint64_t>(u) >> hi) == want) atomicAdd(&sh.hist[(u >> shift) & (nb - 1)], 1);
     }
     __syncthreads();
     if (warp == 0) {
+      // suffix sums from the top digit down: the digit where they reach k_rem
       int lsum = 0;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) lsum += (lane * 8 + q < nb) ? hist[lane * 8 + q] : 0;
+      for (int q = 0; q < 8; ++q) lsum += (lane * 8 + q < nb) ? sh.hist[lane * 8 + q] : 0;
       int suf = lsum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -425,75 +378,183 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
         if (lane + o < 32) suf += v;
       }
       int above = suf - lsum;
-      int digit = -1, above_digit = 0;
       if (above < k_rem && suf >= k_rem) {
         for (int q = 7; q >= 0; --q) {
           const int bb = lane * 8 + q;
-          const int hh = (bb < nb) ? hist[bb] : 0;
-          if (above + hh >= k_rem) { digit = bb; above_digit = above; break; }
+          const int hh = (bb < nb) ? sh.hist[bb] : 0;
+          if (above + hh >= k_rem) { sh.digit = bb; sh.above = above; break; }
           above += hh;
         }
       }
-      if (digit >= 0) { s_digit = digit; s_above = above_digit; }
     }
     __syncthreads();
-    prefix |= static_cast<uint32_t>(s_digit) << shift;
-    k_rem -= s_above;
+    prefix |= static_cast<uint32_t>(sh.digit) << shift;
+    k_rem -= sh.above;
     hi = shift;
-    __syncthreads();
+    __syncthreads();                            // hist, digit and above are rewritten by the next pass
   }
-  const uint32_t T = kmin + prefix;
-  // ordered output: INIT, chosen candidates ascending, LOCAL, padding
+  const uint32_t T = kmin + prefix;             // the top_k-th largest key; k_rem keys equal to it are taken
+  // one ordered pass: thread tid owns candidates [tid*per, tid*per + per)
+  const int per = (ncand + kSelThreads - 1) / kSelThreads;
+  const int c0 = min(ncand, tid * per), c1 = min(ncand, c0 + per);
+  int n_gt = 0, n_eq = 0;
+  for (int i = c0; i < c1; ++i) {
+    n_gt += keys[i] > T;
+    n_eq += keys[i] == T;
+  }
+  int tot;
+  const int eq_before = cta_exclusive_scan(n_eq, sh.wsum, &tot);
+  const int eq_take = max(0, min(n_eq, k_rem - eq_before));
+  const int pos0 = cta_exclusive_scan(n_gt + eq_take, sh.wsum, &tot);
+  int pos = init_hi + pos0, eq_seen = 0;
+  for (int i = c0; i < c1; ++i) {
+    const uint32_t k = keys[i];
+    const bool take = (k > T) || (k == T && eq_seen++ < eq_take);
+    if (take) out[pos++] = init_hi + i;
+  }
   for (int i = tid; i < init_hi; i += kSelThreads) out[i] = i;
-  int pos = init_hi, eq_seen = 0;
-  for (int base = 0; base < ncand; base += kSelThreads) {
-    const int i = base + tid;
-    const bool valid = i < ncand;
-    const uint32_t k = valid ? keys[i] : 0u;
-    const bool gt = valid && k > T, eq = valid && k == T;
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s_wsum[warp] = __popc(eqm);
-    __syncthreads();
-    int eq_before = eq_seen;
-    for (int w = 0; w < warp; ++w) eq_before += s_wsum[w];
-    int eq_tot = 0;
-    for (int w = 0; w < NW; ++w) eq_tot += s_wsum[w];
-    const bool take = gt || (eq && eq_before + __popc(eqm & lanemask_lt()) < k_rem);
-    const uint32_t tm = __ballot_sync(0xffffffffu, take);
-    if (lane == 0) s_wsum2[warp] = __popc(tm);
-    __syncthreads();
-    int take_before = pos;
-    for (int w = 0; w < warp; ++w) take_before += s_wsum2[w];
-    int take_tot = 0;
-    for (int w = 0; w < NW; ++w) take_tot += s_wsum2[w];
-    if (take) out[take_before + __popc(tm & lanemask_lt())] = init_hi + i;
-    pos += take_tot;
-    eq_seen += eq_tot;
-    __syncthreads();
-  }
   const int nloc = b_t - loc_lo + 1;
-  for (int i = tid; i < nloc; i += kSelThreads) out[pos + i] = loc_lo + i;
-  pos += nloc;
-  for (int i = pos + tid; i < n_sel; i += kSelThreads) out[i] = -1;
+  for (int i = tid; i < nloc; i += kSelThreads) out[init_hi + top_k + i] = loc_lo + i;
+  for (int i = init_hi + top_k + nloc + tid; i < n_sel; i += kSelThreads) out[i] = -1;
 }
 
-// ---------------------------------------------------------------- E: split-KV sparse attention
-// grid (batch*h_kv, nsplit), kAttWarps warps.  CTA (bg, sp) covers the
-// entries [sp*bps, sp*bps + bps) of the block list of (sequence b, group g);
-// each entry is two 32-key chunks, and warp w takes chunks w, w + kAttWarps, ...
-// Per chunk the warp stages K and V (cp.async, 16 B pieces, 16-byte
-// chunks of a key row XOR-swizzled by the row index so ldmatrix is free of
-// bank conflicts), then
-//   S[16 heads, 32 keys] = Q . K^T     (mma.sync m16n8k16, K via ldmatrix)
-//   online softmax in log2 units (running max m, sum l per head)
-//   O[16, D] += P . V                  (P re-used from the S fragments,
-//                                        V via ldmatrix.trans)
-// The next chunk's K is issued as soon as S is done and its V as soon as
-// the PV product is done, so every warp keeps a copy in flight.  The warps'
-// (m, l, O) are merged in shared memory and written as one partial
-// (unnormalised O, m, l) per CTA for the combine kernel.
-// Keys past t (and chunks of invalid or not-yet-visible blocks) are never
-// read: their staging rows are zero-filled and their scores are -inf.
+// ---------------------------------------------------------------- K2: scores, max-pool, selection
+// grid (batch*h_kv, nsplit1), 8 warps; CTA c covers stage-1 windows
+// [256c - 1, 256c + 255) and writes block scores [64c, 64c + 64) (one
+// window of halo, so a block never straddles CTAs).  Per window: the 16
+// heads' scores, normalised by their LSE and summed over the group
+// ([top168] §三 second stage, §四); per block: the max over its 5 windows.
+// The last CTA of (b, g) to finish runs the selection.
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) score_select_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
+    const float2* __restrict__ part2, int nsplit2, int capacity, int h_q, int h_kv, int cap_c1, int nblk_cap,
+    int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel, float* __restrict__ bscore,
+    int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
+  extern __shared__ uint32_t sel_keys[];       // [cand_cap], used by the selecting CTA
+  __shared__ float nlse[16];
+  __shared__ float2 lsep[16][17];
+  __shared__ float sw[kScoreWin + 8];
+  __shared__ SelScratch sel_sh;
+  __shared__ int s_last;
+  const int bg = blockIdx.x, c = blockIdx.y;
+  const int b = bg / h_kv, g = bg % h_kv;
+  const int G = h_q / h_kv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int t = seq_len[b];
+  if (t < 0 || t >= capacity) return;          // recorded by the append kernel
+  const int n1 = min(visible_windows_dev(t, 32, 16), cap_c1);
+  const int n2 = visible_windows_dev(t, 128, 64);
+  const int j0 = c * kScoreWin - 1;
+  const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
+  if (c == 0 || j0 + 1 < n1) {                 // this CTA has visible windows
+    const float cs = scale * kLog2e;
+    const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
+    // this warp's n-tiles are nt = warp + 8 i (i < 5): issue every load first
+    constexpr int kMaxNt = (kScoreWin / 8 + 1 + 7) / 8;
+    uint4 kv[kMaxNt][D / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxNt; ++i) {
+      const int nt = warp + 8 * i;
+      const int wr = j0 + nt * 8 + gid;
+      const bool ok = (nt * 8 < kScoreWin + 1) && wr >= 0 && wr < n1;
+      load_krow<D>(kv[i], ok ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+    }
+    // per-head LSE: thread (h, k0) folds the coarse partials k0, k0 + 16, ...
+    {
+      const int h = threadIdx.x & 15, k0 = threadIdx.x >> 4;
+      float mm = -INFINITY, ll = 0.f;
+      if (h < G && n2 > 0) {
+        for (int k = k0; k < nsplit2; k += 16) {
+          const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + k) * 16 + h];
+          const float mn = fmaxf(mm, v.x);
+          if (mn != -INFINITY) {
+            ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
+            mm = mn;
+          }
+        }
+      }
+      lsep[h][k0] = make_float2(mm, ll);
+    }
+    __syncthreads();
+    if (threadIdx.x < 16) {
+      const int h = threadIdx.x;
+      float mm = -INFINITY, ll = 0.f;
+      if (h < G) {
+        if (n2 > 0) {
+          for (int k = 0; k < 16; ++k) {
+            const float2 v = lsep[h][k];
+            const float mn = fmaxf(mm, v.x);
+            if (mn != -INFINITY) {
+              ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
+              mm = mn;
+            }
+          }
+        } else {
+          // no coarse window yet (t < 127): exact log-sum-exp over the visible stage-1 windows
+          for (int j = 0; j < n1; ++j) {
+            float dot = 0.f;
+            for (int e = 0; e < D; ++e)
+              dot += __bfloat162float(qh[h * D + e]) * __bfloat162float(base[static_cast<int64_t>(j) * D + e]);
+            const float x = dot * cs;
+            const float mn = fmaxf(mm, x);
+            ll = ll * ex2(mm - mn) + ex2(x - mn);
+            mm = mn;
+          }
+        }
+      }
+      nlse[h] = (h < G && ll > 0.f) ? -(mm + log2f(ll)) : -INFINITY;
+    }
+    QFrag<D> f;
+    load_qfrag<D>(f, qh, lane, G);
+    __syncthreads();
+    const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
+#pragma unroll
+    for (int i = 0; i < kMaxNt; ++i) {
+      const int nt = warp + 8 * i;
+      if (nt * 8 >= kScoreWin + 1) break;
+      const int w0 = j0 + nt * 8;
+      float sc[4];
+      scores_16x8_reg<D>(sc, f, kv[i]);
+      // head-group sum for keys 2tig and 2tig+1: two heads here, the other 14 on the lanes with the same tig
+      float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
+      float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        e0 += __shfl_xor_sync(0xffffffffu, e0, o);
+        e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+      }
+      if (gid == 0) {
+        const int i0 = nt * 8 + 2 * tig;
+        if (i0 < kScoreWin + 8) sw[i0] = (w0 + 2 * tig >= 0 && w0 + 2 * tig < n1) ? e0 : -INFINITY;
+        if (i0 + 1 < kScoreWin + 8) sw[i0 + 1] = (w0 + 2 * tig + 1 >= 0 && w0 + 2 * tig + 1 < n1) ? e1 : -INFINITY;
+      }
+    }
+    __syncthreads();
+    // block scores: block blk = 64c + i takes windows 4 blk - 1 .. 4 blk + 3 = sw[4i .. 4i + 4]
+    if (threadIdx.x < kScoreWin / 4) {
+      const int i = threadIdx.x;
+      const int blk = c * (kScoreWin / 4) + i;
+      if (blk < nblk_cap) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int q4 = 0; q4 < 5; ++q4) m = fmaxf(m, sw[4 * i + q4]);
+        bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
+      }
+    }
+  }
+  // the last CTA of (b, g) to finish selects the blocks
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&cnt[bg], 1u) == gridDim.y - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  select_blocks_cta(bscore + static_cast<int64_t>(bg) * nblk_cap, t, n_init, n_local, top_k, n_sel, cand_cap,
+                    idx + static_cast<int64_t>(bg) * n_sel, sel_keys, sel_sh);
+}
+
 constexpr int kAttWarps = 4;
 constexpr int kChunkKeys = 32;
 
@@ -524,26 +585,52 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int D>
 struct AttCfg {
   static constexpr int CH = D / 8;                            // 16-byte pieces per key row
+  static constexpr int kRow = D + 8;                          // merge rows: D values, m, l, padding (bank spread)
+  static constexpr int kPart = D + 4;                         // partial rows in HBM: D values, m, l, padding (16 B rows)
   static constexpr uint32_t kTile = kChunkKeys * D * 2;       // one K or V chunk
   static constexpr uint32_t kSmem = kAttWarps * 2 * kTile;    // per-warp K and V buffers
-  static_assert(kAttWarps * 16 * (D + 2) * 4 <= kSmem, "merge area fits in the staging buffers");
+  static_assert(kAttWarps * 16 * kRow * 4 <= kSmem, "warp merge area fits in the staging buffers");
+  static_assert(kMaxSplits * 16 * 4 * 2 <= kSmem, "split maxima and sums fit in the staging buffers");
+  static_assert(16 * (D / 4) <= 4 * 32 * kAttWarps, "four merge items per thread cover every (head, quad)");
 };
 
+// ---------------------------------------------------------------- K3: split-KV sparse attention + merge
+// grid (batch*h_kv, nsplit), kAttWarps warps.  CTA (bg, sp) covers the
+// entries [sp*bps, sp*bps + bps) of the block list of (sequence b, group g);
+// each entry is two 32-key chunks, and warp w takes chunks w, w + kAttWarps, ...
+// Per chunk the warp stages K and V (cp.async, 16 B pieces; the 16-byte
+// pieces of a key row are XOR-swizzled by the row index so ldmatrix is free
+// of bank conflicts), then
+//   S[16 heads, 32 keys] = Q . K^T     (mma.sync m16n8k16, K via ldmatrix)
+//   P = 2^(S*scale*log2e - m_ref)      (m_ref per head, raised only when a
+//                                        score passes it by more than 2^8;
+//                                        then O and l are rescaled once)
+//   O[16, D] += P . V                  (P re-used from the S fragments,
+//                                        V via ldmatrix.trans)
+// The next chunk's K is issued as soon as S is done and its V as soon as
+// the PV product is done, so every warp keeps a copy in flight.  The warps'
+// (m_ref, l, O) are merged in shared memory into one partial per CTA; the
+// last CTA of (b, g) to finish merges the partials, writes the output, and
+// the last group of b to finish advances seq_len[b].
+// Keys past t (and chunks of invalid or not yet visible blocks) are never
+// read: their staging rows are zero-filled and their scores are -inf.
 template <int D>
 __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ seq_len, int capacity, int h_q, int h_kv, int n_sel,
-    int bps, float scale, float* __restrict__ part) {
+    const int32_t* __restrict__ idx, int32_t* seq_len, int capacity, int h_q, int h_kv, int n_sel, int bps,
+    float scale, float* __restrict__ part, __nv_bfloat16* __restrict__ out, unsigned* __restrict__ cnt) {
   using C = AttCfg<D>;
   extern __shared__ __align__(128) uint8_t att_smem[];
-  const int bg = blockIdx.x, sp = blockIdx.y, nsplit = gridDim.y;
+  __shared__ float s_wgt[kAttWarps][16], s_M[16], s_L[16];
+  __shared__ int s_last;
+  const int bg = blockIdx.x, sp = blockIdx.y, nsplit = gridDim.y, nbg = gridDim.x;
   const int b = bg / h_kv, g = bg % h_kv;
   const int G = h_q / h_kv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
-  // the new token's position; keys 0..t are visible (t is clamped into the
-  // cache, so no address below can leave it)
-  const int t = min(seq_len[b], capacity - 1);
+  // the new token's position; keys 0..t are visible
+  const int t = seq_len[b];
+  if (t < 0 || t >= capacity) return;          // recorded by the append kernel
   const int32_t* list = idx + static_cast<int64_t>(bg) * n_sel + static_cast<int64_t>(sp) * bps;
   const int nb = max(0, min(bps, n_sel - sp * bps));
   const int nmine = (2 * nb > warp) ? (2 * nb - 1 - warp) / kAttWarps + 1 : 0;
@@ -591,7 +678,7 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
   float o[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads gid, gid + 8
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads gid, gid + 8: reference max, row sum
   const float cs = scale * kLog2e;
 
   int k0 = chunk_key0(0);
@@ -636,30 +723,34 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      // k0 <= t, so key k0 is visible and both maxima are finite
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float a0 = ex2(m0 - mn0), a1 = ex2(m1 - mn1);    // m = -inf: 0
-      m0 = mn0;
-      m1 = mn1;
-      float ps0 = 0.f, ps1 = 0.f;
+      // key k0 is visible, so both maxima are finite; the reference maxima
+      // move only past the margin (the first chunk always sets them)
+      const bool up0 = mx0 > m0 + kRescaleLog2, up1 = mx1 > m1 + kRescaleLog2;
+      if (__any_sync(0xffffffffu, up0 || up1)) {
+        const float n0 = up0 ? mx0 : m0, n1 = up1 ? mx1 : m1;
+        const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - n0);
+        const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        l0 *= a0;
+        l1 *= a1;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] *= a0;
+          o[n][1] *= a0;
+          o[n][2] *= a1;
+          o[n][3] *= a1;
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          s[j][e] = ex2(s[j][e] - mn0);
-          s[j][2 + e] = ex2(s[j][2 + e] - mn1);
-          ps0 += s[j][e];
-          ps1 += s[j][2 + e];
+          s[j][e] = ex2(s[j][e] - m0);
+          s[j][2 + e] = ex2(s[j][2 + e] - m1);
+          l0 += s[j][e];
+          l1 += s[j][2 + e];
         }
-      }
-      l0 = l0 * a0 + ps0;
-      l1 = l1 * a1 + ps1;
-#pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        o[n][0] *= a0;
-        o[n][1] *= a0;
-        o[n][2] *= a1;
-        o[n][3] *= a1;
       }
     }
     cp_async_wait1();                        // V of chunk i (the next K may still be in flight)
@@ -690,18 +781,16 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
 
-  // merge the warps: [warp][16 heads][D + 2] in the (now idle) staging buffers
+  // ---- merge the warps in the (now idle) staging buffers: [warp][16][kRow]
   __syncthreads();
   float* mw = reinterpret_cast<float*>(att_smem);
   {
-    float* r0 = mw + (warp * 16 + gid) * (D + 2);
-    float* r1 = mw + (warp * 16 + gid + 8) * (D + 2);
+    float* r0 = mw + (warp * 16 + gid) * C::kRow;
+    float* r1 = mw + (warp * 16 + gid + 8) * C::kRow;
 #pragma unroll
     for (int n = 0; n < D / 8; ++n) {
-      r0[8 * n + 2 * tig] = o[n][0];
-      r0[8 * n + 2 * tig + 1] = o[n][1];
-      r1[8 * n + 2 * tig] = o[n][2];
-      r1[8 * n + 2 * tig + 1] = o[n][3];
+      *reinterpret_cast<float2*>(r0 + 8 * n + 2 * tig) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(r1 + 8 * n + 2 * tig) = make_float2(o[n][2], o[n][3]);
     }
     if (tig == 0) {
       r0[D] = m0;
@@ -711,83 +800,126 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
     }
   }
   __syncthreads();
-  float* dst = part + (static_cast<int64_t>(bg) * nsplit + sp) * G * (D + 2);
-  for (int e = threadIdx.x; e < G * (D + 1); e += 32 * kAttWarps) {
-    const int h = e / (D + 1), d = e - h * (D + 1);   // d == D: the row sum
+  if (threadIdx.x < 16) {
+    const int h = threadIdx.x;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, mw[(w * 16 + h) * (D + 2) + D]);
-    float acc = 0.f;
-    const int col = (d < D) ? d : D + 1;
+    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, mw[(w * 16 + h) * C::kRow + D]);
+    float L = 0.f;
 #pragma unroll
     for (int w = 0; w < kAttWarps; ++w) {
-      const float mwh = mw[(w * 16 + h) * (D + 2) + D];
-      if (mwh != -INFINITY) acc += mw[(w * 16 + h) * (D + 2) + col] * ex2(mwh - M);
+      const float mwh = mw[(w * 16 + h) * C::kRow + D];
+      const float wg = (mwh == -INFINITY) ? 0.f : ex2(mwh - M);
+      s_wgt[w][h] = wg;
+      L += wg * mw[(w * 16 + h) * C::kRow + D + 1];
     }
-    if (d < D) {
-      dst[h * (D + 2) + d] = acc;
-    } else {
-      dst[h * (D + 2) + D] = M;
-      dst[h * (D + 2) + D + 1] = acc;
+    s_M[h] = M;
+    s_L[h] = L;
+  }
+  __syncthreads();
+  float* pb = part + static_cast<int64_t>(bg) * nsplit * G * C::kPart;
+  {
+    float* dst = pb + static_cast<int64_t>(sp) * G * C::kPart;
+    for (int e = threadIdx.x; e < G * D; e += 32 * kAttWarps) {
+      const int h = e / D, d = e % D;
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kAttWarps; ++w) acc += s_wgt[w][h] * mw[(w * 16 + h) * C::kRow + d];
+      dst[h * C::kPart + d] = acc;
+    }
+    if (threadIdx.x < G) {
+      dst[threadIdx.x * C::kPart + D] = s_M[threadIdx.x];
+      dst[threadIdx.x * C::kPart + D + 1] = s_L[threadIdx.x];
     }
   }
-}
 
-// ---------------------------------------------------------------- F: combine + advance
-// grid (batch*h_kv, G), D threads: one (sequence, group, head) per CTA.  The
-// split weights 2^(m_s - M) are computed once in shared memory, then each
-// thread folds its column of d over the splits (coalesced across threads).
-template <int D>
-__global__ void __launch_bounds__(D) combine_kernel(const float* __restrict__ part, int nsplit, int h_q, int h_kv,
-                                                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ seq_len) {
-  extern __shared__ float cw[];           // [nsplit] weights
-  __shared__ float red[D / 32];
-  __shared__ float s_M, s_L;
-  const int bg = blockIdx.x, h = blockIdx.y;
-  const int b = bg / h_kv, g = bg % h_kv;
-  const int G = gridDim.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float* base = part + (static_cast<int64_t>(bg) * nsplit * G + h) * (D + 2);
-  const int64_t sstride = static_cast<int64_t>(G) * (D + 2);
-  float m = -INFINITY;
-  for (int s2 = tid; s2 < nsplit; s2 += D) m = fmaxf(m, base[s2 * sstride + D]);
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[warp] = m;
+  // ---- the last CTA of (b, g) to finish merges the splits
+  __threadfence();
   __syncthreads();
-  if (tid == 0) {
+  if (threadIdx.x == 0) s_last = (atomicAdd(&cnt[nbg + bg], 1u) == nsplit - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // split maxima and sums, all loaded at once
+  float* wsp = reinterpret_cast<float*>(att_smem);          // [nsplit][16] maxima, then weights
+  float* lsp = wsp + kMaxSplits * 16;                        // [nsplit][16] row sums
+  for (int e = threadIdx.x; e < nsplit * 16; e += 32 * kAttWarps) {
+    const int s2 = e >> 4, h = e & 15;
+    const float2 ml = (h < G) ? __ldcg(reinterpret_cast<const float2*>(pb + (static_cast<int64_t>(s2) * G + h) * C::kPart + D))
+                              : make_float2(-INFINITY, 0.f);
+    wsp[e] = ml.x;
+    lsp[e] = ml.y;
+  }
+  __syncthreads();
+  if (threadIdx.x < 16) {
+    const int h = threadIdx.x;
     float M = -INFINITY;
-    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
-    s_M = M;
-  }
-  __syncthreads();
-  const float M = s_M;
-  float l = 0.f;
-  for (int s2 = tid; s2 < nsplit; s2 += D) {
-    const float ms = base[s2 * sstride + D];
-    const float wgt = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
-    cw[s2] = wgt;
-    l += base[s2 * sstride + D + 1] * wgt;
-  }
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  __syncthreads();
-  if (lane == 0) red[warp] = l;
-  __syncthreads();
-  if (tid == 0) {
+    for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, wsp[s2 * 16 + h]);
     float L = 0.f;
-    for (int w = 0; w < D / 32; ++w) L += red[w];
-    s_L = L;
+    for (int s2 = 0; s2 < nsplit; ++s2) {
+      const float ms = wsp[s2 * 16 + h];
+      if (ms != -INFINITY) L += ex2(ms - M) * lsp[s2 * 16 + h];
+    }
+    s_M[h] = M;
+    s_L[h] = (L > 0.f) ? 1.f / L : 0.f;
   }
   __syncthreads();
-  float o = 0.f;
-  for (int s2 = 0; s2 < nsplit; ++s2) {
-    const float wgt = cw[s2];
-    if (wgt != 0.f) o += base[s2 * sstride + tid] * wgt;
+  for (int e = threadIdx.x; e < nsplit * 16; e += 32 * kAttWarps) {
+    const int h = e & 15;
+    const float ms = wsp[e];
+    wsp[e] = (ms == -INFINITY) ? 0.f : ex2(ms - s_M[h]) * s_L[h];
   }
-  const float L = s_L;
-  out[(static_cast<int64_t>(b) * h_q + g * G + h) * D + tid] = __float2bfloat16_rn(L > 0.f ? o / L : 0.f);
-  // advance the sequence: nothing in this kernel reads seq_len, and every
-  // kernel before it in the step has finished
-  if (g == 0 && h == 0 && tid == 0) seq_len[b] = seq_len[b] + 1;
+  __syncthreads();
+  // out[h, 4 q .. 4 q + 3] = sum over splits of weight * O: thread items
+  // it = tid + 128 k (k < 4) cover the G * D / 4 (head, quad) pairs; four
+  // splits of all four items are in flight at once
+  {
+    constexpr int kIt = 4, kU = 4;
+    const int nitems = G * (D / 4);
+    float4 acc[kIt];
+#pragma unroll
+    for (int k = 0; k < kIt; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < nsplit; s0 += kU) {
+      float4 v[kIt][kU];
+#pragma unroll
+      for (int k = 0; k < kIt; ++k) {
+        const int it = threadIdx.x + 32 * kAttWarps * k;
+        const int h = it / (D / 4), q4 = it % (D / 4);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const bool ok = it < nitems && s0 + u < nsplit;
+          v[k][u] = ok ? __ldcg(reinterpret_cast<const float4*>(pb + (static_cast<int64_t>(s0 + u) * G + h) * C::kPart) + q4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kIt; ++k) {
+        const int it = threadIdx.x + 32 * kAttWarps * k;
+        const int h = min(it / (D / 4), 15);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const float wg = (s0 + u < nsplit) ? wsp[(s0 + u) * 16 + h] : 0.f;
+          acc[k].x = fmaf(wg, v[k][u].x, acc[k].x);
+          acc[k].y = fmaf(wg, v[k][u].y, acc[k].y);
+          acc[k].z = fmaf(wg, v[k][u].z, acc[k].z);
+          acc[k].w = fmaf(wg, v[k][u].w, acc[k].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kIt; ++k) {
+      const int it = threadIdx.x + 32 * kAttWarps * k;
+      if (it < nitems) {
+        const int h = it / (D / 4), q4 = it % (D / 4);
+        uint2 w2;
+        w2.x = pack_bf16(acc[k].x, acc[k].y);
+        w2.y = pack_bf16(acc[k].z, acc[k].w);
+        *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b) * h_q + g * G + h) * D + 4 * q4) = w2;
+      }
+    }
+  }
+  // every CTA of every group of b has read seq_len[b] once all groups got here
+  if (threadIdx.x == 0 && atomicAdd(&cnt[2 * nbg + b], 1u) == static_cast<unsigned>(h_kv) - 1) seq_len[b] = t + 1;
 }
 
 // ---------------------------------------------------------------- pooled caches of a prefix
@@ -862,10 +994,13 @@ __global__ void __launch_bounds__(256) build_caches_kernel(const __nv_bfloat16* 
 // ---------------------------------------------------------------- host side
 struct DecodePlan {
   int cap_c1, cap_c2, nblk_cap, cand_cap, nsplit2, nsplit1, nsplit, bps, n_sel;
-  size_t off_part2, off_bscore, off_idx, off_part, bytes;
+  size_t off_part2, off_bscore, off_idx, off_part, off_cnt, bytes;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Largest capacity whose candidate keys fit the selecting CTA's shared memory.
+static bool decode_plan_supported(const DecodePlan& p) { return static_cast<size_t>(p.cand_cap) * 4 <= 160 * 1024; }
 
 DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_sel, int sms) {
   DecodePlan p{};
@@ -877,8 +1012,8 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   p.nsplit2 = std::max(1, (p.cap_c2 + dec::kLseWin - 1) / dec::kLseWin);
   p.nsplit1 = std::max(1, (p.cap_c1 + dec::kScoreWin) / dec::kScoreWin);
   const int bg = batch * h_kv;
-  // attention splits: about three CTAs of the attention kernel per SM
-  const int per_bg = std::max(1, (3 * sms) / std::max(1, bg));
+  // attention splits: about three attention CTAs per SM
+  const int per_bg = std::min(dec::kMaxSplits, std::max(1, (3 * sms) / std::max(1, bg)));
   p.bps = std::max(1, (n_sel + per_bg - 1) / per_bg);
   p.nsplit = std::max(1, (n_sel + p.bps - 1) / p.bps);
   const int G = h_q / h_kv;
@@ -886,55 +1021,49 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   p.off_part2 = off; off = align256(off + static_cast<size_t>(bg) * p.nsplit2 * 16 * sizeof(float2));
   p.off_bscore = off; off = align256(off + static_cast<size_t>(bg) * p.nblk_cap * sizeof(float));
   p.off_idx = off; off = align256(off + static_cast<size_t>(bg) * n_sel * sizeof(int32_t));
-  p.off_part = off; off = align256(off + static_cast<size_t>(bg) * p.nsplit * G * (d + 2) * sizeof(float));
+  p.off_part = off; off = align256(off + static_cast<size_t>(bg) * p.nsplit * G * (d + 4) * sizeof(float));
+  p.off_cnt = off; off = align256(off + static_cast<size_t>(2 * bg + batch) * sizeof(unsigned));
   p.bytes = off;
   return p;
 }
 
-
 template <int D>
 static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, const void* k_new, const void* v_new,
                                  void* out, void* ws, const DecodePlan& P, int n_init, int n_local, int top_k,
-                                 float scale, cudaStream_t st, bool* map_fail) {
+                                 float scale, cudaStream_t st) {
   using bf = __nv_bfloat16;
-  *map_fail = false;                       // the decode step builds no tensor maps
   const int bg = s->batch * s->h_kv;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float2* part2 = reinterpret_cast<float2*>(w + P.off_part2);
   float* bscore = reinterpret_cast<float*>(w + P.off_bscore);
   int32_t* idx = reinterpret_cast<int32_t*>(w + P.off_idx);
   float* part = reinterpret_cast<float*>(w + P.off_part);
-  dec::append_kernel<D><<<bg, 128, 0, st>>>(static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
-                                            static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache),
-                                            static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2), s->seq_len,
-                                            s->capacity, s->h_kv, P.cap_c1, P.cap_c2);
-  dec::lse_kernel<D><<<dim3(bg, P.nsplit2), 128, 0, st>>>(static_cast<const bf*>(q), static_cast<const bf*>(s->k_c2),
-                                                          s->seq_len, s->h_q, s->h_kv, P.cap_c2, scale, part2);
-  dec::score_pool_kernel<D><<<dim3(bg, P.nsplit1), 256, 0, st>>>(
-      static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->h_q, s->h_kv,
-      P.cap_c1, P.nblk_cap, scale, bscore);
+  unsigned* cnt = reinterpret_cast<unsigned*>(w + P.off_cnt);
+  dec::lse_append_kernel<D><<<dim3(bg, P.nsplit2), 128, 0, st>>>(
+      static_cast<const bf*>(q), static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
+      static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache), static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2),
+      s->seq_len, s->capacity, s->h_q, s->h_kv, P.cap_c1, P.cap_c2, scale, part2, cnt);
   const size_t sel_smem = static_cast<size_t>(P.cand_cap) * 4;
-  cudaError_t e = cudaFuncSetAttribute(dec::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(dec::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sel_smem));
   if (e != cudaSuccess) return e;
-  dec::select_kernel<<<bg, dec::kSelThreads, sel_smem, st>>>(bscore, s->seq_len, s->h_kv, P.nblk_cap, P.cand_cap,
-                                                             n_init, n_local, top_k, P.n_sel, idx);
+  dec::score_select_kernel<D><<<dim3(bg, P.nsplit1), dec::kSelThreads, sel_smem, st>>>(
+      static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->capacity, s->h_q,
+      s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt);
   e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(dec::AttCfg<D>::kSmem));
   if (e != cudaSuccess) return e;
   dec::attend_kernel<D><<<dim3(bg, P.nsplit), 32 * dec::kAttWarps, dec::AttCfg<D>::kSmem, st>>>(
       static_cast<const bf*>(q), static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache), idx,
-      s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps, scale, part);
-  dec::combine_kernel<D><<<dim3(bg, s->h_q / s->h_kv), D, P.nsplit * sizeof(float), st>>>(
-      part, P.nsplit, s->h_q, s->h_kv, static_cast<bf*>(out), s->seq_len);
+      s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps, scale, part, static_cast<bf*>(out), cnt);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_step(const infllm2_decode_state* s, const void* q, const void* k_new, const void* v_new,
                                void* out, void* ws, const DecodePlan& P, int n_init, int n_local, int top_k,
-                               float scale, cudaStream_t st, bool* map_fail) {
-  if (s->d == 128) return decode_step_t<128>(s, q, k_new, v_new, out, ws, P, n_init, n_local, top_k, scale, st, map_fail);
-  return decode_step_t<64>(s, q, k_new, v_new, out, ws, P, n_init, n_local, top_k, scale, st, map_fail);
+                               float scale, cudaStream_t st) {
+  if (s->d == 128) return decode_step_t<128>(s, q, k_new, v_new, out, ws, P, n_init, n_local, top_k, scale, st);
+  return decode_step_t<64>(s, q, k_new, v_new, out, ws, P, n_init, n_local, top_k, scale, st);
 }
 
 cudaError_t launch_decode_build_caches(const infllm2_decode_state* s, const DecodePlan& P, cudaStream_t st) {

@@ -249,17 +249,22 @@ static int check_decode_state(const infllm2_decode_state* s) {
   return check_heads(s->h_q, s->h_kv, s->d);
 }
 
+static DecodePlan plan_of(const infllm2_decode_state* st, const infllm2_params* p) {
+  return decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d, p->n_init + p->n_local + p->top_k,
+                     num_sms());
+}
+
 size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infllm2_params* p) {
   if (check_decode_state(st) || check_params(p)) return 0;
-  return decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d, p->n_init + p->n_local + p->top_k,
-                     num_sms()).bytes;
+  const DecodePlan P = plan_of(st, p);
+  return decode_plan_supported(P) ? P.bytes : 0;
 }
 
 int infllm2_decode_build_caches(const infllm2_decode_state* st, const infllm2_params* p, void* stream) {
   int r;
   if ((r = check_decode_state(st)) || (r = check_params(p))) return r;
-  const DecodePlan P = decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d,
-                                   p->n_init + p->n_local + p->top_k, num_sms());
+  const DecodePlan P = plan_of(st, p);
+  if (!decode_plan_supported(P)) return INFLLM2_ERR_UNSUPPORTED;
   cudaError_t e = launch_decode_build_caches(st, P, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
@@ -271,13 +276,11 @@ int infllm2_decode_step(const infllm2_decode_state* st, const void* q, const voi
   if (!q || !k_new || !v_new || !out || !workspace || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
       !aligned16(out) || !aligned16(workspace))
     return INFLLM2_ERR_INVALID_ARG;
-  const DecodePlan P = decode_plan(st->batch, st->capacity, st->h_q, st->h_kv, st->d,
-                                   p->n_init + p->n_local + p->top_k, num_sms());
+  const DecodePlan P = plan_of(st, p);
+  if (!decode_plan_supported(P)) return INFLLM2_ERR_UNSUPPORTED;
   if (workspace_bytes < P.bytes) return INFLLM2_ERR_WORKSPACE_TOO_SMALL;
-  bool map_fail = false;
   cudaError_t e = launch_decode_step(st, q, k_new, v_new, out, workspace, P, p->n_init, p->n_local, p->top_k,
-                                     softmax_scale(p, st->d), static_cast<cudaStream_t>(stream), &map_fail);
-  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
+                                     softmax_scale(p, st->d), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
 
