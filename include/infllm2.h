@@ -195,10 +195,22 @@ int infllm2_select_blocks_noalloc(const void* Q, const void* K_c1, const void* K
  *   out[t,h] = softmax_u(scale * q[t,h] . K[u,g]) V[u,g]
  * over u <= t with u / 64 in block_idx[g, t, :] (entries < 0 ignored).
  *   out  [total, h_q, d], bf16 (INFLLM2_OUT_BF16) or fp32 (INFLLM2_OUT_F32)
+ * Each row of block_idx must be ascending (valid entries first, then -1)
+ * and must hold the row's init blocks (0 .. min(n_init, b_t + 1) - 1) and
+ * its local run (the n_local blocks ending at b_t = t / 64), as every list
+ * of infllm2_select_blocks / infllm2_topk_blocks does: the shared init and
+ * local blocks are attended once per group of query tokens and the other
+ * entries per token, and the two partials are merged.  A row that breaks
+ * this rule gets a wrong result (no fault).
+ * workspace: device, 16-byte aligned, at least
+ * infllm2_sparse_workspace_bytes(vl, h_q) bytes (one fp32 per (token,
+ * query head)); nothing in it outlives the call's kernels.
  * ------------------------------------------------------------------- */
+size_t infllm2_sparse_workspace_bytes(const infllm2_varlen* vl, int32_t h_q);
 int infllm2_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* block_idx,
                         const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
-                        void* out, int32_t out_dtype, const infllm2_params* p, void* stream);
+                        void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                        const infllm2_params* p, void* stream);
 
 /* Dense causal attention, the short-sequence side of the dense/sparse switch
  * ([blog] "Dense-Sparse Switchable Attention"; [news] §二.2.c).  Same

@@ -48,6 +48,8 @@ class GpuRun:
         self.idx = torch.empty(w.h_kv, self.vl.total, self.p.n_sel, dtype=torch.int32, device=dev)
         self.out = torch.empty(self.vl.total, w.h_q, d,
                                dtype=torch.float32 if w.out_fp32 else torch.bfloat16, device=dev)
+        self.sws = torch.empty(max(256, T.infllm2_sparse_workspace_bytes(self.vl, w.h_q)), dtype=torch.uint8,
+                               device=dev)
 
     def compress(self):
         T.infllm2_compress_k(self.K, self.vl, self.Kc1, self.Kc2, self.p)
@@ -59,7 +61,8 @@ class GpuRun:
         T.infllm2_topk_blocks(self.S if S is None else S, self.ld, self.vl, self.w.h_kv, self.idx, self.p)
 
     def sparse(self, idx=None):
-        T.infllm2_sparse_attn(self.Q, self.K, self.V, self.idx if idx is None else idx, self.vl, self.out, self.p)
+        T.infllm2_sparse_attn(self.Q, self.K, self.V, self.idx if idx is None else idx, self.vl, self.out, self.p,
+                              workspace=self.sws)
 
     def dense(self):
         T.infllm2_dense_attn(self.Q, self.K, self.V, self.vl, self.out, self.p)

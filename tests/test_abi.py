@@ -85,7 +85,16 @@ def test_argument_errors_are_caught_on_host(L):
     assert L.infllm2_select_blocks(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 16, 0x1000, None, by(p),
                                    None) == -3
     # bad output dtype
-    assert L.infllm2_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 7, by(p), None) == -1
+    ws = T.infllm2_sparse_workspace_bytes(vl, 4)
+    assert L.infllm2_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 7, 0x1000, ws, by(p),
+                                 None) == -1
+    # sparse workspace missing, misaligned or too small
+    assert L.infllm2_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 0, None, ws, by(p),
+                                 None) == -1
+    assert L.infllm2_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 0, 0x1008, ws, by(p),
+                                 None) == -1
+    assert L.infllm2_sparse_attn(0x1000, 0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 0, 0x1000, ws - 4, by(p),
+                                 None) == -3
     # inconsistent varlen
     bad = _vl(batch=0)
     assert L.infllm2_dense_attn(0x1000, 0x1000, 0x1000, by(bad), 4, 1, 64, 0x1000, 0, by(p), None) == -1
@@ -97,3 +106,5 @@ def test_argument_errors_are_caught_on_host(L):
 def test_workspace_size(L):
     vl = _vl(max_seqlen=131072, total=131072)
     assert T.infllm2_select_workspace_bytes(vl, 2) == 2 * 131072 * 8192 * 4
+    # one fp32 log-sum-exp per (token, query head)
+    assert T.infllm2_sparse_workspace_bytes(vl, 32) == 131072 * 32 * 4

@@ -20,7 +20,8 @@ from . import build as _build
 __all__ = [
     "InfLLM2Error", "Params", "Varlen", "lib", "default_params", "make_varlen", "window_count",
     "infllm2_compress_k", "infllm2_shared_scores", "infllm2_topk_blocks", "infllm2_select_blocks",
-    "infllm2_select_workspace_bytes", "infllm2_scores_ld", "infllm2_sparse_attn", "infllm2_dense_attn",
+    "infllm2_select_workspace_bytes", "infllm2_scores_ld", "infllm2_sparse_workspace_bytes", "infllm2_sparse_attn",
+    "infllm2_dense_attn",
     "infllm2_get_device_status", "infllm2_clear_device_status", "infllm2_debug_wait_timeout",
     "DecodeState", "make_decode_state", "infllm2_decode_workspace_bytes", "infllm2_decode_build_caches",
     "infllm2_decode_step", "OUT_BF16", "OUT_F32",
@@ -88,7 +89,9 @@ def lib() -> ctypes.CDLL:
         "infllm2_topk_blocks": (ctypes.c_int, [_P, i64, vp, i32, _P, pp, _P]),
         "infllm2_select_workspace_bytes": (ctypes.c_size_t, [vp, i32, pp]),
         "infllm2_select_blocks": (ctypes.c_int, [_P, _P, _P, vp, i32, i32, i32, _P, ctypes.c_size_t, _P, _P, pp, _P]),
-        "infllm2_sparse_attn": (ctypes.c_int, [_P, _P, _P, _P, vp, i32, i32, i32, _P, i32, pp, _P]),
+        "infllm2_sparse_workspace_bytes": (ctypes.c_size_t, [vp, i32]),
+        "infllm2_sparse_attn": (ctypes.c_int, [_P, _P, _P, _P, vp, i32, i32, i32, _P, i32, _P, ctypes.c_size_t, pp,
+                                                _P]),
         "infllm2_dense_attn": (ctypes.c_int, [_P, _P, _P, vp, i32, i32, i32, _P, i32, pp, _P]),
         "infllm2_get_device_status": (ctypes.c_int, []),
         "infllm2_clear_device_status": (ctypes.c_int, []),
@@ -198,13 +201,24 @@ def infllm2_select_blocks(Q: torch.Tensor, K_c1: torch.Tensor, K_c2: torch.Tenso
     _check("infllm2_select_blocks", rc)
 
 
+def infllm2_sparse_workspace_bytes(vl: Varlen, h_q: int) -> int:
+    return lib().infllm2_sparse_workspace_bytes(ctypes.byref(vl), h_q)
+
+
 def infllm2_sparse_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block_idx: torch.Tensor, vl: Varlen,
-                        out: torch.Tensor, params: Optional[Params] = None, stream=None) -> None:
+                        out: torch.Tensor, params: Optional[Params] = None, stream=None,
+                        workspace: Optional[torch.Tensor] = None) -> None:
+    """`workspace`: a device byte tensor of at least infllm2_sparse_workspace_bytes(vl, h_q) bytes; one is
+    allocated for the call when it is None."""
     h_q, d = Q.shape[1], Q.shape[2]
     h_kv = K.shape[1]
     od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    need = infllm2_sparse_workspace_bytes(vl, h_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=Q.device)
     rc = lib().infllm2_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(block_idx), ctypes.byref(vl), h_q, h_kv, d,
-                                   _ptr(out), od, ctypes.byref(params or default_params()), _stream(stream))
+                                   _ptr(out), od, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   ctypes.byref(params or default_params()), _stream(stream))
     _check("infllm2_sparse_attn", rc)
 
 

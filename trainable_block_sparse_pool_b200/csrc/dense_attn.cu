@@ -2,9 +2,20 @@
 // switch (paper-reading blog, "Dense-Sparse Switchable Attention"; dtcms
 // article §二.2.c).  Same inputs and output form as the sparse kernel.
 //
+// The same kernel, in its LOCAL form, computes the shared part of the
+// block-sparse attention: every query token attends to its init blocks and
+// to the n_local blocks that end at its own block (top168 article §七), and
+// these are the same for all tokens of a 64-token block.  Attending to them
+// once per CTA of 128/G tokens (instead of once per token) leaves only the
+// top-k blocks to the per-token sparse kernel, which runs first and leaves
+// its normalised partial in out and its log-sum-exp in lse; the row's thread
+// here merges the two partials through their log-sum-exps.
+//
 // A CTA owns one kv group and TQ = 128/G consecutive query tokens: its 128
 // query rows (t, h) share every key of the group, so one K/V tile feeds all
-// of them (GQA packing).  Per 128-key tile:
+// of them (GQA packing).  A tile is two 64-key blocks, each gathered by TMA
+// (dense: blocks 2i, 2i+1; LOCAL: consecutive blocks of the CTA's init and
+// local range).  Per 128-key tile:
 //   S[128 rows, 128 keys] = Q . K^T        tcgen05, A = Q (smem), B = K (smem)
 //   softmax, one thread per row (two passes over the TMEM row: max, then
 //   exp2 + bf16 P written to shared memory in the 128-byte-swizzled K-major
@@ -55,11 +66,31 @@ struct Bars {
 __device__ __forceinline__ bool aborted(const Bars* b) { return *reinterpret_cast<const volatile int*>(&b->abort) != 0; }
 __device__ __forceinline__ void set_abort(Bars* b) { *reinterpret_cast<volatile int*>(&b->abort) = 1; }
 
-template <int D, int G, bool OUT_F32>
+// The blocks a CTA walks.  Dense: 0 .. t_last/64.  LOCAL: the init blocks
+// [0, i_hi) followed by [l_start, b_hi], the union of the init and local
+// blocks of the CTA's query tokens (blocks b_lo .. b_hi); block(p) < 0 past
+// the end.  in_set tells whether block blk is shared for query token t.
+struct BlockWalk {
+  int i_hi, l_start, nblk;
+  __device__ int block(int p) const { return p >= nblk ? -1 : (p < i_hi ? p : l_start + (p - i_hi)); }
+};
+__device__ __forceinline__ BlockWalk local_walk(int b_lo, int b_hi, int n_init, int n_local) {
+  BlockWalk w;
+  w.i_hi = min(n_init, b_hi + 1);
+  w.l_start = max(w.i_hi, max(0, b_lo - n_local + 1));
+  w.nblk = w.i_hi + max(0, b_hi - w.l_start + 1);
+  return w;
+}
+__device__ __forceinline__ bool in_set(int blk, int t, int n_init, int n_local) {
+  const int bt = t >> 6;
+  return blk < min(n_init, bt + 1) || blk >= bt - n_local + 1;
+}
+
+template <int D, int G, bool OUT_F32, bool LOCAL>
 __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu, int h_q, float scale,
-    void* __restrict__ out) {
+    void* __restrict__ out, int n_init, int n_local, float* __restrict__ lse) {
   using C = Cfg<D, G>;
   constexpr int TQ = C::TQ;
   static_assert(G >= 1 && G <= 16 && (16 % G) == 0, "group size must be a power of two <= 16");
@@ -78,7 +109,15 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
   if (static_cast<int>(blockIdx.x) >= ntiles) return;
   const int t0 = (ntiles - 1 - blockIdx.x) * TQ;        // heaviest query tiles first
   const int t_last = min(len - 1, t0 + TQ - 1);
-  const int nkt = t_last / kKeys + 1;                    // key tiles covering 0 .. t_last
+  BlockWalk walk;
+  if (LOCAL) {
+    walk = local_walk(t0 >> 6, t_last >> 6, n_init, n_local);
+  } else {
+    walk.i_hi = t_last / 64 + 1;
+    walk.l_start = walk.i_hi;
+    walk.nblk = walk.i_hi;
+  }
+  const int nkt = (walk.nblk + 1) / 2;                   // tiles of two blocks
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -111,10 +150,15 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
         if (!mbar_wait(&bars->kv_empty[st], ((it / kStages) & 1) ^ 1) || aborted(bars)) { set_abort(bars); break; }
         uint8_t* dK = sKV + st * C::kStageBytes;
         uint8_t* dV = dK + C::kKBytes;
+        const int ba = walk.block(2 * it);
+        int bb = walk.block(2 * it + 1);
+        if (bb < 0) bb = ba;                             // odd count: reload, masked by the softmax
         mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
         for (int ch = 0; ch < C::KCH; ++ch) {
-          tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, g, row0 + it * kKeys);
-          tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, g, row0 + it * kKeys);
+          tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, g, row0 + 64 * ba);
+          tma_load_3d(dK + ch * C::kChunk + C::kChunk / 2, &tmK, &bars->kv_full[st], ch * 64, g, row0 + 64 * bb);
+          tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, g, row0 + 64 * ba);
+          tma_load_3d(dV + ch * C::kChunk + C::kChunk / 2, &tmV, &bars->kv_full[st], ch * 64, g, row0 + 64 * bb);
         }
       }
       mbar_wait(&bars->q_full, 0);
@@ -187,14 +231,23 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_addr + sb * kKeys;
-      const int kbase = it * kKeys;
+      // keys of this tile: half e is block walk.block(2 it + e); key i of a
+      // 16-key group at cc is token ubase[e] + (cc & 63) + i (visible when
+      // <= t); a block the row does not share is masked whole
+      int ub0, ub1;
+      {
+        const int blk0 = walk.block(2 * it), blk1 = walk.block(2 * it + 1);
+        ub0 = (blk0 >= 0 && (!LOCAL || in_set(blk0, t, n_init, n_local))) ? 64 * blk0 : INT_MAX / 2;
+        ub1 = (blk1 >= 0 && (!LOCAL || in_set(blk1, t, n_init, n_local))) ? 64 * blk1 : INT_MAX / 2;
+      }
       float mx = -INFINITY;
 #pragma unroll 1
       for (int cc = 0; cc < kKeys; cc += 16) {
         float v[16];
         tmem_load16(s_addr + cc, v);
+        const int u0 = ((cc >> 6) ? ub1 : ub0) + (cc & 63);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) if (kbase + cc + i <= t) mx = fmaxf(mx, v[i] * c);
+        for (int i = 0; i < 16; ++i) if (u0 + i <= t) mx = fmaxf(mx, v[i] * c);
       }
       const float m_new = fmaxf(m_run, mx);
       const bool none = (m_new == -INFINITY);
@@ -204,21 +257,22 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       for (int cc = 0; cc < kKeys; cc += 16) {
         float v[16];
         tmem_load16(s_addr + cc, v);
+        const int u0 = ((cc >> 6) ? ub1 : ub0) + (cc & 63);
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const float p0 = (!none && kbase + cc + i <= t) ? ex2(fmaf(v[i], c, -m_new)) : 0.f;
-          const float p1 = (!none && kbase + cc + i + 1 <= t) ? ex2(fmaf(v[i + 1], c, -m_new)) : 0.f;
+          const float p0 = (!none && u0 + i <= t) ? ex2(fmaf(v[i], c, -m_new)) : 0.f;
+          const float p1 = (!none && u0 + i + 1 <= t) ? ex2(fmaf(v[i + 1], c, -m_new)) : 0.f;
           lsum += p0 + p1;
           __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
           pk[i >> 1] = *reinterpret_cast<uint32_t*>(&b2);
         }
         // keys cc .. cc+15 of this tile: chunk cc/64, 16-byte units (cc%64)/8 and +1
         const int chunk = cc >> 6;
-        const int u0 = (cc & 63) >> 3;
+        const int q0 = (cc & 63) >> 3;
         uint8_t* base = prow + chunk * 16384;
-        *reinterpret_cast<uint4*>(base + ((u0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(base + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        *reinterpret_cast<uint4*>(base + ((q0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(base + (((q0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
       l_run = l_run * alpha + lsum;
       m_run = m_new;
@@ -244,19 +298,55 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
     if (ok && t < len) {
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const int64_t base = (static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h) * D;
+      float w_own = inv;   // weight of o_acc; the top-k partial (if any) gets w_top
+      float w_top = 0.f;
+      if (LOCAL) {
+        // out[row] holds the top-k partial (normalised) when its log-sum-exp
+        // lb (log2 units) is finite; la is this partial's
+        const float lb = lse[static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h];
+        if (lb != -INFINITY && l_run > 0.f) {
+          const float la = m_run + log2f(l_run);
+          const float mm = fmaxf(la, lb);
+          const float wa = ex2(la - mm), wb = ex2(lb - mm);
+          const float iw = 1.f / (wa + wb);
+          w_own = inv * wa * iw;
+          w_top = wb * iw;
+        }
+      }
       if (OUT_F32) {
         float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + base);
 #pragma unroll
-        for (int j = 0; j < D; j += 4)
-          o4[j / 4] = make_float4(o_acc[j] * inv, o_acc[j + 1] * inv, o_acc[j + 2] * inv, o_acc[j + 3] * inv);
+        for (int j = 0; j < D; j += 4) {
+          float4 v = make_float4(o_acc[j] * w_own, o_acc[j + 1] * w_own, o_acc[j + 2] * w_own, o_acc[j + 3] * w_own);
+          if (LOCAL && w_top != 0.f) {
+            const float4 b4 = o4[j / 4];
+            v.x = fmaf(b4.x, w_top, v.x); v.y = fmaf(b4.y, w_top, v.y);
+            v.z = fmaf(b4.z, w_top, v.z); v.w = fmaf(b4.w, w_top, v.w);
+          }
+          o4[j / 4] = v;
+        }
       } else {
         uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + base);
 #pragma unroll
         for (int j = 0; j < D; j += 8) {
+          float top[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) top[q] = 0.f;
+          if (LOCAL && w_top != 0.f) {
+            const uint4 b4 = o4[j / 8];
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b4);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 f = __bfloat1622float2(b2[q]);
+              top[2 * q] = f.x * w_top;
+              top[2 * q + 1] = f.y * w_top;
+            }
+          }
           uint32_t w[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(o_acc[j + 2 * q] * inv, o_acc[j + 2 * q + 1] * inv);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(o_acc[j + 2 * q], w_own, top[2 * q]),
+                                                      fmaf(o_acc[j + 2 * q + 1], w_own, top[2 * q + 1]));
             w[q] = *reinterpret_cast<uint32_t*>(&b2);
           }
           o4[j / 8] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -276,10 +366,10 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
 bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                const uint32_t* box);
 
-template <int D, int G, bool F32>
+template <int D, int G, bool F32, bool LOCAL>
 static cudaError_t launch_dense_t(const void* Q, const void* K, const void* V, const int32_t* cu, int batch,
                                   int max_seqlen, int64_t total, int h_q, int h_kv, float scale, void* out,
-                                  cudaStream_t st, bool* map_fail) {
+                                  int n_init, int n_local, float* lse, cudaStream_t st, bool* map_fail) {
   using C = dense::Cfg<D, G>;
   CUtensorMap mQ, mK, mV;
   {
@@ -291,29 +381,38 @@ static cudaError_t launch_dense_t(const void* Q, const void* K, const void* V, c
   {
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)h_kv, (uint64_t)total};
     const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)h_kv * D * 2};
-    const uint32_t box[3] = {64, 1, dense::kKeys};
+    const uint32_t box[3] = {64, 1, 64};
     if (!make_tmap(&mK, K, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
     if (!make_tmap(&mV, V, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
   }
-  auto kern = dense::dense_attn_kernel<D, G, F32>;
+  auto kern = dense::dense_attn_kernel<D, G, F32, LOCAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((max_seqlen + C::TQ - 1) / C::TQ, batch, h_kv);
   if (grid.x == 0) return cudaSuccess;
-  kern<<<grid, dense::kThreads, C::kSmem, st>>>(mQ, mK, mV, cu, h_q, scale, out);
+  kern<<<grid, dense::kThreads, C::kSmem, st>>>(mQ, mK, mV, cu, h_q, scale, out, n_init, n_local, lse);
   return cudaGetLastError();
 }
 
+// Dense causal attention (lse == nullptr), or the LOCAL part of the sparse
+// attention: attention over each token's init and local blocks, merged with
+// the top-k partial that out and lse ([total, h_q] fp32, log2 units) hold.
 cudaError_t launch_dense_attn(const void* Q, const void* K, const void* V, const int32_t* cu, int batch,
                               int max_seqlen, int64_t total, int h_q, int h_kv, int d, float scale, void* out,
-                              bool out_f32, cudaStream_t st, bool* map_fail) {
+                              bool out_f32, int n_init, int n_local, float* lse, cudaStream_t st, bool* map_fail) {
   const int G = h_q / h_kv;
 #define INFLLM2_DENSE_CASE(DD, GG)                                                                               \
-  if (d == DD && G == GG)                                                                                       \
-    return out_f32 ? launch_dense_t<DD, GG, true>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, out, st, \
-                                                  map_fail)                                                    \
-                   : launch_dense_t<DD, GG, false>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, out, \
-                                                   st, map_fail);
+  if (d == DD && G == GG) {                                                                                     \
+    if (lse)                                                                                                    \
+      return out_f32 ? launch_dense_t<DD, GG, true, true>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, \
+                                                          out, n_init, n_local, lse, st, map_fail)             \
+                     : launch_dense_t<DD, GG, false, true>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, \
+                                                           out, n_init, n_local, lse, st, map_fail);           \
+    return out_f32 ? launch_dense_t<DD, GG, true, false>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, \
+                                                         out, 0, 0, nullptr, st, map_fail)                     \
+                   : launch_dense_t<DD, GG, false, false>(Q, K, V, cu, batch, max_seqlen, total, h_q, h_kv, scale, \
+                                                          out, 0, 0, nullptr, st, map_fail);                   \
+  }
   INFLLM2_DENSE_CASE(128, 16)
   INFLLM2_DENSE_CASE(128, 8)
   INFLLM2_DENSE_CASE(128, 4)

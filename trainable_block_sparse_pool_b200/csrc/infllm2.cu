@@ -208,19 +208,33 @@ int infllm2_select_blocks(const void* Q, const void* K_c1, const void* K_c2, con
   return infllm2_topk_blocks(S, ld, vl, h_kv, block_idx, p, stream);
 }
 
+size_t infllm2_sparse_workspace_bytes(const infllm2_varlen* vl, int32_t h_q) {
+  if (check_varlen(vl) || h_q <= 0) return 0;
+  return (static_cast<size_t>(vl->total) * h_q * sizeof(float) + 255) & ~size_t(255);
+}
+
 int infllm2_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* block_idx,
                         const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d, void* out, int32_t out_dtype,
-                        const infllm2_params* p, void* stream) {
+                        void* workspace, size_t workspace_bytes, const infllm2_params* p, void* stream) {
   int r;
   if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
   if (!Q || !K || !V || !block_idx || !out || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
     return INFLLM2_ERR_INVALID_ARG;
   if (out_dtype != INFLLM2_OUT_BF16 && out_dtype != INFLLM2_OUT_F32) return INFLLM2_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return INFLLM2_ERR_INVALID_ARG;
+  if (workspace_bytes < infllm2_sparse_workspace_bytes(vl, h_q)) return INFLLM2_ERR_WORKSPACE_TOO_SMALL;
   bool map_fail = false;
   const int n_sel = p->n_init + p->n_local + p->top_k;
+  const float scale = softmax_scale(p, d);
+  const bool f32 = out_dtype == INFLLM2_OUT_F32;
+  float* lse = static_cast<float*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the top-k blocks of each token, then the init and local blocks once per 128/G tokens, merged in
   cudaError_t e = launch_sparse_attn(Q, K, V, block_idx, vl->cu_seqlens, vl->batch, vl->total, h_q, h_kv, d, n_sel,
-                                     softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32,
-                                     static_cast<cudaStream_t>(stream), &map_fail);
+                                     p->n_init, p->n_local, scale, out, f32, lse, st, &map_fail);
+  if (e == cudaSuccess && !map_fail)
+    e = launch_dense_attn(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d, scale, out,
+                          f32, p->n_init, p->n_local, lse, st, &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
@@ -234,7 +248,7 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V, const infllm
   if (out_dtype != INFLLM2_OUT_BF16 && out_dtype != INFLLM2_OUT_F32) return INFLLM2_ERR_INVALID_ARG;
   bool map_fail = false;
   cudaError_t e = launch_dense_attn(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d,
-                                    softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32,
+                                    softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32, 0, 0, nullptr,
                                     static_cast<cudaStream_t>(stream), &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);

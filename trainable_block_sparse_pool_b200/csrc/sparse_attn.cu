@@ -3,7 +3,13 @@
 // single output — paper-reading blog, "对齐计算图"; top168 article §七).
 //
 // Work unit: one (kv group g, query token t).  Its G query heads share the
-// selected block list I(g,t) (|I| <= 96 blocks of 64 keys).  With G = 16 a
+// selected block list I(g,t) (|I| <= 96 blocks of 64 keys).  The init and
+// local blocks of I are the same for every token of a 64-token block, so
+// the dense kernel's LOCAL form attends to them once per 128/G tokens; this
+// kernel gathers only the top-k blocks of each token (the entries of the
+// ascending list between the init and the local run) and leaves its
+// normalised partial in out with its log-sum-exp, which the LOCAL kernel
+// (launched next) merges with its own.  With G = 16 a
 // unit is too small for the M dimension of tcgen05 (64 or 128), so the
 // contractions are transposed ("swap AB"): keys fill M, heads fill N.
 //   S^T [128 keys, 16] = K_pair[128, d]  . Q_t[16, d]^T      (M=128, N=16)
@@ -145,15 +151,16 @@ struct Unit {
 };
 
 // Unit u = (kv group, packed row), u = g * total + row; its list is
-// block_idx[g, row, :].
+// block_idx[g, row, :] without the shared (init and local) blocks.
 struct SparseArgs {
   const int32_t* block_idx;
   const int32_t* cu;
   int batch;
   int64_t total;       // packed rows
-  int h_q, h_kv, n_sel;
+  int h_q, h_kv, n_sel, n_init, n_local;
   float scale;
-  void* out;
+  void* out;           // the top-k partial, normalised (rows without top-k blocks are not written)
+  float* lse;          // [total, h_q] its log-sum-exp, log2 units (-inf: no top-k block)
 };
 
 __device__ __forceinline__ int64_t num_units(const SparseArgs& a) { return static_cast<int64_t>(a.h_kv) * a.total; }
@@ -165,9 +172,17 @@ __device__ __forceinline__ Unit get_unit(int64_t u, const SparseArgs& a) {
   const int s = find_sequence(a.cu, a.batch, x.row);
   x.seq_start = a.cu[s];
   x.t = static_cast<int>(x.row - x.seq_start);
-  x.I = a.block_idx + u * a.n_sel;
-  x.nlist = a.n_sel;
-  x.nvalid = count_valid(x.I, x.nlist);
+  const int32_t* list = a.block_idx + u * a.n_sel;
+  const int nall = count_valid(list, a.n_sel);
+  // the ascending list starts with the i_hi init blocks and ends with the
+  // local run; the top-k entries sit between them
+  const int bt = x.t >> 6;
+  const int i_hi = min(a.n_init, bt + 1);
+  const int l_start = max(i_hi, max(0, bt - a.n_local + 1));
+  const int nshared = i_hi + max(0, bt - l_start + 1);
+  x.I = list + i_hi;
+  x.nlist = a.n_sel - i_hi;
+  x.nvalid = max(0, nall - nshared);
   return x;
 }
 
@@ -538,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
       }
       ab = ab || aborted(bars);
       if (bar_red_or(bar_id, 128, ab)) { stop = true; break; }
-      if (kl < D) {
+      if (kl < D && nt > 0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float l = red_w[h] + red_w[16 + h] + red_w[32 + h] + red_w[48 + h];
@@ -547,6 +562,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
           if (OUT_F32) reinterpret_cast<float*>(args.out)[idx] = r;
           else reinterpret_cast<__nv_bfloat16*>(args.out)[idx] = __float2bfloat16_rn(r);
         }
+      }
+      if (kl < G) {
+        float mr = m_ref[0];
+#pragma unroll
+        for (int h = 1; h < 16; ++h) if (kl == h) mr = m_ref[h];
+        const float l = red_w[kl] + red_w[16 + kl] + red_w[32 + kl] + red_w[48 + kl];
+        args.lse[x.row * args.h_q + static_cast<int64_t>(x.g) * G + kl] =
+            (nt > 0 && l > 0.f) ? mr + log2f(l) : -INFINITY;
       }
       tc_fence_before();
       named_bar_sync(bar_id, 128);           // red_w and this O buffer are free again
@@ -595,12 +618,15 @@ static cudaError_t launch_sparse_t(const void* Q, const void* K, const void* V, 
   return cudaGetLastError();
 }
 
+// The top-k part of the sparse attention: its normalised partial into out,
+// its log-sum-exp into lse (the LOCAL kernel merges its own into both).
 cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cu,
-                               int batch, int64_t total, int h_q, int h_kv, int d, int n_sel, float scale,
-                               void* out, bool out_f32, cudaStream_t st, bool* map_fail) {
+                               int batch, int64_t total, int h_q, int h_kv, int d, int n_sel, int n_init,
+                               int n_local, float scale, void* out, bool out_f32, float* lse, cudaStream_t st,
+                               bool* map_fail) {
   sparse::SparseArgs a{};
   a.block_idx = idx; a.cu = cu; a.batch = batch; a.total = total; a.h_q = h_q; a.h_kv = h_kv; a.n_sel = n_sel;
-  a.scale = scale; a.out = out;
+  a.n_init = n_init; a.n_local = n_local; a.scale = scale; a.out = out; a.lse = lse;
   const int G = h_q / h_kv;
 #define INFLLM2_SPARSE_CASE(DD, GG)                                                            \
   if (d == DD && G == GG)                                                                     \
