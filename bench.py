@@ -49,21 +49,27 @@ def _peaks():
 
 
 # ---------------------------------------------------------------- work counts
-def visible_counts(n: int):
+def visible_counts(n: int, n_init: int = 1, n_local: int = 32, top_k: int = 63):
     """Per query position t of an n-token sequence: visible C1 windows, C2
-    windows and sparse keys (96 blocks of 64; the query's own block is the
-    only partial one)."""
+    windows, sparse keys (|I| blocks of 64; the query's own block is the
+    only partial one) and, of those, the keys of the shared blocks (init and
+    local, the query's own block among them) and of the top-k blocks."""
     t = np.arange(n, dtype=np.int64)
     n1 = np.where(t >= 31, (t - 31) // 16 + 1, 0)
     n2 = np.where(t >= 127, (t - 127) // 64 + 1, 0)
     b_t = t // 64
-    nsel = np.minimum(96, b_t + 1)
+    nsel = np.minimum(n_init + n_local + top_k, b_t + 1)
     keys = (nsel - 1) * 64 + (t % 64) + 1
-    return n1, n2, keys
+    i_hi = np.minimum(n_init, b_t + 1)
+    l_start = np.maximum(i_hi, b_t - n_local + 1)
+    nshared = i_hi + np.maximum(0, b_t - l_start + 1)
+    shared_keys = (nshared - 1) * 64 + (t % 64) + 1
+    topk_keys = keys - shared_keys
+    return n1, n2, keys, shared_keys, topk_keys
 
 
 def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
-    n1, n2, keys = visible_counts(n)
+    n1, n2, keys, shared_keys, topk_keys = visible_counts(n)
     G = h_q // h_kv
     ld = ((n - 32) // 16 + 1 + 3) // 4 * 4
     w = {}
@@ -78,9 +84,43 @@ def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
     # sparse attention: QK^T and PV over the visible selected keys
     w["sparse_flops"] = 4 * d * h_q * int(keys.sum())
     w["sparse_exps"] = h_q * int(keys.sum())
-    w["sparse_gather_bytes"] = h_kv * 2 * d * 2 * int(keys.sum())
+    # K and V rows moved L2 -> SM: the top-k blocks of every (token, group),
+    # and the shared blocks once per CTA of 128/G tokens (the union over its
+    # tokens: one 64-token block's init and local blocks when 128/G <= 64)
+    tq = 128 // G
+    t0 = np.arange(0, n, tq)
+    b0 = t0 // 64
+    shared_blocks = np.minimum(1, b0 + 1) + np.maximum(0, b0 - np.maximum(np.minimum(1, b0 + 1), b0 - 31) + 1)
+    w["sparse_topk_gather_bytes"] = h_kv * 2 * d * 2 * int(topk_keys.sum())
+    w["sparse_shared_gather_bytes"] = h_kv * 2 * d * 2 * 64 * int(shared_blocks.sum())
+    w["sparse_gather_bytes"] = w["sparse_topk_gather_bytes"] + w["sparse_shared_gather_bytes"]
     w["ld"] = ld
     return w
+
+
+# ---------------------------------------------------------------- L2 gather probe
+def measure_l2_gather(T, torch, K, V, stream, target_bytes: float = 8e9, reps: int = 3) -> dict:
+    """Best L2 -> SM gather bandwidth (GB/s) over the probe's producer counts:
+    random pairs of 64-key blocks of K and V of one kv group (the first
+    2048 blocks, 67 MB: L2-resident), 192 KB in flight per SM."""
+    nsm = torch.cuda.get_device_properties(K.device).multi_processor_count
+    nblk = min(2048, K.shape[0] // 64)
+    out = {}
+    for prod in (1, 2, 3, 6):
+        tiles = max(1, int(target_bytes / (nsm * prod * 32768)))
+        T.infllm2_probe_l2_gather(K, V, nblk, tiles, prod, stream)
+        best = None
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            T.infllm2_probe_l2_gather(K, V, nblk, tiles, prod, stream)
+            b.record(stream)
+            b.synchronize()
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+        out[f"producers_{prod}"] = nsm * prod * tiles * 32768 / (best / 1e3) / 1e9
+    return {"GB/s": max(out.values()), "variants": out, "footprint_MB": 2 * nblk * 64 * K.shape[1] * 256 / 1e6}
 
 
 # ---------------------------------------------------------------- ranks
@@ -406,14 +446,19 @@ def main():
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
+    # ---- L2 -> SM gather bandwidth with the attention's tile shape (this run)
+    l2 = measure_l2_gather(T, torch, K, V, stream)
+
     # ---- roofline of the dominant kernel
     hbm, tflops, tflops_sus, src = _peaks()
     work = algorithmic_work(w.seqlen, w.h_q, w.h_kv, w.d)
     dom = max(per_kernel, key=per_kernel.get)
     if dom == "sparse":
-        ach = work["sparse_flops"] / (per_kernel["sparse"] / 1e3) / 1e12
-        roof = {"kernel": "sparse_attn", "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
-                "frac": ach / tflops, "traffic": None, "peak_source": f"{src} bf16 burst"}
+        # the top-k gather (and the shared tiles) are L2 -> SM bound: see the design doc
+        ach = work["sparse_gather_bytes"] / (per_kernel["sparse"] / 1e3) / 1e9
+        roof = {"kernel": "sparse_attn (top-k gather + shared init/local tiles)", "bound": "l2", "achieved": ach,
+                "peak": l2["GB/s"], "unit": "GB/s", "frac": ach / l2["GB/s"], "traffic": None,
+                "peak_source": "L2 gather probe, same tile shape, same run (measured)"}
     elif dom == "scores":
         ach = work["score_flops"] / (per_kernel["scores"] / 1e3) / 1e12
         roof = {"kernel": "shared_scores", "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
@@ -423,6 +468,26 @@ def main():
         ach = b / (per_kernel[dom] / 1e3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                 "traffic": None, "peak_source": f"{src} HBM copy"}
+
+    # ---- the whole step against the sum of its steps' rooflines (each step's
+    # time bound = the slowest of tensor, SFU exp, HBM and L2-gather time)
+    sm_mhz = (clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0) if isinstance(clk, dict) else 1965.0
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu = 16.0 * nsm * sm_mhz * 1e6            # ex2 per second: 16 per SM per clock
+    tens = tflops_sus * 1e12                   # a long step: the sustained GEMM figure
+    bw = hbm * 1e9
+    l2bw = l2["GB/s"] * 1e9
+    t_roof = {
+        "compress": work["compress_bytes"] / bw,
+        "scores": max(work["score_flops"] / tens, work["score_exps"] / sfu, work["score_bytes"] / bw),
+        "topk": work["topk_bytes"] / bw,
+        "sparse": max(work["sparse_flops"] / tens, work["sparse_exps"] / sfu, work["sparse_gather_bytes"] / l2bw),
+    }
+    step_roof = {"roofline_ms": {k: v * 1e3 for k, v in t_roof.items()},
+                 "measured_ms": dict(per_kernel),
+                 "frac": sum(t_roof.values()) * 1e3 / ms_per_step,
+                 "peaks": {"tensor_TFLOP/s": tflops_sus, "sfu_Gexp/s": sfu / 1e9, "hbm_GB/s": hbm,
+                           "l2_gather_GB/s": l2["GB/s"], "sm_mhz": sm_mhz}}
 
     kern_detail = {}
     for nm in kernels:
@@ -451,6 +516,8 @@ def main():
         "gpu_launches": (len(kernels) + 1) * args.steps,   # the sparse call is two launches (local + top-k)
         "kernels": kern_detail,
         "roofline": roof,
+        "step_roofline": step_roof,
+        "l2_gather_probe": l2,
         "clocks": clk,
         "device_status": status,
     }

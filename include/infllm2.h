@@ -263,6 +263,18 @@ int infllm2_decode_step(const infllm2_decode_state* st, const void* q, const voi
                         void* out, void* workspace, size_t workspace_bytes, const infllm2_params* p,
                         void* stream);
 
+/* Measurement: L2 -> SM gather bandwidth with the block-sparse attention's
+ * access pattern: the roofline denominator of the gather-bound attention
+ * kernel.  K, V: [rows, h_kv, 128] bf16 device tensors (any contents).
+ * One CTA per SM; `producers` (1, 2, 3 or 6) warps each gather `tiles`
+ * tiles of two random 64-key blocks (32 KB) of kv group 0 from the first
+ * nblk blocks, with 192 KB in flight per SM, and discard them.  The caller
+ * times the call (bytes = num_SMs * producers * tiles * 32768).  Returns
+ * INFLLM2_ERR_INVALID_ARG for null or misaligned tensors, nblk * 64 > rows
+ * or tiles < 1. */
+int infllm2_probe_l2_gather(const void* K, const void* V, int64_t rows, int32_t h_kv, int32_t nblk,
+                            int32_t tiles, int32_t producers, void* stream);
+
 /* Device status word (per device).  Returns INFLLM2_OK or the first
  * INFLLM2_ERR_DEVICE_* recorded by a kernel since the last clear.
  * Synchronises the device. */

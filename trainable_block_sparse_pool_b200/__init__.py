@@ -23,6 +23,7 @@ __all__ = [
     "infllm2_select_workspace_bytes", "infllm2_scores_ld", "infllm2_sparse_workspace_bytes", "infllm2_sparse_attn",
     "infllm2_dense_attn",
     "infllm2_get_device_status", "infllm2_clear_device_status", "infllm2_debug_wait_timeout",
+    "infllm2_probe_l2_gather",
     "DecodeState", "make_decode_state", "infllm2_decode_workspace_bytes", "infllm2_decode_build_caches",
     "infllm2_decode_step", "OUT_BF16", "OUT_F32",
 ]
@@ -96,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "infllm2_get_device_status": (ctypes.c_int, []),
         "infllm2_clear_device_status": (ctypes.c_int, []),
         "infllm2_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
+        "infllm2_probe_l2_gather": (ctypes.c_int, [_P, _P, i64, i32, i32, i32, i32, _P]),
         "infllm2_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(DecodeState), pp]),
         "infllm2_decode_build_caches": (ctypes.c_int, [ctypes.POINTER(DecodeState), pp, _P]),
         "infllm2_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P, ctypes.c_size_t, pp,
@@ -220,6 +222,14 @@ def infllm2_sparse_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block
                                    _ptr(out), od, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    ctypes.byref(params or default_params()), _stream(stream))
     _check("infllm2_sparse_attn", rc)
+
+
+def infllm2_probe_l2_gather(K: torch.Tensor, V: torch.Tensor, nblk: int, tiles: int, producers: int,
+                            stream=None) -> None:
+    """L2 gather bandwidth probe with the sparse attention's tile shape (K, V: [rows, h_kv, 128] bf16)."""
+    rc = lib().infllm2_probe_l2_gather(_ptr(K), _ptr(V), K.shape[0], K.shape[1], nblk, tiles, producers,
+                                       _stream(stream))
+    _check("infllm2_probe_l2_gather", rc)
 
 
 def infllm2_dense_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, vl: Varlen, out: torch.Tensor,

@@ -17,21 +17,24 @@
 // (dense: blocks 2i, 2i+1; LOCAL: consecutive blocks of the CTA's init and
 // local range).  Per 128-key tile:
 //   S[128 rows, 128 keys] = Q . K^T        tcgen05, A = Q (smem), B = K (smem)
-//   softmax, one thread per row (two passes over the TMEM row: max, then
-//   exp2 + bf16 P written to shared memory in the 128-byte-swizzled K-major
-//   layout the next MMA reads)
+//   softmax, two threads per row (warps w and w + 4 share TMEM lane
+//   quadrant w % 4; each owns 64 of the tile's score columns): one TMEM
+//   read of its 64 scores, the row maximum exchanged with the partner
+//   through shared memory at the pair's barrier, exp2 + bf16 P written to
+//   shared memory in the 128-byte-swizzled K-major layout the next MMA reads
 //   O_tile[128 rows, d] = P . V            A = P (smem), B = V (MN-major)
-// O_tile lands in a fresh TMEM accumulator and is folded into registers
-// (O = O * alpha + O_tile) by the row's thread.
+// O_tile lands in a fresh TMEM accumulator and each thread folds its d/2
+// columns into registers (O = O * alpha + O_tile).
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer / TMEM owner,
-// warps 2-5 softmax + correction.
+// warps 2-9 softmax + correction.
 #include "sm100.cuh"
 
 namespace infllm2 {
 
 namespace dense {
 
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;                // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kSoftWarps;
 constexpr int kKeys = 128;
 constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -45,7 +48,8 @@ struct Cfg {
   static constexpr uint32_t kKBytes = kChunk * KCH;
   static constexpr uint32_t kStageBytes = 2 * kKBytes;
   static constexpr uint32_t kPBytes = 128 * 128 * 2;         // 128 rows x 128 keys bf16, 2 chunks
-  static constexpr uint32_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + 512;
+  static constexpr uint32_t kRed = 3 * 128 * 2 * 4;            // row-max exchange (two slots), row-sum exchange
+  static constexpr uint32_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + kRed + 512;
   static constexpr uint32_t kOCol = 256;                     // O buffers after the two S buffers
 };
 
@@ -99,7 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + C::kQBytes;
   uint8_t* sP = sKV + kStages * C::kStageBytes;
-  Bars* bars = reinterpret_cast<Bars*>(sP + C::kPBytes);
+  float* xch = reinterpret_cast<float*>(sP + C::kPBytes);   // [slot][row][half]: maxima (slots 0, 1), sums (2)
+  Bars* bars = reinterpret_cast<Bars*>(xch + 3 * 128 * 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.y, g = blockIdx.z;
@@ -124,11 +129,11 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
     for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_empty[i], 4);
+      mbar_init(&bars->s_empty[i], kSoftWarps);
       mbar_init(&bars->o_full[i], 1);
-      mbar_init(&bars->o_empty[i], 4);
+      mbar_init(&bars->o_empty[i], kSoftWarps);
     }
-    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->p_full, kSoftWarps);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_barrier_init();
@@ -213,66 +218,67 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       mbar_wait(&bars->mma_done, 0);
     }
   } else {
-    const int wq = warp & 3;
+    const int wq = warp & 3;                      // TMEM lane quadrant
+    const int hf = (warp - 2) >> 2;               // which half of the columns
     const int r = wq * 32 + lane;                 // query row (t_loc, h)
     const int t = t0 + r / G;
     const int h = r % G;
+    const int pair = 1 + wq;                      // named barrier of the two warps of this quadrant
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    constexpr int DH = D / 2;                     // output columns of this thread
     const float c = scale * kLog2e;
-    float o_acc[D];
+    float o_acc[DH];
 #pragma unroll
-    for (int j = 0; j < D; ++j) o_acc[j] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;
-    // swizzled P row: 16-byte unit q of 128-byte row r sits at unit q ^ (r & 7)
-    uint8_t* prow = sP + (r >> 3) * 1024 + (r & 7) * 128;
+    for (int j = 0; j < DH; ++j) o_acc[j] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;         // l_run: this thread's 64 columns only
+    // swizzled P row: 16-byte unit q of 128-byte row r sits at unit q ^ (r & 7);
+    // this thread's 64 keys are P chunk hf
+    uint8_t* prow = sP + hf * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
     for (int it = 0; it < nkt; ++it) {
       const int sb = it & 1;
-      if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (it >> 1) & 1));
+      if (!got) set_abort(bars);
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_addr + sb * kKeys;
-      // keys of this tile: half e is block walk.block(2 it + e); key i of a
-      // 16-key group at cc is token ubase[e] + (cc & 63) + i (visible when
-      // <= t); a block the row does not share is masked whole
-      int ub0, ub1;
+      // the tile's keys: half e is block walk.block(2 it + e), this thread's
+      // is e = hf; key i of it is token ub + i (visible when <= t); a block
+      // the row does not share is masked whole
+      int ub;
       {
-        const int blk0 = walk.block(2 * it), blk1 = walk.block(2 * it + 1);
-        ub0 = (blk0 >= 0 && (!LOCAL || in_set(blk0, t, n_init, n_local))) ? 64 * blk0 : INT_MAX / 2;
-        ub1 = (blk1 >= 0 && (!LOCAL || in_set(blk1, t, n_init, n_local))) ? 64 * blk1 : INT_MAX / 2;
+        const int blk = walk.block(2 * it + hf);
+        ub = (blk >= 0 && (!LOCAL || in_set(blk, t, n_init, n_local))) ? 64 * blk : INT_MAX / 2;
       }
+      float v[64];
+      if (got) tmem_load64(tmem + lane_addr + sb * kKeys + hf * 64, v);
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < kKeys; cc += 16) {
-        float v[16];
-        tmem_load16(s_addr + cc, v);
-        const int u0 = ((cc >> 6) ? ub1 : ub0) + (cc & 63);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) if (u0 + i <= t) mx = fmaxf(mx, v[i] * c);
+      for (int i = 0; i < 64; ++i) {
+        v[i] = (ub + i <= t) ? v[i] * c : -INFINITY;
+        mx = fmaxf(mx, v[i]);
       }
-      const float m_new = fmaxf(m_run, mx);
+      float* slot = xch + sb * 256;
+      slot[r * 2 + hf] = mx;
+      // one barrier per tile for the pair: the partner's maximum, and a
+      // stop decision both warps take alike
+      if (bar_red_or(pair, 64, !got || aborted(bars))) { set_abort(bars); ok = false; break; }
+      const float m_new = fmaxf(m_run, fmaxf(mx, slot[r * 2 + (hf ^ 1)]));
       const bool none = (m_new == -INFINITY);
       const float alpha = none ? 1.f : ex2(m_run - m_new);
       float lsum = 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < kKeys; cc += 16) {
-        float v[16];
-        tmem_load16(s_addr + cc, v);
-        const int u0 = ((cc >> 6) ? ub1 : ub0) + (cc & 63);
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 16) {
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const float p0 = (!none && u0 + i <= t) ? ex2(fmaf(v[i], c, -m_new)) : 0.f;
-          const float p1 = (!none && u0 + i + 1 <= t) ? ex2(fmaf(v[i + 1], c, -m_new)) : 0.f;
+          const float p0 = none ? 0.f : ex2(v[cc + i] - m_new);
+          const float p1 = none ? 0.f : ex2(v[cc + i + 1] - m_new);
           lsum += p0 + p1;
           __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
           pk[i >> 1] = *reinterpret_cast<uint32_t*>(&b2);
         }
-        // keys cc .. cc+15 of this tile: chunk cc/64, 16-byte units (cc%64)/8 and +1
-        const int chunk = cc >> 6;
-        const int q0 = (cc & 63) >> 3;
-        uint8_t* base = prow + chunk * 16384;
-        *reinterpret_cast<uint4*>(base + ((q0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(base + (((q0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        const int q0 = cc >> 3;                   // 16-byte units q0, q0 + 1 of the 128-byte row
+        *reinterpret_cast<uint4*>(prow + ((q0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(prow + (((q0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
       l_run = l_run * alpha + lsum;
       m_run = m_new;
@@ -280,32 +286,39 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) { mbar_arrive(&bars->p_full); mbar_arrive(&bars->s_empty[sb]); }
-      // fold this tile's P.V into the registers
+      // fold this tile's P.V (this thread's d/2 columns) into the registers
       const int pb = it & 1;
-      if (!mbar_wait(&bars->o_full[pb], (it >> 1) & 1)) { set_abort(bars); ok = false; break; }
+      const bool gotO = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[pb], (it >> 1) & 1));
+      if (!gotO) { set_abort(bars); ok = false; }
       tc_fence_after();
+      if (gotO) {
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 16) {
-        float v[16];
-        tmem_load16(tmem + lane_addr + C::kOCol + pb * D + cc, v);
+        for (int cc = 0; cc < DH; cc += 16) {
+          float w[16];
+          tmem_load16(tmem + lane_addr + C::kOCol + pb * D + hf * DH + cc, w);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) o_acc[cc + i] = fmaf(o_acc[cc + i], alpha, v[i]);
+          for (int i = 0; i < 16; ++i) o_acc[cc + i] = fmaf(o_acc[cc + i], alpha, w[i]);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->o_empty[pb]);
     }
+    // the row sum over both halves (both warps of the pair get here alike)
+    xch[512 + r * 2 + hf] = l_run;
+    bar_red_or(pair, 64, false);
+    const float l_row = l_run + xch[512 + r * 2 + (hf ^ 1)];
     if (ok && t < len) {
-      const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      const int64_t base = (static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h) * D;
+      const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
+      const int64_t base = (static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h) * D + hf * DH;
       float w_own = inv;   // weight of o_acc; the top-k partial (if any) gets w_top
       float w_top = 0.f;
       if (LOCAL) {
         // out[row] holds the top-k partial (normalised) when its log-sum-exp
         // lb (log2 units) is finite; la is this partial's
         const float lb = lse[static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h];
-        if (lb != -INFINITY && l_run > 0.f) {
-          const float la = m_run + log2f(l_run);
+        if (lb != -INFINITY && l_row > 0.f) {
+          const float la = m_run + log2f(l_row);
           const float mm = fmaxf(la, lb);
           const float wa = ex2(la - mm), wb = ex2(lb - mm);
           const float iw = 1.f / (wa + wb);
@@ -316,19 +329,19 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       if (OUT_F32) {
         float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + base);
 #pragma unroll
-        for (int j = 0; j < D; j += 4) {
-          float4 v = make_float4(o_acc[j] * w_own, o_acc[j + 1] * w_own, o_acc[j + 2] * w_own, o_acc[j + 3] * w_own);
+        for (int j = 0; j < DH; j += 4) {
+          float4 v4 = make_float4(o_acc[j] * w_own, o_acc[j + 1] * w_own, o_acc[j + 2] * w_own, o_acc[j + 3] * w_own);
           if (LOCAL && w_top != 0.f) {
             const float4 b4 = o4[j / 4];
-            v.x = fmaf(b4.x, w_top, v.x); v.y = fmaf(b4.y, w_top, v.y);
-            v.z = fmaf(b4.z, w_top, v.z); v.w = fmaf(b4.w, w_top, v.w);
+            v4.x = fmaf(b4.x, w_top, v4.x); v4.y = fmaf(b4.y, w_top, v4.y);
+            v4.z = fmaf(b4.z, w_top, v4.z); v4.w = fmaf(b4.w, w_top, v4.w);
           }
-          o4[j / 4] = v;
+          o4[j / 4] = v4;
         }
       } else {
         uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + base);
 #pragma unroll
-        for (int j = 0; j < D; j += 8) {
+        for (int j = 0; j < DH; j += 8) {
           float top[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) top[q] = 0.f;

@@ -20,6 +20,7 @@
 #include "sparse_attn.cu"
 #include "dense_attn.cu"
 #include "decode.cu"
+#include "probe.cu"
 
 namespace infllm2 {
 
@@ -312,6 +313,19 @@ int infllm2_clear_device_status(void) {
   cudaError_t e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaDeviceSynchronize();
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_probe_l2_gather(const void* K, const void* V, int64_t rows, int32_t h_kv, int32_t nblk,
+                            int32_t tiles, int32_t producers, void* stream) {
+  if (!K || !V || !aligned16(K) || !aligned16(V) || rows < 64 || h_kv < 1 || nblk < 1 ||
+      static_cast<int64_t>(nblk) * 64 > rows || tiles < 1)
+    return INFLLM2_ERR_INVALID_ARG;
+  if (producers != 1 && producers != 2 && producers != 3 && producers != 6) return INFLLM2_ERR_UNSUPPORTED;
+  bool map_fail = false;
+  cudaError_t e = launch_l2_gather_probe(K, V, rows, h_kv, nblk, tiles, producers, static_cast<cudaStream_t>(stream),
+                                         &map_fail);
+  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
 

@@ -86,22 +86,6 @@ __device__ __forceinline__ void set_abort(Bars* b) {
   *reinterpret_cast<volatile int*>(&b->abort) = 1;
 }
 
-// Barrier over `nthreads` threads on named barrier `id` that also ORs a
-// predicate across them; every participant gets the same result.
-__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pin, pout;\n\t"
-      "setp.ne.u32 pin, %1, 0;\n\t"
-      "bar.red.or.pred pout, %2, %3, pin;\n\t"
-      "selp.u32 %0, 1, 0, pout;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
-
 // Number of valid (>= 0) entries of a block list, with independent vector
 // loads (lists hold their valid entries first, then -1 padding).
 __device__ __forceinline__ int count_valid(const int32_t* I, int n_sel) {
