@@ -20,11 +20,13 @@
 //   softmax, two threads per row (warps w and w + 4 share TMEM lane
 //   quadrant w % 4; each owns 64 of the tile's score columns): one TMEM
 //   read of its 64 scores, the row maximum exchanged with the partner
-//   through shared memory at the pair's barrier, exp2 + bf16 P written to
-//   shared memory in the 128-byte-swizzled K-major layout the next MMA reads
-//   O_tile[128 rows, d] = P . V            A = P (smem), B = V (MN-major)
-// O_tile lands in a fresh TMEM accumulator and each thread folds its d/2
-// columns into registers (O = O * alpha + O_tile).
+//   through shared memory at the pair's barrier, exp2, and bf16 P written
+//   back to TMEM over the tile's own score columns (key k in column k/2)
+//   O_tile[128 rows, d] = P . V            A = P (TMEM), B = V (smem, MN-major)
+// O_tile lands in a fresh TMEM accumulator; each thread folds its d/2
+// columns into registers (O = O * alpha + O_tile) one tile later, after it
+// has written the next tile's P, so the softmax never waits for the P.V of
+// the tile it has just produced.
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer / TMEM owner,
 // warps 2-9 softmax + correction.
 #include "sm100.cuh"
@@ -47,9 +49,8 @@ struct Cfg {
   static constexpr uint32_t kChunk = kKeys * 128;            // 16 KB
   static constexpr uint32_t kKBytes = kChunk * KCH;
   static constexpr uint32_t kStageBytes = 2 * kKBytes;
-  static constexpr uint32_t kPBytes = 128 * 128 * 2;         // 128 rows x 128 keys bf16, 2 chunks
   static constexpr uint32_t kRed = 3 * 128 * 2 * 4;            // row-max exchange (two slots), row-sum exchange
-  static constexpr uint32_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kPBytes + kRed + 512;
+  static constexpr uint32_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kRed + 512;
   static constexpr uint32_t kOCol = 256;                     // O buffers after the two S buffers
 };
 
@@ -102,8 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + C::kQBytes;
-  uint8_t* sP = sKV + kStages * C::kStageBytes;
-  float* xch = reinterpret_cast<float*>(sP + C::kPBytes);   // [slot][row][half]: maxima (slots 0, 1), sums (2)
+  float* xch = reinterpret_cast<float*>(sKV + kStages * C::kStageBytes);   // [slot][row][half]: maxima (slots 0, 1), sums (2)
   Bars* bars = reinterpret_cast<Bars*>(xch + 3 * 128 * 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,7 +174,6 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       const uint32_t idS = idesc_bf16_f32(128, kKeys, 0, 0);
       const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_base = smem_u32(sQ);
-      const uint32_t p_base = smem_u32(sP);
       bool ok = mbar_wait(&bars->q_full, 0);
       if (!ok) set_abort(bars);
       auto issue_pv = [&](int j) -> bool {
@@ -184,11 +183,11 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
         if (!mbar_wait(&bars->o_empty[pb], ((j >> 1) & 1) ^ 1)) return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(sKV + st * C::kStageBytes + C::kKBytes);
+        const uint32_t p_tmem = tmem + (j & 1) * kKeys;     // P(j) over S(j)'s columns: keys 16k.. in column 8k..
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k) {
-          const uint64_t a = make_sdesc(p_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kLayoutSW128);
           const uint64_t b = make_sdesc(v_base + k * 2048, C::kChunk, 1024, kLayoutSW128);
-          umma_bf16(tmem + C::kOCol + pb * D, a, b, idO, k > 0);
+          umma_bf16_ts(tmem + C::kOCol + pb * D, p_tmem + k * 8, b, idO, k > 0);
         }
         umma_commit(&bars->kv_empty[st]);
         umma_commit(&bars->o_full[pb]);
@@ -231,10 +230,28 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
 #pragma unroll
     for (int j = 0; j < DH; ++j) o_acc[j] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;         // l_run: this thread's 64 columns only
-    // swizzled P row: 16-byte unit q of 128-byte row r sits at unit q ^ (r & 7);
-    // this thread's 64 keys are P chunk hf
-    uint8_t* prow = sP + hf * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+    float alpha_prev = 1.f;                       // rescale of o_acc that goes with the pending fold
     bool ok = true;
+    // o_acc = o_acc * alpha + (P.V of tile j): this thread's d/2 columns
+    auto fold = [&](int j, float alpha) {
+      const int pb = j & 1;
+      const bool gotO = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[pb], (j >> 1) & 1));
+      if (!gotO) { set_abort(bars); ok = false; }
+      tc_fence_after();
+      if (gotO) {
+#pragma unroll
+        for (int cc = 0; cc < DH; cc += 16) {
+          float w[16];
+          tmem_load16(tmem + lane_addr + C::kOCol + pb * D + hf * DH + cc, w);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o_acc[cc + i] = fmaf(o_acc[cc + i], alpha, w[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_empty[pb]);
+    };
+    int done = 0;                                 // tiles whose P has been handed to the MMA warp
     for (int it = 0; it < nkt; ++it) {
       const int sb = it & 1;
       const bool got = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (it >> 1) & 1));
@@ -259,51 +276,35 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       float* slot = xch + sb * 256;
       slot[r * 2 + hf] = mx;
       // one barrier per tile for the pair: the partner's maximum, and a
-      // stop decision both warps take alike
+      // stop decision both warps take alike; both have read their scores
+      // before it, so P may overwrite them after it
       if (bar_red_or(pair, 64, !got || aborted(bars))) { set_abort(bars); ok = false; break; }
       const float m_new = fmaxf(m_run, fmaxf(mx, slot[r * 2 + (hf ^ 1)]));
       const bool none = (m_new == -INFINITY);
       const float alpha = none ? 1.f : ex2(m_run - m_new);
+      // P (bf16 pairs) into TMEM columns sb * 128 + hf * 32 .. + 31: key k of the tile in column k / 2
       float lsum = 0.f;
+      uint32_t pk[32];
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 16) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          const float p0 = none ? 0.f : ex2(v[cc + i] - m_new);
-          const float p1 = none ? 0.f : ex2(v[cc + i + 1] - m_new);
-          lsum += p0 + p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          pk[i >> 1] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        const int q0 = cc >> 3;                   // 16-byte units q0, q0 + 1 of the 128-byte row
-        *reinterpret_cast<uint4*>(prow + ((q0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(prow + (((q0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = none ? 0.f : ex2(v[2 * i] - m_new);
+        const float p1 = none ? 0.f : ex2(v[2 * i + 1] - m_new);
+        lsum += p0 + p1;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        pk[i] = *reinterpret_cast<uint32_t*>(&b2);
       }
+      tmem_store32u(tmem + lane_addr + sb * kKeys + hf * 32, pk);
       l_run = l_run * alpha + lsum;
       m_run = m_new;
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) { mbar_arrive(&bars->p_full); mbar_arrive(&bars->s_empty[sb]); }
-      // fold this tile's P.V (this thread's d/2 columns) into the registers
-      const int pb = it & 1;
-      const bool gotO = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[pb], (it >> 1) & 1));
-      if (!gotO) { set_abort(bars); ok = false; }
-      tc_fence_after();
-      if (gotO) {
-#pragma unroll
-        for (int cc = 0; cc < DH; cc += 16) {
-          float w[16];
-          tmem_load16(tmem + lane_addr + C::kOCol + pb * D + hf * DH + cc, w);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o_acc[cc + i] = fmaf(o_acc[cc + i], alpha, w[i]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->o_empty[pb]);
+      done = it + 1;
+      // the previous tile's P.V has had this tile's softmax to finish
+      if (it > 0) fold(it - 1, alpha_prev);
+      alpha_prev = alpha;
     }
+    if (ok && done > 0) fold(done - 1, alpha_prev);
     // the row sum over both halves (both warps of the pair get here alike)
     xch[512 + r * 2 + hf] = l_run;
     bar_red_or(pair, 64, false);

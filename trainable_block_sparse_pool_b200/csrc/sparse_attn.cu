@@ -53,13 +53,15 @@ struct Cfg {
   static constexpr uint32_t kChunk = kPairKeys * 128;         // 16 KB: 128 keys x 64 dims
   static constexpr uint32_t kHalf = 64 * 128;                 // one block inside a chunk
   static constexpr uint32_t kKBytes = kChunk * KCH;
-  static constexpr uint32_t kStageBytes = 2 * kKBytes;        // one K slot plus one V slot
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  // ring depths (measured at 128K: 3 + 3 beats 2 + 4 and 4 + 2)
+  static constexpr int kKStages = (D == 128) ? 3 : 6;
+  static constexpr int kVStages = (D == 128) ? 3 : 6;
+  static constexpr int kStages = kKStages + kVStages;           // K and V slots in all
   static constexpr uint32_t kQBuf = 2048 * KCH;               // 16 head rows x d
   static constexpr uint32_t kPBuf = kPairKeys * 16 * 2;       // 4 KB
   static constexpr uint32_t kRed = kNumWG * 4 * 16 * 4;       // per-warp partial maxima / sums
   static constexpr uint32_t kSmem =
-      1024 + kStages * kStageBytes + kNumWG * 2 * kQBuf + kNumWG * 2 * kPBuf + kRed + 512;
+      1024 + kStages * kKBytes + kNumWG * 2 * kQBuf + kNumWG * 2 * kPBuf + kRed + 512;
 };
 
 struct Bars {
@@ -181,9 +183,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem;
-  uint8_t* sKr = sKV;                                                  // K ring [kStages][kKBytes]
-  uint8_t* sVr = sKV + C::kStages * C::kKBytes;                        // V ring [kStages][kKBytes]
-  uint8_t* sQ = sKV + C::kStages * C::kStageBytes;                    // [wg][2]
+  uint8_t* sKr = sKV;                                                  // K ring [kKStages][kKBytes]
+  uint8_t* sVr = sKV + C::kKStages * C::kKBytes;                       // V ring [kVStages][kKBytes]
+  uint8_t* sQ = sKV + C::kStages * C::kKBytes;                        // [wg][2]
   uint8_t* sP = sQ + kNumWG * 2 * C::kQBuf;                           // [wg][2]
   float* red = reinterpret_cast<float*>(sP + kNumWG * 2 * C::kPBuf);  // [wg][4][16]
   Bars* bars = reinterpret_cast<Bars*>(red + kNumWG * 4 * 16);
@@ -197,9 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);   // head rows past G stay zero
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
+    for (int i = 0; i < C::kKStages; ++i) {
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < C::kVStages; ++i) {
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
     }
@@ -230,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     // same stream of tiles.  The whole warp walks the units (their block
     // lists live in its registers); lane 0 waits and issues the copies.
     const bool isV = (warp == kVWarp);
+    const int nst = isV ? C::kVStages : C::kKStages;
     const CUtensorMap* tm = isV ? &tmV : &tmK;
     uint8_t* ring = isV ? sVr : sKr;
     uint64_t* full = isV ? bars->v_full : bars->k_full;
@@ -273,10 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
           const int b0 = warp_list_get(Le[w], x[w].I, x[w].nvalid, x[w].nlist, j, 0);
           int b1 = warp_list_get(Lo[w], x[w].I, x[w].nvalid, x[w].nlist, j, 1);
           if (b1 < 0) b1 = b0;   // odd count: reload the first block, masked by the softmax
-          const int st = it % C::kStages;
+          const int st = it % nst;
           int good = 1;
           if (lane == 0) {
-            good = mbar_wait(&empty[st], ((it / C::kStages) & 1) ^ 1) && !aborted(bars);
+            good = mbar_wait(&empty[st], ((it / nst) & 1) ^ 1) && !aborted(bars);
             if (good) {
               uint8_t* dst = ring + st * C::kKBytes;
               mbar_arrive_expect_tx(&full[st], C::kKBytes);
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     }
     // wait for every copy still in flight before the CTA may exit
     if (lane == 0) {
-      for (int i = max(0, it - C::kStages); i < it; ++i) mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
+      for (int i = max(0, it - nst); i < it; ++i) mbar_wait(&full[i % nst], (i / nst) & 1);
       if (!isV)
         for (int w = 0; w < kNumWG; ++w)
           for (int i = max(0, ucnt[w] - 2); i < ucnt[w]; ++i) mbar_wait(&bars->q_full[w][i & 1], (i >> 1) & 1);
@@ -326,9 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         for (int j = 0; ok && j < nmax; ++j) {
           for (int w = 0; w < kNumWG; ++w) {
             if (j >= nt[w]) continue;
-            const int st = it % C::kStages;
+            const int st = it % C::kKStages;
             const int sb = tcnt[w] & 1;
-            if (!mbar_wait(&bars->k_full[st], (it / C::kStages) & 1) ||
+            if (!mbar_wait(&bars->k_full[st], (it / C::kKStages) & 1) ||
                 !mbar_wait(&bars->s_empty[w][sb], ((tcnt[w] >> 1) & 1) ^ 1) || aborted(bars)) {
               set_abort(bars); ok = false; break;
             }
@@ -380,10 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
           for (int w = 0; w < kNumWG; ++w) {
             if (j >= nt[w]) continue;
             if (w == pw) {
-              const int st = it % C::kStages;
+              const int st = it % C::kVStages;
               const int pb = tcnt & 1;
               if (!mbar_wait(&bars->p_full[pw][pb], (tcnt >> 1) & 1) ||
-                  !mbar_wait(&bars->v_full[st], (it / C::kStages) & 1) || aborted(bars)) {
+                  !mbar_wait(&bars->v_full[st], (it / C::kVStages) & 1) || aborted(bars)) {
                 set_abort(bars); ok = false; break;
               }
               tc_fence_after();
