@@ -239,7 +239,7 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V,
  * infllm2_decode_workspace_bytes (device, caller-owned, no alignment beyond
  * 16 bytes, contents need no initialisation and carry nothing from one step
  * to the next; one workspace must not serve two steps in flight at once).
- * Capacities above 2.6M tokens (more than 40960 candidate blocks) are
+ * Capacities above 1441792 tokens (more than 22528 candidate blocks) are
  * INFLLM2_ERR_UNSUPPORTED, and infllm2_decode_workspace_bytes returns 0 for
  * them.  infllm2_decode_build_caches pools the seq_len[b] tokens already in
  * the cache into k_c1 / k_c2 (for a prefix written by the caller).

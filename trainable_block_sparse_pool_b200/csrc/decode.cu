@@ -103,6 +103,26 @@ __device__ __forceinline__ void scores_16x8_reg(float (&c)[4], const QFrag<D>& f
   }
 }
 
+// ---------------------------------------------------------------- cp.async staging
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(full ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
 // ---------------------------------------------------------------- pooling of the window that ends at t
 // Window [t - len + 1, t] of kv group g: rows before t from the cache, row t
 // from k_new (it may not be in the cache yet).  Exact mean in fp64, one bf16
@@ -424,14 +444,28 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
 // window of halo, so a block never straddles CTAs).  Per window: the 16
 // heads' scores, normalised by their LSE and summed over the group
 // ([top168] §三 second stage, §四); per block: the max over its 5 windows.
-// The last CTA of (b, g) to finish runs the selection.
+// The CTA's pooled keys are staged with cp.async into shared memory
+// (16-byte pieces of a row XOR-swizzled by the row's parity, so the
+// fragment loads are free of bank conflicts), which keeps registers low
+// enough for three CTAs per SM; the LSE partials and the query rows load
+// meanwhile.  The last CTA of (b, g) to finish runs the selection.
+constexpr int kScoreRows = kScoreWin / 8 * 8 + 8;   // 33 n-tiles of 8 windows; 257 used
+
 template <int D>
-__global__ void __launch_bounds__(kSelThreads) score_select_kernel(
+struct ScoreCfg {
+  static constexpr int CH = D / 8;                                 // 16-byte pieces per row
+  static constexpr uint32_t kBuf = kScoreRows * D * 2;             // the CTA's rows
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
     const float2* __restrict__ part2, int nsplit2, int capacity, int h_q, int h_kv, int cap_c1, int nblk_cap,
     int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel, float* __restrict__ bscore,
     int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
-  extern __shared__ uint32_t sel_keys[];       // [cand_cap], used by the selecting CTA
+  using C = ScoreCfg<D>;
+  extern __shared__ __align__(128) uint8_t sc_smem[];            // [kBuf] rows; the selection's keys reuse it
+  uint32_t* sel_keys = reinterpret_cast<uint32_t*>(sc_smem);
   __shared__ float nlse[16];
   __shared__ float2 lsep[16][17];
   __shared__ float sw[kScoreWin + 8];
@@ -440,7 +474,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
   const int bg = blockIdx.x, c = blockIdx.y;
   const int b = bg / h_kv, g = bg % h_kv;
   const int G = h_q / h_kv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int t = seq_len[b];
   if (t < 0 || t >= capacity) return;          // recorded by the append kernel
@@ -451,23 +485,25 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
   if (c == 0 || j0 + 1 < n1) {                 // this CTA has visible windows
     const float cs = scale * kLog2e;
     const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
-    // this warp's n-tiles are nt = warp + 8 i (i < 5): issue every load first
-    constexpr int kMaxNt = (kScoreWin / 8 + 1 + 7) / 8;
-    uint4 kv[kMaxNt][D / 32];
-#pragma unroll
-    for (int i = 0; i < kMaxNt; ++i) {
-      const int nt = warp + 8 * i;
-      const int wr = j0 + nt * 8 + gid;
-      const bool ok = (nt * 8 < kScoreWin + 1) && wr >= 0 && wr < n1;
-      load_krow<D>(kv[i], ok ? base + static_cast<int64_t>(wr) * D : nullptr, lane);
+    // stage windows j0 .. j0 + 263 (rows past the visible windows zero-filled)
+    {
+      const uint32_t dst0 = smem_u32(sc_smem);
+      for (int pc = tid; pc < kScoreRows * C::CH; pc += kSelThreads) {
+        const int r = pc / C::CH, piece = pc - r * C::CH;
+        const int wr = j0 + r;
+        const bool ok = r < kScoreWin + 1 && wr >= 0 && wr < n1;
+        const __nv_bfloat16* src = base + (ok ? static_cast<int64_t>(wr) * D + piece * 8 : 0);
+        cp_async16(dst0 + r * (D * 2) + ((piece ^ ((r & 1) << 2)) << 4), src, ok);
+      }
+      cp_async_commit();
     }
     // per-head LSE: thread (h, k0) folds the coarse partials k0, k0 + 16, ...
     {
-      const int h = threadIdx.x & 15, k0 = threadIdx.x >> 4;
+      const int h = tid & 15, k0 = tid >> 4;
       float mm = -INFINITY, ll = 0.f;
       if (h < G && n2 > 0) {
-        for (int k = k0; k < nsplit2; k += 16) {
-          const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + k) * 16 + h];
+        for (int kk = k0; kk < nsplit2; kk += 16) {
+          const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + kk) * 16 + h];
           const float mn = fmaxf(mm, v.x);
           if (mn != -INFINITY) {
             ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
@@ -478,13 +514,13 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
       lsep[h][k0] = make_float2(mm, ll);
     }
     __syncthreads();
-    if (threadIdx.x < 16) {
-      const int h = threadIdx.x;
+    if (tid < 16) {
+      const int h = tid;
       float mm = -INFINITY, ll = 0.f;
       if (h < G) {
         if (n2 > 0) {
-          for (int k = 0; k < 16; ++k) {
-            const float2 v = lsep[h][k];
+          for (int kk = 0; kk < 16; ++kk) {
+            const float2 v = lsep[h][kk];
             const float mn = fmaxf(mm, v.x);
             if (mn != -INFINITY) {
               ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
@@ -508,15 +544,18 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     }
     QFrag<D> f;
     load_qfrag<D>(f, qh, lane, G);
+    cp_async_wait0();
     __syncthreads();
     const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
-#pragma unroll
-    for (int i = 0; i < kMaxNt; ++i) {
-      const int nt = warp + 8 * i;
-      if (nt * 8 >= kScoreWin + 1) break;
+    for (int nt = warp; nt * 8 < kScoreWin + 1; nt += 8) {
       const int w0 = j0 + nt * 8;
+      const int r = nt * 8 + gid;
+      const uint4* rowp = reinterpret_cast<const uint4*>(sc_smem + r * (D * 2));
+      uint4 kv[D / 32];
+#pragma unroll
+      for (int p = 0; p < D / 32; ++p) kv[p] = rowp[(4 * p + tig) ^ ((r & 1) << 2)];
       float sc[4];
-      scores_16x8_reg<D>(sc, f, kv[i]);
+      scores_16x8_reg<D>(sc, f, kv);
       // head-group sum for keys 2tig and 2tig+1: two heads here, the other 14 on the lanes with the same tig
       float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
       float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
@@ -533,13 +572,12 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     }
     __syncthreads();
     // block scores: block blk = 64c + i takes windows 4 blk - 1 .. 4 blk + 3 = sw[4i .. 4i + 4]
-    if (threadIdx.x < kScoreWin / 4) {
-      const int i = threadIdx.x;
-      const int blk = c * (kScoreWin / 4) + i;
+    if (tid < kScoreWin / 4) {
+      const int blk = c * (kScoreWin / 4) + tid;
       if (blk < nblk_cap) {
         float m = -INFINITY;
 #pragma unroll
-        for (int q4 = 0; q4 < 5; ++q4) m = fmaxf(m, sw[4 * i + q4]);
+        for (int q4 = 0; q4 < 5; ++q4) m = fmaxf(m, sw[4 * tid + q4]);
         bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
       }
     }
@@ -547,7 +585,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
   // the last CTA of (b, g) to finish selects the blocks
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&cnt[bg], 1u) == gridDim.y - 1);
+  if (tid == 0) s_last = (atomicAdd(&cnt[bg], 1u) == gridDim.y - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -558,25 +596,6 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
 constexpr int kAttWarps = 4;
 constexpr int kChunkKeys = 32;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool full) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(full ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -999,8 +1018,9 @@ struct DecodePlan {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Largest capacity whose candidate keys fit the selecting CTA's shared memory.
-static bool decode_plan_supported(const DecodePlan& p) { return static_cast<size_t>(p.cand_cap) * 4 <= 160 * 1024; }
+// Largest capacity whose candidate keys fit the selecting CTA's shared memory
+// next to the two staging buffers of the score kernel.
+static bool decode_plan_supported(const DecodePlan& p) { return static_cast<size_t>(p.cand_cap) * 4 <= 88 * 1024; }
 
 DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_sel, int sms) {
   DecodePlan p{};
@@ -1043,11 +1063,11 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
       static_cast<const bf*>(q), static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
       static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache), static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2),
       s->seq_len, s->capacity, s->h_q, s->h_kv, P.cap_c1, P.cap_c2, scale, part2, cnt);
-  const size_t sel_smem = static_cast<size_t>(P.cand_cap) * 4;
+  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kBuf, static_cast<size_t>(P.cand_cap) * 4);
   cudaError_t e = cudaFuncSetAttribute(dec::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sel_smem));
+                                       static_cast<int>(k2_smem));
   if (e != cudaSuccess) return e;
-  dec::score_select_kernel<D><<<dim3(bg, P.nsplit1), dec::kSelThreads, sel_smem, st>>>(
+  dec::score_select_kernel<D><<<dim3(bg, P.nsplit1), dec::kSelThreads, k2_smem, st>>>(
       static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->capacity, s->h_q,
       s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt);
   e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
