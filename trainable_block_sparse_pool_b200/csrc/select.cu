@@ -172,12 +172,35 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
   const float* srow = S + (static_cast<int64_t>(g) * total + row) * ld;
   const int n1 = visible_windows_dev(t, 32, 16);
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = lane; i < ncand; i += 32) {
-    const float sc = fmaxf(block_score(srow, cand_lo + i, n1), 0.f);
-    const uint32_t k = __float_as_uint(sc);
-    keys[i] = k;
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
+  // a candidate ends at least n_local blocks before b_t, so its five
+  // windows 4b-1 .. 4b+3 are all visible: one 16-byte load and one scalar;
+  // eight candidates per lane are loaded before any is used
+  constexpr int kU = 8;
+  for (int i0 = 0; i0 < ncand; i0 += 32 * kU) {
+    float4 v4[kU];
+    float pv[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * 32 + lane;
+      const int b = cand_lo + i;
+      const bool fast = i < ncand && b >= 1 && 4 * b + 3 < n1;
+      v4[u] = fast ? __ldg(reinterpret_cast<const float4*>(srow + 4 * b)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      pv[u] = fast ? __ldg(srow + 4 * b - 1) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * 32 + lane;
+      if (i < ncand) {
+        const int b = cand_lo + i;
+        const float m = (b >= 1 && 4 * b + 3 < n1)
+                            ? fmaxf(fmaxf(pv[u], v4[u].x), fmaxf(fmaxf(v4[u].y, v4[u].z), v4[u].w))
+                            : block_score(srow, b, n1);
+        const uint32_t k = __float_as_uint(fmaxf(m, 0.f));
+        keys[i] = k;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
   }
   warp_select_write(keys, hist, ncand, cand_lo, init_hi, loc_lo, b_t, top_k, n_sel, kmin, kmax, out, lane);
 }
