@@ -27,8 +27,9 @@
 // columns into registers (O = O * alpha + O_tile) one tile later, after it
 // has written the next tile's P, so the softmax never waits for the P.V of
 // the tile it has just produced.
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer / TMEM owner,
-// warps 2-9 softmax + correction.
+// Warp roles: warp 0 loads Q and the K ring, warp 10 the V ring (a K slot is
+// free once its QK product is done, a V slot only once its P.V product is),
+// warp 1 issues the MMAs and owns TMEM, warps 2-9 softmax + correction.
 #include "sm100.cuh"
 
 namespace infllm2 {
@@ -36,9 +37,11 @@ namespace infllm2 {
 namespace dense {
 
 constexpr int kSoftWarps = 8;                // two per TMEM lane quadrant
-constexpr int kThreads = 64 + 32 * kSoftWarps;
+constexpr int kVWarp = 2 + kSoftWarps;        // the V producer
+constexpr int kThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kKeys = 128;
-constexpr int kStages = 2;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D, int G>
@@ -48,16 +51,17 @@ struct Cfg {
   static constexpr uint32_t kQBytes = 128 * 128 * KCH;
   static constexpr uint32_t kChunk = kKeys * 128;            // 16 KB
   static constexpr uint32_t kKBytes = kChunk * KCH;
-  static constexpr uint32_t kStageBytes = 2 * kKBytes;
   static constexpr uint32_t kRed = 3 * 128 * 2 * 4;            // row-max exchange (two slots), row-sum exchange
-  static constexpr uint32_t kSmem = 1024 + kQBytes + kStages * kStageBytes + kRed + 512;
+  static constexpr uint32_t kSmem = 1024 + kQBytes + (kKStages + kVStages) * kKBytes + kRed + 512;
   static constexpr uint32_t kOCol = 256;                     // O buffers after the two S buffers
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t k_full[kKStages];
+  uint64_t k_empty[kKStages];
+  uint64_t v_full[kVStages];
+  uint64_t v_empty[kVStages];
   uint64_t s_full[2];
   uint64_t s_empty[2];
   uint64_t p_full;
@@ -103,7 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + C::kQBytes;
-  float* xch = reinterpret_cast<float*>(sKV + kStages * C::kStageBytes);   // [slot][row][half]: maxima (slots 0, 1), sums (2)
+  uint8_t* sKr = sKV;                                       // K ring [kKStages][kKBytes]
+  uint8_t* sVr = sKV + kKStages * C::kKBytes;               // V ring [kVStages][kKBytes]
+  float* xch = reinterpret_cast<float*>(sKV + (kKStages + kVStages) * C::kKBytes);   // [slot][row][half]: maxima (slots 0, 1), sums (2)
   Bars* bars = reinterpret_cast<Bars*>(xch + 3 * 128 * 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,7 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < kStages; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
+    for (int i = 0; i < kKStages; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1); }
+    for (int i = 0; i < kVStages; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->s_empty[i], kSoftWarps);
@@ -144,30 +151,37 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == kVWarp) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bars->q_full, C::kQBytes);
-      for (int ch = 0; ch < C::KCH; ++ch) tma_load_4d(sQ + ch * 16384, &tmQ, &bars->q_full, ch * 64, 0, g, row0 + t0);
+      const bool isV = (warp == kVWarp);
+      const int nst = isV ? kVStages : kKStages;
+      const CUtensorMap* tm = isV ? &tmV : &tmK;
+      uint8_t* ring = isV ? sVr : sKr;
+      uint64_t* full = isV ? bars->v_full : bars->k_full;
+      uint64_t* empty = isV ? bars->v_empty : bars->k_empty;
+      tma_prefetch_desc(tm);
+      if (!isV) {
+        tma_prefetch_desc(&tmQ);
+        mbar_arrive_expect_tx(&bars->q_full, C::kQBytes);
+        for (int ch = 0; ch < C::KCH; ++ch) tma_load_4d(sQ + ch * 16384, &tmQ, &bars->q_full, ch * 64, 0, g, row0 + t0);
+      }
       int it = 0;
       for (; it < nkt; ++it) {
-        const int st = it % kStages;
-        if (!mbar_wait(&bars->kv_empty[st], ((it / kStages) & 1) ^ 1) || aborted(bars)) { set_abort(bars); break; }
-        uint8_t* dK = sKV + st * C::kStageBytes;
-        uint8_t* dV = dK + C::kKBytes;
+        const int st = it % nst;
+        if (!mbar_wait(&empty[st], ((it / nst) & 1) ^ 1) || aborted(bars)) { set_abort(bars); break; }
+        uint8_t* dst = ring + st * C::kKBytes;
         const int ba = walk.block(2 * it);
         int bb = walk.block(2 * it + 1);
         if (bb < 0) bb = ba;                             // odd count: reload, masked by the softmax
-        mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageBytes);
+        mbar_arrive_expect_tx(&full[st], C::kKBytes);
         for (int ch = 0; ch < C::KCH; ++ch) {
-          tma_load_3d(dK + ch * C::kChunk, &tmK, &bars->kv_full[st], ch * 64, g, row0 + 64 * ba);
-          tma_load_3d(dK + ch * C::kChunk + C::kChunk / 2, &tmK, &bars->kv_full[st], ch * 64, g, row0 + 64 * bb);
-          tma_load_3d(dV + ch * C::kChunk, &tmV, &bars->kv_full[st], ch * 64, g, row0 + 64 * ba);
-          tma_load_3d(dV + ch * C::kChunk + C::kChunk / 2, &tmV, &bars->kv_full[st], ch * 64, g, row0 + 64 * bb);
+          tma_load_3d(dst + ch * C::kChunk, tm, &full[st], ch * 64, g, row0 + 64 * ba);
+          tma_load_3d(dst + ch * C::kChunk + C::kChunk / 2, tm, &full[st], ch * 64, g, row0 + 64 * bb);
         }
       }
-      mbar_wait(&bars->q_full, 0);
-      for (int i = max(0, it - kStages); i < it; ++i) mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1);
+      // wait for every copy still in flight before the CTA may exit
+      if (!isV) mbar_wait(&bars->q_full, 0);
+      for (int i = max(0, it - nst); i < it; ++i) mbar_wait(&full[i % nst], (i / nst) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -178,31 +192,32 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       if (!ok) set_abort(bars);
       auto issue_pv = [&](int j) -> bool {
         const int pb = j & 1;
-        const int st = j % kStages;
+        const int st = j % kVStages;
         if (!mbar_wait(&bars->p_full, j & 1)) return false;
         if (!mbar_wait(&bars->o_empty[pb], ((j >> 1) & 1) ^ 1)) return false;
+        if (!mbar_wait(&bars->v_full[st], (j / kVStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(sKV + st * C::kStageBytes + C::kKBytes);
+        const uint32_t v_base = smem_u32(sVr + st * C::kKBytes);
         const uint32_t p_tmem = tmem + (j & 1) * kKeys;     // P(j) over S(j)'s columns: keys 16k.. in column 8k..
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k) {
           const uint64_t b = make_sdesc(v_base + k * 2048, C::kChunk, 1024, kLayoutSW128);
           umma_bf16_ts(tmem + C::kOCol + pb * D, p_tmem + k * 8, b, idO, k > 0);
         }
-        umma_commit(&bars->kv_empty[st]);
+        umma_commit(&bars->v_empty[st]);
         umma_commit(&bars->o_full[pb]);
         return true;
       };
       int it = 0;
       for (; ok && it < nkt; ++it) {
-        const int st = it % kStages;
+        const int st = it % kKStages;
         const int sb = it & 1;
-        if (!mbar_wait(&bars->kv_full[st], (it / kStages) & 1) ||
+        if (!mbar_wait(&bars->k_full[st], (it / kKStages) & 1) ||
             !mbar_wait(&bars->s_empty[sb], ((it >> 1) & 1) ^ 1) || aborted(bars)) {
           set_abort(bars); ok = false; break;
         }
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sKV + st * C::kStageBytes);
+        const uint32_t k_base = smem_u32(sKr + st * C::kKBytes);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t a = make_sdesc(q_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kLayoutSW128);
@@ -210,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
           umma_bf16(tmem + sb * kKeys, a, b, idS, k > 0);
         }
         umma_commit(&bars->s_full[sb]);
+        umma_commit(&bars->k_empty[st]);                 // the K slot is free once this product is done
         if (it > 0 && !issue_pv(it - 1)) { set_abort(bars); ok = false; break; }
       }
       if (ok && nkt > 0 && !issue_pv(nkt - 1)) set_abort(bars);
@@ -265,14 +281,20 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
         const int blk = walk.block(2 * it + hf);
         ub = (blk >= 0 && (!LOCAL || in_set(blk, t, n_init, n_local))) ? 64 * blk : INT_MAX / 2;
       }
-      float v[64];
+      float v[64];                                // raw scores; the scale c > 0 goes into the exponent
       if (got) tmem_load64(tmem + lane_addr + sb * kKeys + hf * 64, v);
       float mx = -INFINITY;
+      if (__all_sync(0xffffffffu, ub + 63 <= t)) {          // every key of this half visible to every row of the warp
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        v[i] = (ub + i <= t) ? v[i] * c : -INFINITY;
-        mx = fmaxf(mx, v[i]);
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, v[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          v[i] = (ub + i <= t) ? v[i] : -INFINITY;
+          mx = fmaxf(mx, v[i]);
+        }
       }
+      mx *= c;                                    // -inf stays -inf
       float* slot = xch + sb * 256;
       slot[r * 2 + hf] = mx;
       // one barrier per tile for the pair: the partner's maximum, and a
@@ -287,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = none ? 0.f : ex2(v[2 * i] - m_new);
-        const float p1 = none ? 0.f : ex2(v[2 * i + 1] - m_new);
+        const float p0 = none ? 0.f : ex2(fmaf(v[2 * i], c, -m_new));
+        const float p1 = none ? 0.f : ex2(fmaf(v[2 * i + 1], c, -m_new));
         lsum += p0 + p1;
         __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
         pk[i] = *reinterpret_cast<uint32_t*>(&b2);
