@@ -1032,8 +1032,9 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   p.nsplit2 = std::max(1, (p.cap_c2 + dec::kLseWin - 1) / dec::kLseWin);
   p.nsplit1 = std::max(1, (p.cap_c1 + dec::kScoreWin) / dec::kScoreWin);
   const int bg = batch * h_kv;
-  // attention splits: about three attention CTAs per SM
-  const int per_bg = std::min(dec::kMaxSplits, std::max(1, (3 * sms) / std::max(1, bg)));
+  // attention splits: about 1.5 attention CTAs per SM (16 x 131072 decode:
+  // 6 splits of 16 blocks; 3 per SM and 1 per SM were both slower)
+  const int per_bg = std::min(dec::kMaxSplits, std::max(1, (3 * sms) / 2 / std::max(1, bg)));
   p.bps = std::max(1, (n_sel + per_bg - 1) / per_bg);
   p.nsplit = std::max(1, (n_sel + p.bps - 1) / p.bps);
   const int G = h_q / h_kv;
