@@ -486,16 +486,22 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     const float cs = scale * kLog2e;
     const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
     // stage windows j0 .. j0 + 263 (rows past the visible windows zero-filled)
+    // in two groups, rows [0, 128) and [128, 264): the first half is scored
+    // while the second lands
     {
       const uint32_t dst0 = smem_u32(sc_smem);
-      for (int pc = tid; pc < kScoreRows * C::CH; pc += kSelThreads) {
-        const int r = pc / C::CH, piece = pc - r * C::CH;
-        const int wr = j0 + r;
-        const bool ok = r < kScoreWin + 1 && wr >= 0 && wr < n1;
-        const __nv_bfloat16* src = base + (ok ? static_cast<int64_t>(wr) * D + piece * 8 : 0);
-        cp_async16(dst0 + r * (D * 2) + ((piece ^ ((r & 1) << 2)) << 4), src, ok);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r_lo = half ? kScoreRows / 2 - 4 : 0, r_hi = half ? kScoreRows : kScoreRows / 2 - 4;
+        for (int pc = r_lo * C::CH + tid; pc < r_hi * C::CH; pc += kSelThreads) {
+          const int r = pc / C::CH, piece = pc - r * C::CH;
+          const int wr = j0 + r;
+          const bool ok = r < kScoreWin + 1 && wr >= 0 && wr < n1;
+          const __nv_bfloat16* src = base + (ok ? static_cast<int64_t>(wr) * D + piece * 8 : 0);
+          cp_async16(dst0 + r * (D * 2) + ((piece ^ ((r & 1) << 2)) << 4), src, ok);
+        }
+        cp_async_commit();
       }
-      cp_async_commit();
     }
     // per-head LSE: thread (h, k0) folds the coarse partials k0, k0 + 16, ...
     {
@@ -544,10 +550,14 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     }
     QFrag<D> f;
     load_qfrag<D>(f, qh, lane, G);
-    cp_async_wait0();
+    cp_async_wait1();                          // rows [0, 128): n-tiles 0 .. 15
     __syncthreads();
     const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
     for (int nt = warp; nt * 8 < kScoreWin + 1; nt += 8) {
+      if (nt - warp == 16) {                   // the second half: every warp's third n-tile (16 + warp <= 23)
+        cp_async_wait0();
+        __syncthreads();
+      }
       const int w0 = j0 + nt * 8;
       const int r = nt * 8 + gid;
       const uint4* rowp = reinterpret_cast<const uint4*>(sc_smem + r * (D * 2));
