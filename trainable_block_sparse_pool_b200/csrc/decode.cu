@@ -303,7 +303,11 @@ struct SelScratch {
   uint32_t red[2][kSelThreads / 32];
   int wsum[kSelThreads / 32];
   int digit, above;
+  uint32_t small[32];                 // the keys of a boundary bin of at most 32
+  int nsmall, gt;
+  uint32_t tu;
 };
+constexpr int kSelBins = 2048;        // first radix pass: the top 11 bits
 
 // exclusive prefix sum of v over the CTA's threads in index order; *total
 // gets the sum over all threads
@@ -329,8 +333,9 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* wsum, int* total) 
   return before + x - v;
 }
 
+// keys: shared scratch of cand_cap entries; big: shared scratch of kSelBins ints.
 __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_local, int top_k, int n_sel,
-                                  int cand_cap, int32_t* out, uint32_t* keys, SelScratch& sh) {
+                                  int cand_cap, int32_t* out, uint32_t* keys, int* big, SelScratch& sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = kSelThreads / 32;
   const int b_t = t / 64;
@@ -375,7 +380,69 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
   int hi = range ? 32 - __clz(range) : 0;
   uint32_t prefix = 0;
   int k_rem = top_k;                            // how many of the keys matching prefix are still to take
-  while (hi > 0) {
+  if (hi > 0) {
+    // first pass over the top (up to) 11 bits of u, 2048 bins; thread tid
+    // owns bins [8 tid, 8 tid + 8)
+    const int d1 = min(hi, 11), shift1 = hi - d1, nb1 = 1 << d1;
+    for (int i = tid; i < nb1; i += kSelThreads) big[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < ncand; i += kSelThreads) atomicAdd(&big[(keys[i] - kmin) >> shift1], 1);
+    __syncthreads();
+    int loc = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) loc += (8 * tid + q < nb1) ? big[8 * tid + q] : 0;
+    int tot;
+    const int below = cta_exclusive_scan(loc, sh.wsum, &tot);
+    const int above = tot - below - loc;        // keys in bins above this thread's
+    if (above < k_rem && above + loc >= k_rem) {
+      int acc = above;
+      for (int q = 7; q >= 0; --q) {
+        const int bb = 8 * tid + q;
+        const int hh = (bb < nb1) ? big[bb] : 0;
+        if (acc + hh >= k_rem) { sh.digit = bb; sh.above = acc; break; }
+        acc += hh;
+      }
+    }
+    __syncthreads();
+    const int dg = sh.digit;
+    const int in_bin = big[dg];
+    prefix = static_cast<uint32_t>(dg) << shift1;
+    k_rem -= sh.above;
+    hi = shift1;
+    if (tid == 0) sh.nsmall = 0;
+    __syncthreads();                            // big, digit and above are read by everyone
+    if (hi > 0 && in_bin <= 32) {
+      // the few keys of the boundary bin: one warp sorts them and takes the
+      // k_rem-th largest exactly
+      for (int i = tid; i < ncand; i += kSelThreads) {
+        const uint32_t u = keys[i] - kmin;
+        if ((u >> shift1) == static_cast<uint32_t>(dg)) sh.small[atomicAdd(&sh.nsmall, 1)] = u;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int n = sh.nsmall;
+        uint32_t x = (lane < n) ? sh.small[lane] : 0u;   // 0 sorts last: no key of the bin is below it
+        // bitonic sort, descending across the 32 lanes
+#pragma unroll
+        for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+          for (int j = k >> 1; j > 0; j >>= 1) {
+            const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            x = keep_max ? max(x, y) : min(x, y);
+          }
+        }
+        const uint32_t tu = __shfl_sync(0xffffffffu, x, k_rem - 1);
+        const int gt = __popc(__ballot_sync(0xffffffffu, lane < n && x > tu));
+        if (lane == 0) { sh.tu = tu; sh.gt = gt; }
+      }
+      __syncthreads();
+      prefix = sh.tu;
+      k_rem -= sh.gt;
+      hi = 0;
+    }
+  }
+  while (hi > 0) {                              // a crowded boundary bin: 8 more bits per pass
     const int shift = max(0, hi - 8);
     const int nb = 1 << (hi - shift);
     sh.hist[tid] = 0;
@@ -464,7 +531,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel, float* __restrict__ bscore,
     int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
   using C = ScoreCfg<D>;
-  extern __shared__ __align__(128) uint8_t sc_smem[];            // [kBuf] rows; the selection's keys reuse it
+  extern __shared__ __align__(128) uint8_t sc_smem[];            // [kBuf] rows; the selection's keys and bins reuse it
   uint32_t* sel_keys = reinterpret_cast<uint32_t*>(sc_smem);
   __shared__ float nlse[16];
   __shared__ float2 lsep[16][17];
@@ -600,7 +667,8 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
   if (!s_last) return;
   __threadfence();
   select_blocks_cta(bscore + static_cast<int64_t>(bg) * nblk_cap, t, n_init, n_local, top_k, n_sel, cand_cap,
-                    idx + static_cast<int64_t>(bg) * n_sel, sel_keys, sel_sh);
+                    idx + static_cast<int64_t>(bg) * n_sel, sel_keys,
+                    reinterpret_cast<int*>(sc_smem + ((static_cast<size_t>(cand_cap) * 4 + 15) & ~size_t(15))), sel_sh);
 }
 
 constexpr int kAttWarps = 4;
@@ -1074,7 +1142,8 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
       static_cast<const bf*>(q), static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
       static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache), static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2),
       s->seq_len, s->capacity, s->h_q, s->h_kv, P.cap_c1, P.cap_c2, scale, part2, cnt);
-  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kBuf, static_cast<size_t>(P.cand_cap) * 4);
+  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kBuf,
+                                          static_cast<size_t>(P.cand_cap) * 4 + 16 + dec::kSelBins * 4);
   cudaError_t e = cudaFuncSetAttribute(dec::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(k2_smem));
   if (e != cudaSuccess) return e;
