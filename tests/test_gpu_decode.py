@@ -108,6 +108,15 @@ def test_decode_tiny_d64_g4():
     _run_case(w, prefix=900, steps=130, batch=2, check_every=3)
 
 
+def test_decode_group_sizes():
+    # G = 1 (d = 128) and G = 8 (d = 64): the remaining group sizes of the decode kernels
+    w = dataclasses.replace(gen.WORKLOADS["prefill_32k"], name="decode_g1", h_q=2, h_kv=2, n_local=4, top_k=6, seed=44)
+    _run_case(w, prefix=1200, steps=20, batch=2, check_every=4)
+    w = dataclasses.replace(gen.WORKLOADS["prefill_32k"], name="decode_g8", h_q=16, h_kv=2, d=64, n_local=4, top_k=6,
+                            seed=45)
+    _run_case(w, prefix=2000, steps=20, batch=2, check_every=4)
+
+
 def test_decode_16x128k_sampled():
     # the benchmark's decode workload: 16 sequences x 131072-token cache;
     # the oracle checks two sequences on the first and a later step

@@ -134,6 +134,24 @@ def test_varlen_tiny_d64_g4():
     _full_case(TINY_VARLEN, TINY_VARLEN_LENS, TINY_VARLEN.seed)
 
 
+# The other supported group sizes and head dims.  G = 1 makes one LOCAL CTA
+# (128 / G = 128 tokens) span two 64-token blocks, so its rows have
+# different init/local sets; G = 2 and 8 exercise the remaining template
+# cases of every kernel.
+OTHER_GROUPS = [
+    ("g1_d64", dict(h_q=4, h_kv=4, d=64)),
+    ("g2_d128", dict(h_q=8, h_kv=4, d=128)),
+    ("g8_d64", dict(h_q=16, h_kv=2, d=64)),
+]
+OTHER_LENS = [1300, 129, 2100, 64]
+
+
+@pytest.mark.parametrize("name,shape", OTHER_GROUPS, ids=[g[0] for g in OTHER_GROUPS])
+def test_varlen_group_sizes(name, shape):
+    w = dataclasses.replace(gen.WORKLOADS["prefill_32k"], name=name, n_local=4, top_k=6, seed=31, **shape)
+    _full_case(w, OTHER_LENS, w.seed)
+
+
 def _sampled_case(name, n_rows):
     w = gen.WORKLOADS[name]
     data = gen.make_prefill(w)
