@@ -54,7 +54,11 @@ enum {
 };
 
 enum { INFLLM2_OUT_BF16 = 0, INFLLM2_OUT_F32 = 1 };
-enum { INFLLM2_LSE_APPROX = 0 };
+/* lse_mode: APPROX takes each head's log-sum-exp from the coarse C2 scores
+ * (the pages' approximation, 1.25x the cost of one scoring pass); EXACT
+ * takes it from the C1 scores themselves (the two-pass computation it
+ * replaces, 2x; each row of S then sums to G).  [top168] §四. */
+enum { INFLLM2_LSE_APPROX = 0, INFLLM2_LSE_EXACT = 1 };
 
 /* Method parameters.  Defaults (infllm2_default_params) are the pages'
  * values: block B = 64 ([blog] worked example "每块 64 个 token");
@@ -132,6 +136,8 @@ int infllm2_compress_k(const void* K, const infllm2_varlen* vl, int32_t h_kv, in
  * A C1 window j is visible when 16j+31 <= t, a C2 window m when 64m+127 <= t
  * (positions within the sequence).  Rows with no visible C2 window
  * (t < 127) take the exact log-sum-exp over their visible C1 windows.
+ * With p->lse_mode == INFLLM2_LSE_EXACT, LSE_h is the log-sum-exp of s_h
+ * over the visible C1 windows for every row.
  * Only visible entries are written; the per-head scores never reach HBM.
  *   Q          bf16 [total, h_q, d]
  *   K_c1, K_c2 as written by infllm2_compress_k
@@ -239,6 +245,8 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V,
  * infllm2_decode_workspace_bytes (device, caller-owned, no alignment beyond
  * 16 bytes, contents need no initialisation and carry nothing from one step
  * to the next; one workspace must not serve two steps in flight at once).
+ * The decode step takes the LSE approximation only (lse_mode EXACT is
+ * INFLLM2_ERR_UNSUPPORTED here).
  * Capacities above 1441792 tokens (more than 22528 candidate blocks) are
  * INFLLM2_ERR_UNSUPPORTED, and infllm2_decode_workspace_bytes returns 0 for
  * them.  infllm2_decode_build_caches pools the seq_len[b] tokens already in

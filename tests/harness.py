@@ -80,10 +80,10 @@ class GpuRun:
         return o
 
 
-def oracle_sequences(data: dict, w, which=None):
+def oracle_sequences(data: dict, w, which=None, p=None):
     """fp64 oracle sequence objects (pooled keys included) for the sequences
     listed in `which` (all by default)."""
-    p = oracle_params(w)
+    p = oracle_params(w) if p is None else p
     cu = data["cu_seqlens"].tolist()
     seqs = {}
     for s in (range(len(data["lens"])) if which is None else which):

@@ -152,6 +152,41 @@ def test_varlen_group_sizes(name, shape):
     _full_case(w, OTHER_LENS, w.seed)
 
 
+def test_exact_lse_mode():
+    # lse_mode EXACT: each head's log-sum-exp over the visible C1 windows
+    # ([top168] §四's two-pass computation).  S_shared against the oracle's
+    # exact variant on every row, and every row with a visible window sums
+    # to G.
+    import trainable_block_sparse_pool_b200 as T
+    w = VARLEN_SMALL
+    data = gen.make_prefill(w, lens=VARLEN_SMALL_LENS, seed=12)
+    run = H.GpuRun(data, w)
+    run.p.lse_mode = T.LSE_EXACT
+    run.compress()
+    run.scores()
+    torch.cuda.synchronize()
+    op = dataclasses.replace(H.oracle_params(w), lse_mode="exact")
+    seqs = H.oracle_sequences(data, w, p=op)
+    S_gpu = run.S.cpu().numpy()
+    rows = np.arange(run.vl.total)
+    sidx, tloc = H.seq_of_rows(run.lens, rows)
+    worst_rel, worst_sum, nrows = 0.0, 0.0, 0
+    for row, s, t in zip(rows, sidx, tloc):
+        for g in range(w.h_kv):
+            S_or = seqs[int(s)].shared_scores(int(t), g)
+            n1 = S_or.shape[0]
+            if n1 == 0:
+                continue
+            got = S_gpu[g, row, :n1].astype(np.float64)
+            worst_rel = max(worst_rel, float((np.abs(got - S_or) / np.maximum(S_or, 1e-30)).max()))
+            worst_sum = max(worst_sum, abs(float(got.sum()) - w.group) / w.group)
+            nrows += 1
+    assert nrows > 0
+    assert worst_rel <= H.S_RTOL, worst_rel
+    assert worst_sum <= H.S_RTOL, worst_sum
+    assert T_status() == 0
+
+
 def _sampled_case(name, n_rows):
     w = gen.WORKLOADS[name]
     data = gen.make_prefill(w)

@@ -25,9 +25,11 @@ __all__ = [
     "infllm2_get_device_status", "infllm2_clear_device_status", "infllm2_debug_wait_timeout",
     "infllm2_probe_l2_gather",
     "DecodeState", "make_decode_state", "infllm2_decode_workspace_bytes", "infllm2_decode_build_caches",
-    "infllm2_decode_step", "OUT_BF16", "OUT_F32",
+    "infllm2_decode_step", "OUT_BF16", "OUT_F32", "LSE_APPROX", "LSE_EXACT",
 ]
 
+LSE_APPROX = 0
+LSE_EXACT = 1
 OUT_BF16 = 0
 OUT_F32 = 1
 

@@ -55,7 +55,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static bool geometry_supported(const infllm2_params* p) {
   return p->block_size == 64 && p->c1_len == 32 && p->c1_stride == 16 && p->c2_len == 128 &&
          p->c2_stride == 64 && p->pool_len == 5 && p->pool_stride == 4 && p->pool_pad == 1 &&
-         p->lse_mode == INFLLM2_LSE_APPROX;
+         (p->lse_mode == INFLLM2_LSE_APPROX || p->lse_mode == INFLLM2_LSE_EXACT);
 }
 
 static int check_varlen(const infllm2_varlen* vl) {
@@ -169,7 +169,8 @@ int infllm2_shared_scores(const void* Q, const void* K_c1, const void* K_c2, con
   bool map_fail = false;
   cudaError_t e = launch_shared_scores(Q, K_c1, K_c2, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total,
                                        vl->total_c1, vl->total_c2, h_q, h_kv, d, S, ld, softmax_scale(p, d),
-                                       static_cast<cudaStream_t>(stream), &map_fail);
+                                       p->lse_mode == INFLLM2_LSE_EXACT, static_cast<cudaStream_t>(stream),
+                                       &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
@@ -270,7 +271,7 @@ static DecodePlan plan_of(const infllm2_decode_state* st, const infllm2_params* 
 }
 
 size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infllm2_params* p) {
-  if (check_decode_state(st) || check_params(p)) return 0;
+  if (check_decode_state(st) || check_params(p) || p->lse_mode != INFLLM2_LSE_APPROX) return 0;
   const DecodePlan P = plan_of(st, p);
   return decode_plan_supported(P) ? P.bytes : 0;
 }
@@ -278,6 +279,7 @@ size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infl
 int infllm2_decode_build_caches(const infllm2_decode_state* st, const infllm2_params* p, void* stream) {
   int r;
   if ((r = check_decode_state(st)) || (r = check_params(p))) return r;
+  if (p->lse_mode != INFLLM2_LSE_APPROX) return INFLLM2_ERR_UNSUPPORTED;
   const DecodePlan P = plan_of(st, p);
   if (!decode_plan_supported(P)) return INFLLM2_ERR_UNSUPPORTED;
   cudaError_t e = launch_decode_build_caches(st, P, static_cast<cudaStream_t>(stream));
@@ -288,6 +290,7 @@ int infllm2_decode_step(const infllm2_decode_state* st, const void* q, const voi
                         void* out, void* workspace, size_t workspace_bytes, const infllm2_params* p, void* stream) {
   int r;
   if ((r = check_decode_state(st)) || (r = check_params(p))) return r;
+  if (p->lse_mode != INFLLM2_LSE_APPROX) return INFLLM2_ERR_UNSUPPORTED;   // decode keeps the approximation
   if (!q || !k_new || !v_new || !out || !workspace || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
       !aligned16(out) || !aligned16(workspace))
     return INFLLM2_ERR_INVALID_ARG;

@@ -4,7 +4,10 @@
 // For one kv group g and a tile of TQ = 256/G query tokens (256 query rows
 // (t, h), h the G heads of the group) a CTA computes
 //   phase A  LSE(t,h) = logsumexp_m  scale * q[t,h] . K_c2[g,m]  over the
-//            visible coarse windows (the LSE approximation),
+//            visible coarse windows (the LSE approximation), or, in the
+//            EXACT form, over the visible stage-1 windows K_c1 themselves
+//            (the two-pass computation the approximation replaces: the
+//            rows of S then sum to G),
 //   phase B  S[g,t,j] = sum_h exp(scale * q[t,h] . K_c1[g,j] - LSE(t,h))
 //            over the visible stage-1 windows,
 // and writes only S (the group sum happens on chip, the per-head scores
@@ -63,7 +66,7 @@ __device__ __forceinline__ void set_abort(Bars* b) {
   *reinterpret_cast<volatile int*>(&b->abort) = 1;
 }
 
-template <int D, int G>
+template <int D, int G, bool EXACT>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK1,
     const __grid_constant__ CUtensorMap tmK2, const __nv_bfloat16* __restrict__ Q,
@@ -92,8 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
   const int c1_off = pooled_offset_block(cu, s, 32, 16, red);
   const int c2_off = pooled_offset_block(cu, s, 128, 64, red);
   const int n1_max = visible_windows_dev(t_last, 32, 16);
-  const int n2_max = visible_windows_dev(t_last, 128, 64);
-  const int nA = (n2_max + kKeysPerTile - 1) / kKeysPerTile;   // coarse key tiles
+  const int n2_max = EXACT ? n1_max : visible_windows_dev(t_last, 128, 64);
+  const int nA = (n2_max + kKeysPerTile - 1) / kKeysPerTile;   // key tiles of phase A
   const int nB = (n1_max + kKeysPerTile - 1) / kKeysPerTile;   // stage-1 key tiles
   const float c = scale * kLog2e;
 
@@ -127,7 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
         uint8_t* dst = sK + st * C::kStageBytes;
         if (it < nA) {
           for (int ch = 0; ch < C::KCH; ++ch)
-            tma_load_3d(dst + ch * C::kKChunk, &tmK2, &bars->full[st], ch * 64, c2_off + it * kKeysPerTile, g);
+            tma_load_3d(dst + ch * C::kKChunk, EXACT ? &tmK1 : &tmK2, &bars->full[st], ch * 64,
+                        (EXACT ? c1_off : c2_off) + it * kKeysPerTile, g);
         } else {
           const int kt = it - nA;
           for (int ch = 0; ch < C::KCH; ++ch)
@@ -188,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
     const int r = hh * 128 + q4 * 32 + lane;
     const int t_loc = r / G, h = r % G;
     const int t = t0 + t_loc;
-    const int n2 = visible_windows_dev(t, 128, 64);
+    const int n2 = EXACT ? visible_windows_dev(t, 32, 16) : visible_windows_dev(t, 128, 64);
     float m_run = -INFINITY, l_run = 0.f;
     int it = 0;
     bool ok = true;
@@ -229,6 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
     float lse;
     if (n2 > 0) {
       lse = m_run + log2f(l_run);
+    } else if (EXACT) {
+      lse = INFINITY;                   // no visible window: the row is empty
     } else {
       // no coarse window visible yet (t < 127): exact log-sum-exp over the
       // visible stage-1 windows (at most 6), straight from global memory
@@ -330,7 +336,7 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dim
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int G>
+template <int D, int G, bool EXACT>
 static cudaError_t launch_score_t(const void* Q, const void* Kc1, const void* Kc2, const int32_t* cu, int batch,
                                   int max_seqlen, int64_t total, int64_t total_c1, int64_t total_c2, int h_q,
                                   int h_kv, float* S, int64_t ld, float scale, cudaStream_t st, bool* map_fail) {
@@ -354,7 +360,7 @@ static cudaError_t launch_score_t(const void* Q, const void* Kc1, const void* Kc
     const uint32_t box[3] = {64, score::kKeysPerTile, 1};
     if (!make_tmap(&mK2, Kc2, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
   }
-  auto kern = score::score_kernel<D, G>;
+  auto kern = score::score_kernel<D, G, EXACT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((max_seqlen + C::TQ - 1) / C::TQ, batch, h_kv);
@@ -367,13 +373,15 @@ static cudaError_t launch_score_t(const void* Q, const void* Kc1, const void* Kc
 
 cudaError_t launch_shared_scores(const void* Q, const void* Kc1, const void* Kc2, const int32_t* cu, int batch,
                                  int max_seqlen, int64_t total, int64_t total_c1, int64_t total_c2, int h_q,
-                                 int h_kv, int d, float* S, int64_t ld, float scale, cudaStream_t st,
+                                 int h_kv, int d, float* S, int64_t ld, float scale, bool exact, cudaStream_t st,
                                  bool* map_fail) {
   const int G = h_q / h_kv;
-#define INFLLM2_SCORE_CASE(DD, GG)                                                                             \
-  if (d == DD && G == GG)                                                                                     \
-    return launch_score_t<DD, GG>(Q, Kc1, Kc2, cu, batch, max_seqlen, total, total_c1, total_c2, h_q, h_kv, S, \
-                                  ld, scale, st, map_fail);
+#define INFLLM2_SCORE_CASE(DD, GG)                                                                                 \
+  if (d == DD && G == GG)                                                                                         \
+    return exact ? launch_score_t<DD, GG, true>(Q, Kc1, Kc2, cu, batch, max_seqlen, total, total_c1, total_c2, h_q, \
+                                                h_kv, S, ld, scale, st, map_fail)                                 \
+                 : launch_score_t<DD, GG, false>(Q, Kc1, Kc2, cu, batch, max_seqlen, total, total_c1, total_c2,   \
+                                                 h_q, h_kv, S, ld, scale, st, map_fail);
   INFLLM2_SCORE_CASE(128, 16)
   INFLLM2_SCORE_CASE(128, 8)
   INFLLM2_SCORE_CASE(128, 4)
