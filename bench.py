@@ -318,6 +318,8 @@ def main():
     ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--decode-batch", type=int, default=0, help="sequences of the decode case (0: the workload's 16)")
+    ap.add_argument("--lse", default="approx", choices=["approx", "exact"],
+                    help="LSE of the scoring step: the coarse approximation (default) or the exact two-pass form")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -364,7 +366,8 @@ def main():
         return
 
     data = gen.make_prefill(w)
-    p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+    p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k,
+                         lse_mode=T.LSE_EXACT if args.lse == "exact" else T.LSE_APPROX)
     Q, K, V = data["Q"].to(dev), data["K"].to(dev), data["V"].to(dev)
     cu = data["cu_seqlens"].to(dev)
     vl = T.make_varlen(data["lens"], cu, p)
@@ -510,7 +513,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q,V; K with per-block offsets)",
         "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
-                   "n_sel": w.n_sel, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "n_sel": w.n_sel, "lse": args.lse,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "working set larger than L2 (Q 1 GiB, S_shared 4.3 GB); no extra flush"},
         "e2e": e2e,
         "gpu_launches": (len(kernels) + 1) * args.steps,   # the sparse call is two launches (local + top-k)
