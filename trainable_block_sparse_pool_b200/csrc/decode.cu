@@ -506,9 +506,11 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
 }
 
 // ---------------------------------------------------------------- K2: scores, max-pool, selection
-// grid (batch*h_kv, nsplit1), 8 warps; CTA c covers stage-1 windows
+// grid (nsplit1, batch*h_kv), 8 warps; CTA c covers stage-1 windows
 // [256c - 1, 256c + 255) and writes block scores [64c, 64c + 64) (one
-// window of halo, so a block never straddles CTAs).  Per window: the 16
+// window of halo, so a block never straddles CTAs).  The split index runs
+// fastest, so the (sequence, group) pairs complete one after another and
+// their selections overlap the scoring of the later ones.  Per window: the 16
 // heads' scores, normalised by their LSE and summed over the group
 // ([top168] §三 second stage, §四); per block: the max over its 5 windows.
 // The CTA's pooled keys are staged with cp.async into shared memory
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
   __shared__ float sw[kScoreWin + 8];
   __shared__ SelScratch sel_sh;
   __shared__ int s_last;
-  const int bg = blockIdx.x, c = blockIdx.y;
+  const int bg = blockIdx.y, c = blockIdx.x;
   const int b = bg / h_kv, g = bg % h_kv;
   const int G = h_q / h_kv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -662,7 +664,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
   // the last CTA of (b, g) to finish selects the blocks
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&cnt[bg], 1u) == gridDim.y - 1);
+  if (tid == 0) s_last = (atomicAdd(&cnt[bg], 1u) == gridDim.x - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -1147,7 +1149,7 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
   cudaError_t e = cudaFuncSetAttribute(dec::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(k2_smem));
   if (e != cudaSuccess) return e;
-  dec::score_select_kernel<D><<<dim3(bg, P.nsplit1), dec::kSelThreads, k2_smem, st>>>(
+  dec::score_select_kernel<D><<<dim3(P.nsplit1, bg), dec::kSelThreads, k2_smem, st>>>(
       static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->capacity, s->h_q,
       s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt);
   e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
