@@ -30,7 +30,6 @@ namespace dec {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kLseWin = 128;   // coarse windows per LSE CTA
-constexpr int kScoreWin = 256; // stage-1 windows per score CTA (64 blocks)
 constexpr int kMaxSplits = 256; // attention splits per (sequence, group)
 constexpr float kRescaleLog2 = 8.f; // attention: raise the reference max only past this margin
 
@@ -111,6 +110,8 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool f
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_n() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -179,7 +180,7 @@ __device__ void pool_window(int len, const __nv_bfloat16* kc, int64_t seq0, int 
 //    then uses it.
 //  * Every CTA writes (max, sum) in log2 units of its windows' scores, per
 //    head: part2[(bg*nsplit2 + c)*16 + h].
-// Counters (cnt): [0, nbg) score CTAs done per (b, g); [nbg, 2 nbg)
+// Counters (cnt): [0, nbg) score pieces done per (b, g); [nbg, 2 nbg)
 // attention CTAs done per (b, g); [2 nbg, 2 nbg + batch) groups of b merged.
 template <int D>
 __global__ void __launch_bounds__(128) lse_append_kernel(
@@ -506,174 +507,295 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
 }
 
 // ---------------------------------------------------------------- K2: scores, max-pool, selection
-// grid (nsplit1, batch*h_kv), 8 warps; CTA c covers stage-1 windows
-// [256c - 1, 256c + 255) and writes block scores [64c, 64c + 64) (one
-// window of halo, so a block never straddles CTAs).  The split index runs
-// fastest, so the (sequence, group) pairs complete one after another and
-// their selections overlap the scoring of the later ones.  Per window: the 16
-// heads' scores, normalised by their LSE and summed over the group
-// ([top168] §三 second stage, §四); per block: the max over its 5 windows.
-// The CTA's pooled keys are staged with cp.async into shared memory
-// (16-byte pieces of a row XOR-swizzled by the row's parity, so the
-// fragment loads are free of bank conflicts), which keeps registers low
-// enough for three CTAs per SM; the LSE partials and the query rows load
-// meanwhile.  The last CTA of (b, g) to finish runs the selection.
-constexpr int kScoreRows = kScoreWin / 8 * 8 + 8;   // 33 n-tiles of 8 windows; 257 used
+// The scoring streams over pieces.  A piece is kPieceWin = 128 consecutive
+// stage-1 windows (32 blocks) of one (sequence, group); (b, g) has np(b)
+// pieces, enough to cover its candidate blocks [0, loc_lo), or a single empty
+// piece when the selection needs no scores.  The pieces of all (b, g), in
+// (b, g) order, are cut into gridDim.x contiguous ranges of near-equal
+// length, and a CTA walks its range through a kScoreStages-deep cp.async
+// ring, so the pooled-key reads of the whole step stream without the gaps of
+// a grid of short-lived CTAs.
+// Per window: the 16 heads' scores, normalised by their LSE and summed over
+// the group ([top168] §三 second stage, §四); per block i: the max over
+// windows 4i-1 .. 4i+3.  The window before a piece (the first block's halo)
+// is the previous piece's last window when the range holds that piece, else
+// an extra staged row.  The 16-byte pieces of a staged row are XOR-swizzled
+// by the row's parity, so the fragment loads are free of bank conflicts.
+// A completion counter per (b, g) counts the pieces done; the CTA that
+// completes the last one runs that selection once its range is done.
+constexpr int kPieceWin = 128;                  // stage-1 windows per piece
+constexpr int kPieceBlk = kPieceWin / 4;        // blocks per piece
+constexpr int kPieceRows = kPieceWin + 8;       // + one n-tile whose first row is the halo window
+constexpr int kScoreStages = 2;
+constexpr int kMaxRange = 64;                   // pieces per CTA at most (the host sizes the grid)
 
 template <int D>
 struct ScoreCfg {
-  static constexpr int CH = D / 8;                                 // 16-byte pieces per row
-  static constexpr uint32_t kBuf = kScoreRows * D * 2;             // the CTA's rows
+  static constexpr int CH = D / 8;                                  // 16-byte pieces per row
+  static constexpr uint32_t kStage = kPieceRows * D * 2;
+  static constexpr uint32_t kRing = kScoreStages * kStage;
 };
+
+// Pieces of a (sequence, group) whose new token is at t: its scored blocks
+// are [0, loc_lo); a single empty piece when every candidate is taken (or t
+// is out of range, which the append kernel records).
+__device__ __forceinline__ bool needs_scores(int t, int n_init, int n_local, int top_k) {
+  const int b_t = t / 64;
+  return max(0, b_t - n_local + 1) - min(n_init, b_t + 1) > top_k;
+}
+__device__ __forceinline__ int score_pieces(int t, int capacity, int n_init, int n_local, int top_k) {
+  if (t < 0 || t >= capacity || !needs_scores(t, n_init, n_local, top_k)) return 1;
+  return (max(0, t / 64 - n_local + 1) + kPieceBlk - 1) / kPieceBlk;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
-    const float2* __restrict__ part2, int nsplit2, int capacity, int h_q, int h_kv, int cap_c1, int nblk_cap,
-    int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel, float* __restrict__ bscore,
-    int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
+    const float2* __restrict__ part2, int nsplit2, int batch, int capacity, int h_q, int h_kv, int cap_c1,
+    int nblk_cap, int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel,
+    float* __restrict__ bscore, int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
   using C = ScoreCfg<D>;
-  extern __shared__ __align__(128) uint8_t sc_smem[];            // [kBuf] rows; the selection's keys and bins reuse it
-  uint32_t* sel_keys = reinterpret_cast<uint32_t*>(sc_smem);
+  extern __shared__ __align__(128) uint8_t sc_smem[];   // the ring; the selection's keys and bins reuse it
+  __shared__ uint32_t plist[kMaxRange];                // bg << 16 | piece index within (b, g)
+  __shared__ int pn1[kMaxRange];                       // visible stage-1 windows; -1: t out of range
+  __shared__ int pnp[kMaxRange];                       // pieces of the piece's (b, g); 0: not scored
   __shared__ float nlse[16];
-  __shared__ float2 lsep[16][17];
-  __shared__ float sw[kScoreWin + 8];
+  __shared__ float sw[2][kPieceWin + 8];
   __shared__ SelScratch sel_sh;
-  __shared__ int s_last;
-  const int bg = blockIdx.y, c = blockIdx.x;
-  const int b = bg / h_kv, g = bg % h_kv;
+  __shared__ int owed[kMaxRange];
+  __shared__ int nowed;
   const int G = h_q / h_kv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
-  const int t = seq_len[b];
-  if (t < 0 || t >= capacity) return;          // recorded by the append kernel
-  const int n1 = min(visible_windows_dev(t, 32, 16), cap_c1);
-  const int n2 = visible_windows_dev(t, 128, 64);
-  const int j0 = c * kScoreWin - 1;
-  const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
-  if (c == 0 || j0 + 1 < n1) {                 // this CTA has visible windows
-    const float cs = scale * kLog2e;
-    const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
-    // stage windows j0 .. j0 + 263 (rows past the visible windows zero-filled)
-    // in two groups, rows [0, 128) and [128, 264): the first half is scored
-    // while the second lands
-    {
-      const uint32_t dst0 = smem_u32(sc_smem);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r_lo = half ? kScoreRows / 2 - 4 : 0, r_hi = half ? kScoreRows : kScoreRows / 2 - 4;
-        for (int pc = r_lo * C::CH + tid; pc < r_hi * C::CH; pc += kSelThreads) {
-          const int r = pc / C::CH, piece = pc - r * C::CH;
-          const int wr = j0 + r;
-          const bool ok = r < kScoreWin + 1 && wr >= 0 && wr < n1;
-          const __nv_bfloat16* src = base + (ok ? static_cast<int64_t>(wr) * D + piece * 8 : 0);
-          cp_async16(dst0 + r * (D * 2) + ((piece ^ ((r & 1) << 2)) << 4), src, ok);
-        }
-        cp_async_commit();
+  const float cs = scale * kLog2e;
+
+  // ---- this CTA's range [P0, P1) of the flattened piece list
+  int R = 0;
+  {
+    int total = -1;                            // known after one pass when the batch fits one scan
+    if (batch > kSelThreads) {
+      total = 0;
+      for (int b0 = 0; b0 < batch; b0 += kSelThreads) {
+        const int b = b0 + tid;
+        const int v = (b < batch) ? h_kv * score_pieces(seq_len[b], capacity, n_init, n_local, top_k) : 0;
+        int tot;
+        cta_exclusive_scan(v, sel_sh.wsum, &tot);
+        total += tot;
       }
     }
-    // per-head LSE: thread (h, k0) folds the coarse partials k0, k0 + 16, ...
-    {
-      const int h = tid & 15, k0 = tid >> 4;
-      float mm = -INFINITY, ll = 0.f;
-      if (h < G && n2 > 0) {
-        for (int kk = k0; kk < nsplit2; kk += 16) {
-          const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + kk) * 16 + h];
-          const float mn = fmaxf(mm, v.x);
-          if (mn != -INFINITY) {
-            ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
-            mm = mn;
-          }
-        }
+    int base = 0;
+    for (int b0 = 0; b0 < batch; b0 += kSelThreads) {
+      const int b = b0 + tid;
+      const int tb = (b < batch) ? seq_len[b] : -1;
+      const int np = (b < batch) ? score_pieces(tb, capacity, n_init, n_local, top_k) : 0;
+      int tot;
+      const int ex = cta_exclusive_scan(h_kv * np, sel_sh.wsum, &tot);
+      if (total < 0) total = tot;
+      const int64_t P0 = static_cast<int64_t>(total) * blockIdx.x / gridDim.x;
+      const int64_t P1 = static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x;
+      R = static_cast<int>(P1 - P0);
+      if (R > kMaxRange) {                     // the host sizes the grid so that this cannot happen
+        if (tid == 0 && b0 == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+        return;
       }
-      lsep[h][k0] = make_float2(mm, ll);
+      // pieces [base + ex, base + ex + h_kv * np) belong to sequence b
+      const bool valid = tb >= 0 && tb < capacity;
+      const int n1 = valid ? min(visible_windows_dev(tb, 32, 16), cap_c1) : -1;
+      const bool sc = valid && needs_scores(tb, n_init, n_local, top_k);
+      const int64_t lo = max(static_cast<int64_t>(base) + ex, P0);
+      const int64_t hi = min(static_cast<int64_t>(base) + ex + h_kv * np, P1);
+      for (int64_t i = lo; i < hi; ++i) {
+        const int rem = static_cast<int>(i - base - ex);
+        const int g = rem / np, p = rem - g * np;
+        const int j = static_cast<int>(i - P0);
+        plist[j] = (static_cast<uint32_t>(b * h_kv + g) << 16) | static_cast<uint32_t>(p);
+        pn1[j] = n1;
+        pnp[j] = sc ? np : 0;
+      }
+      base += tot;
+      if (base >= P1) break;                   // uniform: base and P1 are the same in every thread
     }
+    if (tid == 0) nowed = 0;
     __syncthreads();
-    if (tid < 16) {
-      const int h = tid;
-      float mm = -INFINITY, ll = 0.f;
-      if (h < G) {
-        if (n2 > 0) {
-          for (int kk = 0; kk < 16; ++kk) {
-            const float2 v = lsep[h][kk];
-            const float mn = fmaxf(mm, v.x);
-            if (mn != -INFINITY) {
-              ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
-              mm = mn;
-            }
-          }
-        } else {
-          // no coarse window yet (t < 127): exact log-sum-exp over the visible stage-1 windows
-          for (int j = 0; j < n1; ++j) {
-            float dot = 0.f;
-            for (int e = 0; e < D; ++e)
-              dot += __bfloat162float(qh[h * D + e]) * __bfloat162float(base[static_cast<int64_t>(j) * D + e]);
-            const float x = dot * cs;
-            const float mn = fmaxf(mm, x);
-            ll = ll * ex2(mm - mn) + ex2(x - mn);
-            mm = mn;
-          }
+  }
+  if (R == 0) return;
+  auto bg_of = [&](int j) { return static_cast<int>(plist[j] >> 16); };
+  auto p_of = [&](int j) { return static_cast<int>(plist[j] & 0xffffu); };
+  auto seg_first = [&](int j) { return j == 0 || bg_of(j - 1) != bg_of(j); };
+  auto seg_last = [&](int j) { return j == R - 1 || bg_of(j + 1) != bg_of(j); };
+
+  // stage piece j (rows past the visible windows zero-filled; the halo row
+  // only for the first piece of a range segment)
+  auto stage = [&](int j) {
+    if (j < R && pnp[j] > 0) {
+      const int bg = bg_of(j), p = p_of(j), n1 = pn1[j];
+      const int w0 = p * kPieceWin;
+      const bool halo = seg_first(j) && p > 0;
+      const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
+      const uint32_t dst0 = smem_u32(sc_smem) + (j % kScoreStages) * C::kStage;
+      const int nrows = halo ? kPieceRows : kPieceWin;
+      for (int pc = tid; pc < nrows * C::CH; pc += kSelThreads) {
+        const int r = pc / C::CH, piece = pc - r * C::CH;
+        const int wr = (r < kPieceWin) ? w0 + r : (r == kPieceWin ? w0 - 1 : -1);
+        const bool ok = wr >= 0 && wr < n1;
+        const __nv_bfloat16* src = base + (ok ? static_cast<int64_t>(wr) * D + piece * 8 : 0);
+        cp_async16(dst0 + r * (D * 2) + ((piece ^ ((r & 1) << 2)) << 4), src, ok);
+      }
+    }
+    cp_async_commit();
+  };
+  // the group's negated log-sum-exp per head (log2 units) from the coarse
+  // partials: thread (h, k0) folds partials k0, k0 + 16, ..., then the 16
+  // lanes of h combine
+  auto group_lse = [&](int j) {                // every thread; scored pieces only
+    const int bg = bg_of(j), n1 = pn1[j];
+    const int b = bg / h_kv, g = bg - b * h_kv;
+    const int tb = seq_len[b];
+    const int n2 = visible_windows_dev(tb, 128, 64);
+    const int h = tid >> 4, k0 = tid & 15;
+    float mm = -INFINITY, ll = 0.f;
+    if (h < G && n2 > 0) {
+      for (int kk = k0; kk < nsplit2; kk += 16) {
+        const float2 v = part2[(static_cast<int64_t>(bg) * nsplit2 + kk) * 16 + h];
+        const float mn = fmaxf(mm, v.x);
+        if (mn != -INFINITY) {
+          ll = ll * ex2(mm - mn) + v.y * ex2(v.x - mn);
+          mm = mn;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, mm, o);
+      const float lo = __shfl_xor_sync(0xffffffffu, ll, o);
+      const float mn = fmaxf(mm, mo);
+      if (mn != -INFINITY) {
+        ll = ll * ex2(mm - mn) + lo * ex2(mo - mn);
+        mm = mn;
+      }
+    }
+    if (k0 == 0) {
+      if (h < G && n2 <= 0 && n1 > 0) {
+        // no coarse window yet (t < 127): exact log-sum-exp over the visible stage-1 windows
+        const __nv_bfloat16* qh = q + (static_cast<int64_t>(b) * h_q + g * G) * D;
+        const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
+        mm = -INFINITY;
+        ll = 0.f;
+        for (int w = 0; w < n1; ++w) {
+          float dot = 0.f;
+          for (int e = 0; e < D; ++e)
+            dot += __bfloat162float(qh[h * D + e]) * __bfloat162float(base[static_cast<int64_t>(w) * D + e]);
+          const float x = dot * cs;
+          const float mn = fmaxf(mm, x);
+          ll = ll * ex2(mm - mn) + ex2(x - mn);
+          mm = mn;
         }
       }
       nlse[h] = (h < G && ll > 0.f) ? -(mm + log2f(ll)) : -INFINITY;
     }
-    QFrag<D> f;
-    load_qfrag<D>(f, qh, lane, G);
-    cp_async_wait1();                          // rows [0, 128): n-tiles 0 .. 15
-    __syncthreads();
-    const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
-    for (int nt = warp; nt * 8 < kScoreWin + 1; nt += 8) {
-      if (nt - warp == 16) {                   // the second half: every warp's third n-tile (16 + warp <= 23)
-        cp_async_wait0();
+  };
+
+#pragma unroll
+  for (int s = 0; s < kScoreStages - 1; ++s) stage(s);
+  if (pnp[0] > 0) group_lse(0);
+  QFrag<D> f;
+  {
+    const int bg = bg_of(0), b = bg / h_kv, g = bg - b * h_kv;
+    load_qfrag<D>(f, q + (static_cast<int64_t>(b) * h_q + g * G) * D, lane, G);
+  }
+  int seg_start = 0;
+  for (int j = 0; j < R; ++j) {
+    cp_async_wait_n<kScoreStages - 2>();
+    __syncthreads();                           // piece j landed; stage (j - 1) % S and sw[(j + 1) & 1] are free
+    stage(j + kScoreStages - 1);
+    const int bg = bg_of(j), p = p_of(j), n1 = pn1[j];
+    const bool live = pnp[j] > 0;
+    if (j > 0 && seg_first(j)) {
+      seg_start = j;
+      if (live) {
+        group_lse(j);
         __syncthreads();
-      }
-      const int w0 = j0 + nt * 8;
-      const int r = nt * 8 + gid;
-      const uint4* rowp = reinterpret_cast<const uint4*>(sc_smem + r * (D * 2));
-      uint4 kv[D / 32];
-#pragma unroll
-      for (int p = 0; p < D / 32; ++p) kv[p] = rowp[(4 * p + tig) ^ ((r & 1) << 2)];
-      float sc[4];
-      scores_16x8_reg<D>(sc, f, kv);
-      // head-group sum for keys 2tig and 2tig+1: two heads here, the other 14 on the lanes with the same tig
-      float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
-      float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        e0 += __shfl_xor_sync(0xffffffffu, e0, o);
-        e1 += __shfl_xor_sync(0xffffffffu, e1, o);
-      }
-      if (gid == 0) {
-        const int i0 = nt * 8 + 2 * tig;
-        if (i0 < kScoreWin + 8) sw[i0] = (w0 + 2 * tig >= 0 && w0 + 2 * tig < n1) ? e0 : -INFINITY;
-        if (i0 + 1 < kScoreWin + 8) sw[i0 + 1] = (w0 + 2 * tig + 1 >= 0 && w0 + 2 * tig + 1 < n1) ? e1 : -INFINITY;
+        const int b = bg / h_kv, g = bg - b * h_kv;
+        load_qfrag<D>(f, q + (static_cast<int64_t>(b) * h_q + g * G) * D, lane, G);
       }
     }
-    __syncthreads();
-    // block scores: block blk = 64c + i takes windows 4 blk - 1 .. 4 blk + 3 = sw[4i .. 4i + 4]
-    if (tid < kScoreWin / 4) {
-      const int blk = c * (kScoreWin / 4) + tid;
-      if (blk < nblk_cap) {
-        float m = -INFINITY;
+    const int w0 = p * kPieceWin;
+    const bool halo = seg_first(j) && p > 0;
+    float* swc = sw[j & 1];
+    if (live) {
+      const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
+      const uint8_t* rows = sc_smem + (j % kScoreStages) * C::kStage;
+      const int ntiles = halo ? kPieceWin / 8 + 1 : kPieceWin / 8;
+      for (int nt = warp; nt < ntiles; nt += kSelThreads / 32) {
+        const int r = nt * 8 + gid;
+        const uint4* rowp = reinterpret_cast<const uint4*>(rows + r * (D * 2));
+        uint4 kv[D / 32];
 #pragma unroll
-        for (int q4 = 0; q4 < 5; ++q4) m = fmaxf(m, sw[4 * tid + q4]);
-        bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
+        for (int pp = 0; pp < D / 32; ++pp) kv[pp] = rowp[(4 * pp + tig) ^ ((r & 1) << 2)];
+        float sc[4];
+        scores_16x8_reg<D>(sc, f, kv);
+        // head-group sum for windows 2tig and 2tig+1 of the n-tile: two heads here, the other 14 on the lanes with the same tig
+        float e0 = ((gid < G) ? ex2(fmaf(sc[0], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[2], cs, nl1)) : 0.f);
+        float e1 = ((gid < G) ? ex2(fmaf(sc[1], cs, nl0)) : 0.f) + ((gid + 8 < G) ? ex2(fmaf(sc[3], cs, nl1)) : 0.f);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          e0 += __shfl_xor_sync(0xffffffffu, e0, o);
+          e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+        }
+        if (gid == 0) {
+          if (nt < kPieceWin / 8) {
+            const int wa = w0 + nt * 8 + 2 * tig;
+            swc[1 + nt * 8 + 2 * tig] = (wa < n1) ? e0 : -INFINITY;
+            swc[2 + nt * 8 + 2 * tig] = (wa + 1 < n1) ? e1 : -INFINITY;
+          } else if (tig == 0) {
+            swc[0] = (w0 - 1 < n1) ? e0 : -INFINITY;   // the halo window w0 - 1 (w0 >= 128 here)
+          }
+        }
+      }
+    }
+    __syncthreads();                           // sw[j & 1] complete
+    if (warp == 0) {
+      if (live && lane < kPieceBlk) {
+        // block 32p + lane takes windows 4(32p + lane) - 1 .. + 3 = swc[4 lane .. 4 lane + 4],
+        // where swc[0] (window w0 - 1) is the staged halo, the previous piece's
+        // last window, or none (p == 0)
+        const int blk = p * kPieceBlk + lane;
+        float m = halo ? swc[0] : (p == 0 ? -INFINITY : sw[(j + 1) & 1][kPieceWin]);
+        m = (lane == 0) ? m : swc[4 * lane];
+#pragma unroll
+        for (int q4 = 1; q4 < 5; ++q4) m = fmaxf(m, swc[4 * lane + q4]);
+        if (blk < nblk_cap) bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
+      }
+      if (seg_last(j)) {
+        // the segment's pieces are done: count them; the CTA that completes
+        // the last piece of (b, g) owes its selection
+        __threadfence();
+        __syncwarp();
+        if (lane == 0 && n1 >= 0) {
+          const unsigned done = static_cast<unsigned>(j - seg_start + 1);
+          const unsigned np = static_cast<unsigned>(live ? pnp[j] : 1);
+          if (atomicAdd(&cnt[bg], done) + done == np) owed[nowed++] = bg;
+        }
       }
     }
   }
-  // the last CTA of (b, g) to finish selects the blocks
-  __threadfence();
+  cp_async_wait0();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&cnt[bg], 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
+  const int no = nowed;
+  if (no == 0) return;
   __threadfence();
-  select_blocks_cta(bscore + static_cast<int64_t>(bg) * nblk_cap, t, n_init, n_local, top_k, n_sel, cand_cap,
-                    idx + static_cast<int64_t>(bg) * n_sel, sel_keys,
-                    reinterpret_cast<int*>(sc_smem + ((static_cast<size_t>(cand_cap) * 4 + 15) & ~size_t(15))), sel_sh);
+  for (int o = 0; o < no; ++o) {
+    const int bg = owed[o];
+    const int t = seq_len[bg / h_kv];
+    select_blocks_cta(bscore + static_cast<int64_t>(bg) * nblk_cap, t, n_init, n_local, top_k, n_sel, cand_cap,
+                      idx + static_cast<int64_t>(bg) * n_sel, reinterpret_cast<uint32_t*>(sc_smem),
+                      reinterpret_cast<int*>(sc_smem + ((static_cast<size_t>(cand_cap) * 4 + 15) & ~size_t(15))),
+                      sel_sh);
+    __syncthreads();                           // the scratch is reused by the next selection
+  }
 }
 
-constexpr int kAttWarps = 4;
+constexpr int kAttWarps = 6;
 constexpr int kChunkKeys = 32;
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -687,10 +809,9 @@ struct AttCfg {
   static constexpr int kRow = D + 8;                          // merge rows: D values, m, l, padding (bank spread)
   static constexpr int kPart = D + 4;                         // partial rows in HBM: D values, m, l, padding (16 B rows)
   static constexpr uint32_t kTile = kChunkKeys * D * 2;       // one K or V chunk
-  static constexpr uint32_t kSmem = kAttWarps * 2 * kTile;    // per-warp K and V buffers
+  static constexpr uint32_t kSmem = kAttWarps * 4 * kTile;    // per warp: two K and two V buffers
   static_assert(kAttWarps * 16 * kRow * 4 <= kSmem, "warp merge area fits in the staging buffers");
   static_assert(kMaxSplits * 16 * 4 * 2 <= kSmem, "split maxima and sums fit in the staging buffers");
-  static_assert(16 * (D / 4) <= 4 * 32 * kAttWarps, "four merge items per thread cover every (head, quad)");
 };
 
 // ---------------------------------------------------------------- K3: split-KV sparse attention + merge
@@ -706,15 +827,16 @@ struct AttCfg {
 //                                        then O and l are rescaled once)
 //   O[16, D] += P . V                  (P re-used from the S fragments,
 //                                        V via ldmatrix.trans)
-// The next chunk's K is issued as soon as S is done and its V as soon as
-// the PV product is done, so every warp keeps a copy in flight.  The warps'
+// Each warp holds two K and two V buffers: chunk i + 2's K is issued as soon
+// as chunk i's S is done and its V as soon as chunk i's PV product is done,
+// so every warp keeps two chunks' copies in flight.  The warps'
 // (m_ref, l, O) are merged in shared memory into one partial per CTA; the
 // last CTA of (b, g) to finish merges the partials, writes the output, and
 // the last group of b to finish advances seq_len[b].
 // Keys past t (and chunks of invalid or not yet visible blocks) are never
 // read: their staging rows are zero-filled and their scores are -inf.
 template <int D>
-__global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
+__global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
     const int32_t* __restrict__ idx, int32_t* seq_len, int capacity, int h_q, int h_kv, int n_sel, int bps,
     float scale, float* __restrict__ part, __nv_bfloat16* __restrict__ out, unsigned* __restrict__ cnt) {
@@ -735,8 +857,8 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
   const int nmine = (2 * nb > warp) ? (2 * nb - 1 - warp) / kAttWarps + 1 : 0;
   const int64_t kstride = static_cast<int64_t>(h_kv) * D;    // elements from one key row to the next
   const int64_t row0 = (static_cast<int64_t>(b) * capacity * h_kv + g) * D;
-  const uint32_t sK = smem_u32(att_smem) + warp * 2 * C::kTile;
-  const uint32_t sV = sK + C::kTile;
+  // the warp's buffers: K of chunks i and i + 1, then V of chunks i and i + 1
+  const uint32_t sbuf = smem_u32(att_smem) + warp * 4 * C::kTile;
 
   // Q of the group's 16 heads (rows >= G are zero) as m16n8k16 A fragments
   uint32_t qa[D / 16][4];
@@ -780,12 +902,20 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads gid, gid + 8: reference max, row sum
   const float cs = scale * kLog2e;
 
+  // copies in flight per warp: two chunks ahead.  Commit order: K0 V0 K1 V1,
+  // then per chunk i: K(i+2) after its S product, V(i+2) after its P.V
+  // product, so K(i) and V(i) each have exactly three younger groups.
   int k0 = chunk_key0(0);
-  stage(sK, kc, k0);
-  stage(sV, vc, k0);
+  int k1 = chunk_key0(1);
+  stage(sbuf, kc, k0);
+  stage(sbuf + 2 * C::kTile, vc, k0);
+  stage(sbuf + C::kTile, kc, k1);
+  stage(sbuf + 3 * C::kTile, vc, k1);
   for (int i = 0; i < nmine; ++i) {
-    const int k0n = chunk_key0(i + 1);
-    cp_async_wait1();                        // K of chunk i (its V may still be in flight)
+    const uint32_t sK = sbuf + (i & 1) * C::kTile;
+    const uint32_t sV = sK + 2 * C::kTile;
+    const int k0n = chunk_key0(i + 2);
+    cp_async_wait_n<3>();                    // K of chunk i
     __syncwarp();
     float s[4][4];
     if (k0 >= 0) {
@@ -852,7 +982,7 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
         }
       }
     }
-    cp_async_wait1();                        // V of chunk i (the next K may still be in flight)
+    cp_async_wait_n<3>();                    // V of chunk i
     __syncwarp();
     if (k0 >= 0) {
 #pragma unroll
@@ -872,7 +1002,8 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
     }
     __syncwarp();                            // every lane is done with this V buffer
     stage(sV, vc, k0n);
-    k0 = k0n;
+    k0 = k1;
+    k1 = k0n;
   }
   cp_async_wait0();
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -970,10 +1101,10 @@ __global__ void __launch_bounds__(32 * kAttWarps, 3) attend_kernel(
   }
   __syncthreads();
   // out[h, 4 q .. 4 q + 3] = sum over splits of weight * O: thread items
-  // it = tid + 128 k (k < 4) cover the G * D / 4 (head, quad) pairs; four
-  // splits of all four items are in flight at once
+  // it = tid + 32 kAttWarps k (k < kIt) cover the G * D / 4 (head, quad)
+  // pairs; four splits of every item are in flight at once
   {
-    constexpr int kIt = 4, kU = 4;
+    constexpr int kIt = (16 * (D / 4) + 32 * kAttWarps - 1) / (32 * kAttWarps), kU = 4;
     const int nitems = G * (D / 4);
     float4 acc[kIt];
 #pragma unroll
@@ -1092,7 +1223,7 @@ __global__ void __launch_bounds__(256) build_caches_kernel(const __nv_bfloat16* 
 
 // ---------------------------------------------------------------- host side
 struct DecodePlan {
-  int cap_c1, cap_c2, nblk_cap, cand_cap, nsplit2, nsplit1, nsplit, bps, n_sel;
+  int cap_c1, cap_c2, nblk_cap, cand_cap, nsplit2, np_cap, nsplit, bps, n_sel, sms, nbg;
   size_t off_part2, off_bscore, off_idx, off_part, off_cnt, bytes;
 };
 
@@ -1100,7 +1231,9 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Largest capacity whose candidate keys fit the selecting CTA's shared memory
 // next to the two staging buffers of the score kernel.
-static bool decode_plan_supported(const DecodePlan& p) { return static_cast<size_t>(p.cand_cap) * 4 <= 88 * 1024; }
+static bool decode_plan_supported(const DecodePlan& p) {
+  return static_cast<size_t>(p.cand_cap) * 4 <= 88 * 1024 && p.nbg <= 65535 && p.np_cap <= 65535;
+}
 
 DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_sel, int sms) {
   DecodePlan p{};
@@ -1110,11 +1243,13 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   p.nblk_cap = (capacity + 63) / 64;
   p.cand_cap = (p.nblk_cap + 31) & ~31;
   p.nsplit2 = std::max(1, (p.cap_c2 + dec::kLseWin - 1) / dec::kLseWin);
-  p.nsplit1 = std::max(1, (p.cap_c1 + dec::kScoreWin) / dec::kScoreWin);
+  p.np_cap = std::max(1, (p.nblk_cap + dec::kPieceBlk - 1) / dec::kPieceBlk);
+  p.sms = std::max(1, sms);
   const int bg = batch * h_kv;
-  // attention splits: about 1.5 attention CTAs per SM (16 x 131072 decode:
-  // 6 splits of 16 blocks; 3 per SM and 1 per SM were both slower)
-  const int per_bg = std::min(dec::kMaxSplits, std::max(1, (3 * sms) / 2 / std::max(1, bg)));
+  p.nbg = bg;
+  // attention splits: one wave of one CTA per SM (its shared memory holds
+  // two chunks ahead per warp); 16 x 131072 decode: 4 splits of 24 blocks
+  const int per_bg = std::min(dec::kMaxSplits, std::max(1, sms / std::max(1, bg)));
   p.bps = std::max(1, (n_sel + per_bg - 1) / per_bg);
   p.nsplit = std::max(1, (n_sel + p.bps - 1) / p.bps);
   const int G = h_q / h_kv;
@@ -1144,14 +1279,22 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
       static_cast<const bf*>(q), static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
       static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache), static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2),
       s->seq_len, s->capacity, s->h_q, s->h_kv, P.cap_c1, P.cap_c2, scale, part2, cnt);
-  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kBuf,
+  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kRing,
                                           static_cast<size_t>(P.cand_cap) * 4 + 16 + dec::kSelBins * 4);
   cudaError_t e = cudaFuncSetAttribute(dec::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(k2_smem));
   if (e != cudaSuccess) return e;
-  dec::score_select_kernel<D><<<dim3(P.nsplit1, bg), dec::kSelThreads, k2_smem, st>>>(
-      static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->capacity, s->h_q,
-      s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt);
+  // one wave of streaming CTAs, each with at most kMaxRange pieces
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dec::score_select_kernel<D>, dec::kSelThreads, k2_smem);
+  if (e != cudaSuccess) return e;
+  const int64_t p_cap = static_cast<int64_t>(bg) * P.np_cap;
+  int64_t grid2 = std::min<int64_t>(p_cap, static_cast<int64_t>(std::max(1, occ)) * P.sms);
+  grid2 = std::max<int64_t>(grid2, (p_cap + dec::kMaxRange - 1) / dec::kMaxRange);
+  dec::score_select_kernel<D><<<static_cast<unsigned>(grid2), dec::kSelThreads, k2_smem, st>>>(
+      static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->batch,
+      s->capacity, s->h_q, s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel,
+      bscore, idx, cnt);
   e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(dec::AttCfg<D>::kSmem));
   if (e != cudaSuccess) return e;
