@@ -517,23 +517,30 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
 // a grid of short-lived CTAs.
 // Per window: the 16 heads' scores, normalised by their LSE and summed over
 // the group ([top168] §三 second stage, §四); per block i: the max over
-// windows 4i-1 .. 4i+3.  The window before a piece (the first block's halo)
-// is the previous piece's last window when the range holds that piece, else
-// an extra staged row.  The 16-byte pieces of a staged row are XOR-swizzled
-// by the row's parity, so the fragment loads are free of bank conflicts.
+// windows 4i-1 .. 4i+3.  A stage is one TMA box of kPieceRows rows starting
+// 8 windows before the piece (zeros before window 0): its first n-tile holds
+// the window before the piece (the first block's halo), which is scored only
+// when the range does not hold the previous piece (else that piece's last
+// window is carried over).  The box is 128-byte swizzled (16-byte chunk c of
+// row r at chunk c ^ (r & 7)); lane group gid of an n-tile reads row
+// (gid >> 1) | ((gid & 1) << 2), so the two rows of each 8-lane phase of a
+// fragment load differ in swizzle bit 2 and the loads are free of bank
+// conflicts.
 // A completion counter per (b, g) counts the pieces done; the CTA that
 // completes the last one runs that selection once its range is done.
 constexpr int kPieceWin = 128;                  // stage-1 windows per piece
 constexpr int kPieceBlk = kPieceWin / 4;        // blocks per piece
-constexpr int kPieceRows = kPieceWin + 8;       // + one n-tile whose first row is the halo window
+constexpr int kPieceRows = kPieceWin + 8;       // the n-tile before the piece, then the piece
 constexpr int kScoreStages = 2;
 constexpr int kMaxRange = 64;                   // pieces per CTA at most (the host sizes the grid)
 
 template <int D>
 struct ScoreCfg {
-  static constexpr int CH = D / 8;                                  // 16-byte pieces per row
-  static constexpr uint32_t kStage = kPieceRows * D * 2;
+  static constexpr uint32_t kHalf = kPieceRows * 128;               // one 64-column box (1024-byte multiple)
+  static constexpr uint32_t kStage = kPieceRows * D * 2;            // D / 64 boxes
   static constexpr uint32_t kRing = kScoreStages * kStage;
+  static constexpr uint32_t kSmem = kRing + 1024;                   // + alignment of the swizzled boxes
+  static_assert(kHalf % 1024 == 0, "128-byte swizzled boxes start on 1024-byte boundaries");
 };
 
 // Pieces of a (sequence, group) whose new token is at t: its scored blocks
@@ -550,12 +557,15 @@ __device__ __forceinline__ int score_pieces(int t, int capacity, int n_init, int
 
 template <int D>
 __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
+    const __grid_constant__ CUtensorMap tmK1, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
     const float2* __restrict__ part2, int nsplit2, int batch, int capacity, int h_q, int h_kv, int cap_c1,
     int nblk_cap, int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel,
     float* __restrict__ bscore, int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
   using C = ScoreCfg<D>;
   extern __shared__ __align__(128) uint8_t sc_smem[];   // the ring; the selection's keys and bins reuse it
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sc_smem) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kScoreStages];
   __shared__ uint32_t plist[kMaxRange];                // bg << 16 | piece index within (b, g)
   __shared__ int pn1[kMaxRange];                       // visible stage-1 windows; -1: t out of range
   __shared__ int pnp[kMaxRange];                       // pieces of the piece's (b, g); 0: not scored
@@ -615,7 +625,11 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
       base += tot;
       if (base >= P1) break;                   // uniform: base and P1 are the same in every thread
     }
-    if (tid == 0) nowed = 0;
+    if (tid == 0) {
+      nowed = 0;
+      for (int st = 0; st < kScoreStages; ++st) mbar_init(&full_bar[st], 1);
+      fence_barrier_init();
+    }
     __syncthreads();
   }
   if (R == 0) return;
@@ -624,25 +638,18 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
   auto seg_first = [&](int j) { return j == 0 || bg_of(j - 1) != bg_of(j); };
   auto seg_last = [&](int j) { return j == R - 1 || bg_of(j + 1) != bg_of(j); };
 
-  // stage piece j (rows past the visible windows zero-filled; the halo row
-  // only for the first piece of a range segment)
+  // stage piece j: one box per 64 columns, windows w0 - 8 .. w0 + 127 (rows
+  // outside the pooled cache read as zeros; rows of windows not yet visible
+  // are masked below)
   auto stage = [&](int j) {
-    if (j < R && pnp[j] > 0) {
-      const int bg = bg_of(j), p = p_of(j), n1 = pn1[j];
-      const int w0 = p * kPieceWin;
-      const bool halo = seg_first(j) && p > 0;
-      const __nv_bfloat16* base = kc1 + static_cast<int64_t>(bg) * cap_c1 * D;
-      const uint32_t dst0 = smem_u32(sc_smem) + (j % kScoreStages) * C::kStage;
-      const int nrows = halo ? kPieceRows : kPieceWin;
-      for (int pc = tid; pc < nrows * C::CH; pc += kSelThreads) {
-        const int r = pc / C::CH, piece = pc - r * C::CH;
-        const int wr = (r < kPieceWin) ? w0 + r : (r == kPieceWin ? w0 - 1 : -1);
-        const bool ok = wr >= 0 && wr < n1;
-        const __nv_bfloat16* src = base + (ok ? static_cast<int64_t>(wr) * D + piece * 8 : 0);
-        cp_async16(dst0 + r * (D * 2) + ((piece ^ ((r & 1) << 2)) << 4), src, ok);
-      }
+    if (tid == 0 && j < R && pnp[j] > 0) {
+      const int st = j % kScoreStages;
+      mbar_arrive_expect_tx(&full_bar[st], C::kStage);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tma_load_3d(ring + st * C::kStage + h * C::kHalf, &tmK1, &full_bar[st], 64 * h, p_of(j) * kPieceWin - 8,
+                    bg_of(j));
     }
-    cp_async_commit();
   };
   // the group's negated log-sum-exp per head (log2 units) from the coarse
   // partials: thread (h, k0) folds partials k0, k0 + 16, ..., then the 16
@@ -704,9 +711,9 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     load_qfrag<D>(f, q + (static_cast<int64_t>(b) * h_q + g * G) * D, lane, G);
   }
   int seg_start = 0;
+  uint32_t phase = 0;                          // bit s: parity of stage s's next fill
   for (int j = 0; j < R; ++j) {
-    cp_async_wait_n<kScoreStages - 2>();
-    __syncthreads();                           // piece j landed; stage (j - 1) % S and sw[(j + 1) & 1] are free
+    __syncthreads();                           // stage (j - 1) % S and sw[(j + 1) & 1] are free
     stage(j + kScoreStages - 1);
     const int bg = bg_of(j), p = p_of(j), n1 = pn1[j];
     const bool live = pnp[j] > 0;
@@ -723,15 +730,22 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     const bool halo = seg_first(j) && p > 0;
     float* swc = sw[j & 1];
     if (live) {
+      const int st = j % kScoreStages;
+      mbar_wait(&full_bar[st], (phase >> st) & 1u);
+      phase ^= 1u << st;
       const float nl0 = nlse[gid], nl1 = nlse[gid + 8];
-      const uint8_t* rows = sc_smem + (j % kScoreStages) * C::kStage;
+      const uint8_t* rows = ring + st * C::kStage;
       const int ntiles = halo ? kPieceWin / 8 + 1 : kPieceWin / 8;
-      for (int nt = warp; nt < ntiles; nt += kSelThreads / 32) {
-        const int r = nt * 8 + gid;
-        const uint4* rowp = reinterpret_cast<const uint4*>(rows + r * (D * 2));
+      for (int i = warp; i < ntiles; i += kSelThreads / 32) {
+        // the piece's n-tiles are box n-tiles 1 .. 16; the halo n-tile (box n-tile 0) comes last
+        const int r = (i < kPieceWin / 8 ? 8 * (i + 1) : 0) + ((gid >> 1) | ((gid & 1) << 2));
         uint4 kv[D / 32];
 #pragma unroll
-        for (int pp = 0; pp < D / 32; ++pp) kv[pp] = rowp[(4 * pp + tig) ^ ((r & 1) << 2)];
+        for (int pp = 0; pp < D / 32; ++pp) {
+          const int ch = 4 * pp + tig;         // 16-byte chunk of the row: box ch >> 3, chunk ch & 7
+          kv[pp] = *reinterpret_cast<const uint4*>(rows + (ch >> 3) * C::kHalf + r * 128 +
+                                                   (((ch & 7) ^ (r & 7)) << 4));
+        }
         float sc[4];
         scores_16x8_reg<D>(sc, f, kv);
         // head-group sum for windows 2tig and 2tig+1 of the n-tile: two heads here, the other 14 on the lanes with the same tig
@@ -742,13 +756,14 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
           e0 += __shfl_xor_sync(0xffffffffu, e0, o);
           e1 += __shfl_xor_sync(0xffffffffu, e1, o);
         }
+        // columns 2tig, 2tig + 1 are rows tig, tig + 4 of the n-tile
         if (gid == 0) {
-          if (nt < kPieceWin / 8) {
-            const int wa = w0 + nt * 8 + 2 * tig;
-            swc[1 + nt * 8 + 2 * tig] = (wa < n1) ? e0 : -INFINITY;
-            swc[2 + nt * 8 + 2 * tig] = (wa + 1 < n1) ? e1 : -INFINITY;
-          } else if (tig == 0) {
-            swc[0] = (w0 - 1 < n1) ? e0 : -INFINITY;   // the halo window w0 - 1 (w0 >= 128 here)
+          if (i < kPieceWin / 8) {
+            const int wa = w0 + 8 * i + tig;
+            swc[1 + 8 * i + tig] = (wa < n1) ? e0 : -INFINITY;
+            swc[5 + 8 * i + tig] = (wa + 4 < n1) ? e1 : -INFINITY;
+          } else if (tig == 3) {
+            swc[0] = (w0 - 1 < n1) ? e1 : -INFINITY;   // row 7: the halo window w0 - 1 (w0 >= 128 here)
           }
         }
       }
@@ -779,8 +794,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
       }
     }
   }
-  cp_async_wait0();
-  __syncthreads();
+  __syncthreads();                             // every fill was consumed: the ring is free
   const int no = nowed;
   if (no == 0) return;
   __threadfence();
@@ -1279,7 +1293,15 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
       static_cast<const bf*>(q), static_cast<const bf*>(k_new), static_cast<const bf*>(v_new),
       static_cast<bf*>(s->k_cache), static_cast<bf*>(s->v_cache), static_cast<bf*>(s->k_c1), static_cast<bf*>(s->k_c2),
       s->seq_len, s->capacity, s->h_q, s->h_kv, P.cap_c1, P.cap_c2, scale, part2, cnt);
-  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kRing,
+  CUtensorMap mK1;
+  {
+    const uint64_t rows = static_cast<uint64_t>(std::max(1, P.cap_c1));
+    const uint64_t dims[3] = {(uint64_t)D, rows, (uint64_t)bg};
+    const uint64_t strides[2] = {(uint64_t)D * 2, rows * D * 2};
+    const uint32_t box[3] = {64, (uint32_t)dec::kPieceRows, 1};
+    if (!make_tmap(&mK1, s->k_c1, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const size_t k2_smem = std::max<size_t>(dec::ScoreCfg<D>::kSmem,
                                           static_cast<size_t>(P.cand_cap) * 4 + 16 + dec::kSelBins * 4);
   cudaError_t e = cudaFuncSetAttribute(dec::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(k2_smem));
@@ -1292,7 +1314,7 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
   int64_t grid2 = std::min<int64_t>(p_cap, static_cast<int64_t>(std::max(1, occ)) * P.sms);
   grid2 = std::max<int64_t>(grid2, (p_cap + dec::kMaxRange - 1) / dec::kMaxRange);
   dec::score_select_kernel<D><<<static_cast<unsigned>(grid2), dec::kSelThreads, k2_smem, st>>>(
-      static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->batch,
+      mK1, static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->batch,
       s->capacity, s->h_q, s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel,
       bscore, idx, cnt);
   e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
