@@ -482,23 +482,37 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
     __syncthreads();                            // hist, digit and above are rewritten by the next pass
   }
   const uint32_t T = kmin + prefix;             // the top_k-th largest key; k_rem keys equal to it are taken
-  // one ordered pass: thread tid owns candidates [tid*per, tid*per + per)
-  const int per = (ncand + kSelThreads - 1) / kSelThreads;
+  // one ordered pass: thread tid owns candidates [tid*per, tid*per + per),
+  // per a multiple of 4 so they load as 16-byte vectors; one scan of the
+  // packed counts (greater in the low 16 bits, equal in the high) gives each
+  // thread its output position and its share of the equal keys
+  const int per = ((ncand + 4 * kSelThreads - 1) / (4 * kSelThreads)) * 4;
   const int c0 = min(ncand, tid * per), c1 = min(ncand, c0 + per);
   int n_gt = 0, n_eq = 0;
-  for (int i = c0; i < c1; ++i) {
-    n_gt += keys[i] > T;
-    n_eq += keys[i] == T;
+  for (int i = c0; i < c1; i += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
+    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      n_gt += (i + u < c1) && kk[u] > T;
+      n_eq += (i + u < c1) && kk[u] == T;
+    }
   }
   int tot;
-  const int eq_before = cta_exclusive_scan(n_eq, sh.wsum, &tot);
+  const int before = cta_exclusive_scan(n_gt | (n_eq << 16), sh.wsum, &tot);
+  const int gt_before = before & 0xffff, eq_before = before >> 16;
   const int eq_take = max(0, min(n_eq, k_rem - eq_before));
-  const int pos0 = cta_exclusive_scan(n_gt + eq_take, sh.wsum, &tot);
-  int pos = init_hi + pos0, eq_seen = 0;
-  for (int i = c0; i < c1; ++i) {
-    const uint32_t k = keys[i];
-    const bool take = (k > T) || (k == T && eq_seen++ < eq_take);
-    if (take) out[pos++] = init_hi + i;
+  int pos = init_hi + gt_before + min(eq_before, k_rem), eq_seen = 0;
+  for (int i = c0; i < c1; i += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
+    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (i + u < c1) {
+        const bool take = (kk[u] > T) || (kk[u] == T && eq_seen++ < eq_take);
+        if (take) out[pos++] = init_hi + i + u;
+      }
+    }
   }
   for (int i = tid; i < init_hi; i += kSelThreads) out[i] = i;
   const int nloc = b_t - loc_lo + 1;
@@ -579,51 +593,77 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
   const int gid = lane >> 2, tig = lane & 3;
   const float cs = scale * kLog2e;
 
-  // ---- this CTA's range [P0, P1) of the flattened piece list
+  // ---- this CTA's pieces.  With at least one CTA per (b, g), (b, g) gets
+  // np(b) * (n - nbg) / total + 1 CTAs (at most n in all), each a contiguous
+  // share of its pieces, so no CTA switches groups; otherwise the flattened
+  // list of all pieces is cut into n contiguous ranges.
+  __shared__ int s_R;
   int R = 0;
   {
-    int total = -1;                            // known after one pass when the batch fits one scan
-    if (batch > kSelThreads) {
-      total = 0;
-      for (int b0 = 0; b0 < batch; b0 += kSelThreads) {
-        const int b = b0 + tid;
-        const int v = (b < batch) ? h_kv * score_pieces(seq_len[b], capacity, n_init, n_local, top_k) : 0;
-        int tot;
-        cta_exclusive_scan(v, sel_sh.wsum, &tot);
-        total += tot;
+    const int n = gridDim.x, nbg = batch * h_kv;
+    const bool aligned = n >= nbg;
+    if (tid == 0) s_R = 0;
+    int total = 0;
+    for (int b0 = 0; b0 < batch; b0 += kSelThreads) {
+      const int b = b0 + tid;
+      const int v = (b < batch) ? h_kv * score_pieces(seq_len[b], capacity, n_init, n_local, top_k) : 0;
+      int tot;
+      cta_exclusive_scan(v, sel_sh.wsum, &tot);
+      total += tot;
+    }
+    const int64_t P0 = static_cast<int64_t>(total) * blockIdx.x / n;
+    const int64_t P1 = static_cast<int64_t>(total) * (blockIdx.x + 1) / n;
+    if (!aligned) {
+      R = static_cast<int>(P1 - P0);
+      if (R > kMaxRange) {                     // the host sizes the grid so that this cannot happen
+        if (tid == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+        return;
       }
     }
-    int base = 0;
+    int base = 0;                              // aligned: CTAs before sequence b; else pieces before it
     for (int b0 = 0; b0 < batch; b0 += kSelThreads) {
       const int b = b0 + tid;
       const int tb = (b < batch) ? seq_len[b] : -1;
       const int np = (b < batch) ? score_pieces(tb, capacity, n_init, n_local, top_k) : 0;
+      const int cg = (b < batch) ? static_cast<int>(static_cast<int64_t>(np) * (n - nbg) / total) + 1 : 0;
       int tot;
-      const int ex = cta_exclusive_scan(h_kv * np, sel_sh.wsum, &tot);
-      if (total < 0) total = tot;
-      const int64_t P0 = static_cast<int64_t>(total) * blockIdx.x / gridDim.x;
-      const int64_t P1 = static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x;
-      R = static_cast<int>(P1 - P0);
-      if (R > kMaxRange) {                     // the host sizes the grid so that this cannot happen
-        if (tid == 0 && b0 == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
-        return;
-      }
-      // pieces [base + ex, base + ex + h_kv * np) belong to sequence b
+      const int ex = cta_exclusive_scan(h_kv * (aligned ? cg : np), sel_sh.wsum, &tot);
       const bool valid = tb >= 0 && tb < capacity;
       const int n1 = valid ? min(visible_windows_dev(tb, 32, 16), cap_c1) : -1;
       const bool sc = valid && needs_scores(tb, n_init, n_local, top_k);
-      const int64_t lo = max(static_cast<int64_t>(base) + ex, P0);
-      const int64_t hi = min(static_cast<int64_t>(base) + ex + h_kv * np, P1);
-      for (int64_t i = lo; i < hi; ++i) {
-        const int rem = static_cast<int>(i - base - ex);
-        const int g = rem / np, p = rem - g * np;
-        const int j = static_cast<int>(i - P0);
-        plist[j] = (static_cast<uint32_t>(b * h_kv + g) << 16) | static_cast<uint32_t>(p);
-        pn1[j] = n1;
-        pnp[j] = sc ? np : 0;
+      if (aligned) {
+        // CTAs [base + ex, base + ex + h_kv * cg) belong to sequence b
+        const int i = static_cast<int>(blockIdx.x) - (base + ex);
+        if (b < batch && i >= 0 && i < h_kv * cg) {
+          const int g = i / cg, u = i - g * cg;
+          const int p0 = np * u / cg, p1 = np * (u + 1) / cg;
+          if (p1 - p0 > kMaxRange) {           // the host sizes the grid so that this cannot happen
+            record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+            s_R = -1;
+          } else {
+            for (int j = 0; j < p1 - p0; ++j) {
+              plist[j] = (static_cast<uint32_t>(b * h_kv + g) << 16) | static_cast<uint32_t>(p0 + j);
+              pn1[j] = n1;
+              pnp[j] = sc ? np : 0;
+            }
+            s_R = p1 - p0;
+          }
+        }
+      } else {
+        // pieces [base + ex, base + ex + h_kv * np) belong to sequence b
+        const int64_t lo = max(static_cast<int64_t>(base) + ex, P0);
+        const int64_t hi = min(static_cast<int64_t>(base) + ex + h_kv * np, P1);
+        for (int64_t i = lo; i < hi; ++i) {
+          const int rem = static_cast<int>(i - base - ex);
+          const int g = rem / np, p = rem - g * np;
+          const int j = static_cast<int>(i - P0);
+          plist[j] = (static_cast<uint32_t>(b * h_kv + g) << 16) | static_cast<uint32_t>(p);
+          pn1[j] = n1;
+          pnp[j] = sc ? np : 0;
+        }
       }
       base += tot;
-      if (base >= P1) break;                   // uniform: base and P1 are the same in every thread
+      if (!aligned && base >= P1) break;      // uniform: base and P1 are the same in every thread
     }
     if (tid == 0) {
       nowed = 0;
@@ -631,6 +671,8 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
       fence_barrier_init();
     }
     __syncthreads();
+    if (aligned) R = s_R;
+    if (R < 0) return;
   }
   if (R == 0) return;
   auto bg_of = [&](int j) { return static_cast<int>(plist[j] >> 16); };
@@ -1312,7 +1354,11 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
   if (e != cudaSuccess) return e;
   const int64_t p_cap = static_cast<int64_t>(bg) * P.np_cap;
   int64_t grid2 = std::min<int64_t>(p_cap, static_cast<int64_t>(std::max(1, occ)) * P.sms);
+  // flattened ranges hold at most ceil(total / grid) pieces; group-aligned
+  // shares (the kernel's choice when grid >= groups) at most
+  // total / (grid - groups) + 1
   grid2 = std::max<int64_t>(grid2, (p_cap + dec::kMaxRange - 1) / dec::kMaxRange);
+  if (grid2 >= bg) grid2 = std::max<int64_t>(grid2, bg + (p_cap + dec::kMaxRange - 2) / (dec::kMaxRange - 1));
   dec::score_select_kernel<D><<<static_cast<unsigned>(grid2), dec::kSelThreads, k2_smem, st>>>(
       mK1, static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->batch,
       s->capacity, s->h_q, s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel,
