@@ -124,6 +124,47 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr)
                : "memory");
 }
+// ---------------------------------------------------------------- programmatic dependent launch
+// The three kernels of a step are chained with programmatic stream
+// serialization: a kernel lets its dependent launch as soon as all of its
+// CTAs have started, and the dependent does its setup (which reads nothing
+// the primary writes) before waiting for the primary grid to complete.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA of the cluster: writes before are visible to reads after
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// the address of this CTA's shared-memory word `local` in the CTA of the cluster with rank `rank`
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+// (volatile: kept in order with the cluster barriers; no memory clobber, so
+// loads of independent items can be in flight together)
+__device__ __forceinline__ float ld_dsmem(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float4 ld_dsmem4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a));
+  return v;
+}
+
 // ---------------------------------------------------------------- pooling of the window that ends at t
 // Window [t - len + 1, t] of kv group g: rows before t from the cache, row t
 // from k_new (it may not be in the cache yet).  Exact mean in fp64, one bf16
@@ -138,6 +179,7 @@ __device__ void pool_window(int len, const __nv_bfloat16* kc, int64_t seq0, int 
   double acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+#pragma unroll 4
   for (int r = rg; r < len; r += NRG) {
     const int u = t - len + 1 + r;
     const __nv_bfloat16* src = (u == t) ? kn : kc + ((seq0 + u) * h_kv + g) * D;
@@ -196,6 +238,7 @@ __global__ void __launch_bounds__(128) lse_append_kernel(
   const int G = h_q / h_kv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
+  griddep_launch_dependents();
   if (c == 0 && threadIdx.x == 0) {
     cnt[bg] = 0u;
     cnt[nbg + bg] = 0u;
@@ -598,6 +641,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
   // share of its pieces, so no CTA switches groups; otherwise the flattened
   // list of all pieces is cut into n contiguous ranges.
   __shared__ int s_R;
+  griddep_launch_dependents();
   int R = 0;
   {
     const int n = gridDim.x, nbg = batch * h_kv;
@@ -672,9 +716,10 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     }
     __syncthreads();
     if (aligned) R = s_R;
-    if (R < 0) return;
   }
-  if (R == 0) return;
+  // the mapping read only seq_len; the pooled keys and the LSE partials come from the append kernel
+  griddep_wait();
+  if (R <= 0) return;
   auto bg_of = [&](int j) { return static_cast<int>(plist[j] >> 16); };
   auto p_of = [&](int j) { return static_cast<int>(plist[j] & 0xffffu); };
   auto seg_first = [&](int j) { return j == 0 || bg_of(j - 1) != bg_of(j); };
@@ -868,6 +913,7 @@ struct AttCfg {
   static constexpr uint32_t kSmem = kAttWarps * 4 * kTile;    // per warp: two K and two V buffers
   static_assert(kAttWarps * 16 * kRow * 4 <= kSmem, "warp merge area fits in the staging buffers");
   static_assert(kMaxSplits * 16 * 4 * 2 <= kSmem, "split maxima and sums fit in the staging buffers");
+  static_assert((kAttWarps * 16 * kRow + 16 * kPart) * 4 <= kSmem, "the warp rows and the CTA partial fit");
 };
 
 // ---------------------------------------------------------------- K3: split-KV sparse attention + merge
@@ -886,12 +932,17 @@ struct AttCfg {
 // Each warp holds two K and two V buffers: chunk i + 2's K is issued as soon
 // as chunk i's S is done and its V as soon as chunk i's PV product is done,
 // so every warp keeps two chunks' copies in flight.  The warps'
-// (m_ref, l, O) are merged in shared memory into one partial per CTA; the
-// last CTA of (b, g) to finish merges the partials, writes the output, and
-// the last group of b to finish advances seq_len[b].
+// (m_ref, l, O) are merged in shared memory into one partial per CTA.  With
+// CLUSTER the nsplit CTAs of (b, g) form one thread-block cluster: each keeps
+// its partial in its shared memory and, after a cluster barrier, rank 0 reads
+// them all through distributed shared memory, merges them and writes the
+// output (a second barrier keeps the partials alive until it is done).
+// Otherwise each CTA writes its partial to the workspace and the last CTA of
+// (b, g) to finish (a completion counter) merges them.  The merging CTA of the
+// last group of b to finish advances seq_len[b].
 // Keys past t (and chunks of invalid or not yet visible blocks) are never
 // read: their staging rows are zero-filled and their scores are -inf.
-template <int D>
+template <int D, bool CLUSTER>
 __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
     const int32_t* __restrict__ idx, int32_t* seq_len, int capacity, int h_q, int h_kv, int n_sel, int bps,
@@ -907,7 +958,6 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
   const int gid = lane >> 2, tig = lane & 3;
   // the new token's position; keys 0..t are visible
   const int t = seq_len[b];
-  if (t < 0 || t >= capacity) return;          // recorded by the append kernel
   const int32_t* list = idx + static_cast<int64_t>(bg) * n_sel + static_cast<int64_t>(sp) * bps;
   const int nb = max(0, min(bps, n_sel - sp * bps));
   const int nmine = (2 * nb > warp) ? (2 * nb - 1 - warp) / kAttWarps + 1 : 0;
@@ -929,6 +979,9 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
       qa[kk][3] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qh + (gid + 8) * D + d0 + 8) : 0u;
     }
   }
+  // the block lists come from the score kernel
+  griddep_wait();
+  if (t < 0 || t >= capacity) return;          // recorded by the append kernel
 
   // first key of the warp's i-th chunk, or -1 when it has no visible key
   auto chunk_key0 = [&](int i) -> int {
@@ -1103,6 +1156,88 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
     s_L[h] = L;
   }
   __syncthreads();
+  if constexpr (CLUSTER) {
+    float* mine = reinterpret_cast<float*>(att_smem) + kAttWarps * 16 * C::kRow;   // [G][kPart], after the warp rows
+    for (int e = threadIdx.x; e < G * D; e += 32 * kAttWarps) {
+      const int h = e / D, d = e % D;
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kAttWarps; ++w) acc += s_wgt[w][h] * mw[(w * 16 + h) * C::kRow + d];
+      mine[h * C::kPart + d] = acc;
+    }
+    if (threadIdx.x < G) {
+      mine[threadIdx.x * C::kPart + D] = s_M[threadIdx.x];
+      mine[threadIdx.x * C::kPart + D + 1] = s_L[threadIdx.x];
+    }
+    cluster_sync_all();
+    if (cluster_rank() == 0) {
+      const uint32_t mine_s = smem_u32(mine);
+      __shared__ float s_cw[8][16];            // split weights
+      if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float ms[8], ls[8];
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2) {
+          if (s2 < nsplit) {
+            const uint32_t a = dsmem_addr(mine_s + (h * C::kPart + D) * 4, s2);
+            ms[s2] = ld_dsmem(a);
+            ls[s2] = ld_dsmem(a + 4);
+            M = fmaxf(M, ms[s2]);
+          }
+        }
+        float L = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < nsplit && ms[s2] != -INFINITY) L += ex2(ms[s2] - M) * ls[s2];
+        const float inv = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < nsplit) s_cw[s2][h] = (ms[s2] == -INFINITY) ? 0.f : ex2(ms[s2] - M) * inv;
+      }
+      __syncthreads();
+      constexpr int kIt = (16 * (D / 4) + 32 * kAttWarps - 1) / (32 * kAttWarps);
+      const int nitems = G * (D / 4);
+      // every item's loads first, so they are all in flight together
+      float4 v[kIt][8];
+#pragma unroll
+      for (int k = 0; k < kIt; ++k) {
+        const int it = min(threadIdx.x + 32 * kAttWarps * k, nitems - 1);
+        const int h = it / (D / 4), q4 = it % (D / 4);
+        const uint32_t local = mine_s + (h * C::kPart + 4 * q4) * 4;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < nsplit) v[k][s2] = ld_dsmem4(dsmem_addr(local, s2));
+      }
+#pragma unroll
+      for (int k = 0; k < kIt; ++k) {
+        const int it = threadIdx.x + 32 * kAttWarps * k;
+        if (it < nitems) {
+          const int h = it / (D / 4), q4 = it % (D / 4);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2) {
+            if (s2 < nsplit) {
+              const float wg = s_cw[s2][h];
+              acc.x = fmaf(wg, v[k][s2].x, acc.x);
+              acc.y = fmaf(wg, v[k][s2].y, acc.y);
+              acc.z = fmaf(wg, v[k][s2].z, acc.z);
+              acc.w = fmaf(wg, v[k][s2].w, acc.w);
+            }
+          }
+          uint2 w2;
+          w2.x = pack_bf16(acc.x, acc.y);
+          w2.y = pack_bf16(acc.z, acc.w);
+          *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b) * h_q + g * G + h) * D + 4 * q4) = w2;
+        }
+      }
+      // every CTA of every group of b has read seq_len[b] once all groups got here
+      if (threadIdx.x == 0 && atomicAdd(&cnt[2 * nbg + b], 1u) == static_cast<unsigned>(h_kv) - 1)
+        seq_len[b] = t + 1;
+    }
+    cluster_sync_all();                        // the partials stay readable until rank 0 is done
+    return;
+  }
   float* pb = part + static_cast<int64_t>(bg) * nsplit * G * C::kPart;
   {
     float* dst = pb + static_cast<int64_t>(sp) * G * C::kPart;
@@ -1359,16 +1494,63 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
   // total / (grid - groups) + 1
   grid2 = std::max<int64_t>(grid2, (p_cap + dec::kMaxRange - 1) / dec::kMaxRange);
   if (grid2 >= bg) grid2 = std::max<int64_t>(grid2, bg + (p_cap + dec::kMaxRange - 2) / (dec::kMaxRange - 1));
-  dec::score_select_kernel<D><<<static_cast<unsigned>(grid2), dec::kSelThreads, k2_smem, st>>>(
-      mK1, static_cast<const bf*>(q), static_cast<const bf*>(s->k_c1), s->seq_len, part2, P.nsplit2, s->batch,
-      s->capacity, s->h_q, s->h_kv, P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel,
-      bscore, idx, cnt);
-  e = cudaFuncSetAttribute(dec::attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(dec::AttCfg<D>::kSmem));
-  if (e != cudaSuccess) return e;
-  dec::attend_kernel<D><<<dim3(bg, P.nsplit), 32 * dec::kAttWarps, dec::AttCfg<D>::kSmem, st>>>(
-      static_cast<const bf*>(q), static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache), idx,
-      s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps, scale, part, static_cast<bf*>(out), cnt);
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid2));
+    cfg.blockDim = dim3(dec::kSelThreads);
+    cfg.dynamicSmemBytes = k2_smem;
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dec::score_select_kernel<D>, mK1, static_cast<const bf*>(q),
+                           static_cast<const bf*>(s->k_c1), static_cast<const int32_t*>(s->seq_len),
+                           static_cast<const float2*>(part2), P.nsplit2, s->batch, s->capacity, s->h_q, s->h_kv,
+                           P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt);
+    if (e != cudaSuccess) return e;
+  }
+  if (P.nsplit <= 8) {
+    // the splits of (b, g) as one cluster: the merge goes through distributed shared memory
+    e = cudaFuncSetAttribute(dec::attend_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(dec::AttCfg<D>::kSmem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(bg, P.nsplit);
+    cfg.blockDim = dim3(32 * dec::kAttWarps);
+    cfg.dynamicSmemBytes = dec::AttCfg<D>::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = P.nsplit;
+    attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl[0];
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, dec::attend_kernel<D, true>, static_cast<const bf*>(q),
+                           static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache),
+                           static_cast<const int32_t*>(idx), s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps,
+                           scale, part, static_cast<bf*>(out), cnt);
+    if (e != cudaSuccess) return e;
+  } else {
+    e = cudaFuncSetAttribute(dec::attend_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(dec::AttCfg<D>::kSmem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(bg, P.nsplit);
+    cfg.blockDim = dim3(32 * dec::kAttWarps);
+    cfg.dynamicSmemBytes = dec::AttCfg<D>::kSmem;
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dec::attend_kernel<D, false>, static_cast<const bf*>(q),
+                           static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache),
+                           static_cast<const int32_t*>(idx), s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps,
+                           scale, part, static_cast<bf*>(out), cnt);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 
