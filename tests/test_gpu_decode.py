@@ -117,6 +117,14 @@ def test_decode_group_sizes():
     _run_case(w, prefix=2000, steps=20, batch=2, check_every=4)
 
 
+def test_decode_many_groups():
+    # 120 sequences x 4 groups: more (sequence, group) pairs than score CTAs in
+    # one wave, so the score kernel cuts the flattened piece list into ranges
+    # that cross from one group into the next
+    w = dataclasses.replace(gen.WORKLOADS["prefill_32k"], name="decode_many", h_q=16, h_kv=4, d=64, seed=46)
+    _run_case(w, prefix=7000, steps=3, batch=120, check_every=2, seqs=[0, 57, 119])
+
+
 def test_decode_16x128k_sampled():
     # the benchmark's decode workload: 16 sequences x 131072-token cache;
     # the oracle checks two sequences on the first and a later step
