@@ -394,6 +394,9 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
     if (tid == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
     return;
   }
+  // the first pass's bins are cleared while the keys load (the barrier after
+  // the key range covers both)
+  for (int i = tid; i < kSelBins; i += kSelThreads) big[i] = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int i0 = 0; i0 < ncand; i0 += 8 * kSelThreads) {        // eight loads in flight per thread
     float v[8];
@@ -428,8 +431,6 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
     // first pass over the top (up to) 11 bits of u, 2048 bins; thread tid
     // owns bins [8 tid, 8 tid + 8)
     const int d1 = min(hi, 11), shift1 = hi - d1, nb1 = 1 << d1;
-    for (int i = tid; i < nb1; i += kSelThreads) big[i] = 0;
-    __syncthreads();
     for (int i = tid; i < ncand; i += kSelThreads) atomicAdd(&big[(keys[i] - kmin) >> shift1], 1);
     __syncthreads();
     int loc = 0;
