@@ -81,6 +81,10 @@ def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
     w["score_bytes"] = n * h_q * d * 2 + 4 * h_kv * int(n1.sum())
     # top-k: read the visible part of S_shared, write the block lists
     w["topk_bytes"] = 4 * h_kv * int(n1.sum()) + 4 * h_kv * n * 96
+    # the pooled form: one (max, last window) pair per group of four visible windows
+    groups = (n1 + 3) // 4
+    w["score_bytes_pooled"] = n * h_q * d * 2 + 8 * h_kv * int(groups.sum())
+    w["topk_bytes_pooled"] = 8 * h_kv * int(groups.sum()) + 4 * h_kv * n * 96
     # sparse attention: QK^T and PV over the visible selected keys
     w["sparse_flops"] = 4 * d * h_q * int(keys.sum())
     w["sparse_exps"] = h_q * int(keys.sum())
@@ -318,6 +322,9 @@ def main():
     ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--decode-batch", type=int, default=0, help="sequences of the decode case (0: the workload's 16)")
+    ap.add_argument("--pool", default="s_shared", choices=["fused", "s_shared"],
+                    help="fused: the score kernel writes the max-pool's (max, last window) pairs; s_shared: it writes "
+                         "S_shared and the selection pools it")
     ap.add_argument("--lse", default="approx", choices=["approx", "exact"],
                     help="LSE of the scoring step: the coarse approximation (default) or the exact two-pass form")
     args = ap.parse_args()
@@ -373,8 +380,9 @@ def main():
     vl = T.make_varlen(data["lens"], cu, p)
     Kc1 = torch.empty(w.h_kv, vl.total_c1, w.d, dtype=torch.bfloat16, device=dev)
     Kc2 = torch.empty(w.h_kv, vl.total_c2, w.d, dtype=torch.bfloat16, device=dev)
-    ld = T.infllm2_scores_ld(vl, p)
-    S = torch.empty(w.h_kv, vl.total, ld, dtype=torch.float32, device=dev)
+    fused = args.pool == "fused"
+    ld = T.infllm2_pooled_ld(vl, p) if fused else T.infllm2_scores_ld(vl, p)
+    S = torch.empty(w.h_kv, vl.total, ld, dtype=torch.float32, device=dev)   # pairs or S_shared
     idx = torch.empty(w.h_kv, vl.total, p.n_sel, dtype=torch.int32, device=dev)
     out = torch.empty(vl.total, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
     sws = torch.empty(T.infllm2_sparse_workspace_bytes(vl, w.h_q), dtype=torch.uint8, device=dev)
@@ -386,9 +394,15 @@ def main():
         if ev is not None: ev[0].record(stream)
         T.infllm2_compress_k(K, vl, Kc1, Kc2, p, stream)
         if ev is not None: ev[1].record(stream)
-        T.infllm2_shared_scores(Q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
+        if fused:
+            T.infllm2_pooled_scores(Q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
+        else:
+            T.infllm2_shared_scores(Q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
         if ev is not None: ev[2].record(stream)
-        T.infllm2_topk_blocks(S, ld, vl, w.h_kv, idx, p, stream)
+        if fused:
+            T.infllm2_topk_blocks_pooled(S, ld, vl, w.h_kv, idx, p, stream)
+        else:
+            T.infllm2_topk_blocks(S, ld, vl, w.h_kv, idx, p, stream)
         if ev is not None: ev[3].record(stream)
         T.infllm2_sparse_attn(Q, K, V, idx, vl, out, p, stream, workspace=sws)
         if ev is not None: ev[4].record(stream)
@@ -455,6 +469,8 @@ def main():
     # ---- roofline of the dominant kernel
     hbm, tflops, tflops_sus, src = _peaks()
     work = algorithmic_work(w.seqlen, w.h_q, w.h_kv, w.d)
+    if fused:
+        work["score_bytes"], work["topk_bytes"] = work["score_bytes_pooled"], work["topk_bytes_pooled"]
     dom = max(per_kernel, key=per_kernel.get)
     if dom == "sparse":
         # the top-k gather (and the shared tiles) are L2 -> SM bound: see the design doc
@@ -513,9 +529,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q,V; K with per-block offsets)",
         "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
-                   "n_sel": w.n_sel, "lse": args.lse,
+                   "n_sel": w.n_sel, "lse": args.lse, "pool": args.pool,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "working set larger than L2 (Q 1 GiB, S_shared 4.3 GB); no extra flush"},
+                   "l2": "working set larger than L2 (Q 1 GiB; S_shared 4.3 GB, or its pooled pairs 2.2 GB); no extra flush"},
         "e2e": e2e,
         "gpu_launches": (len(kernels) + 1) * args.steps,   # the sparse call is two launches (local + top-k)
         "kernels": kern_detail,

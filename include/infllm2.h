@@ -160,6 +160,31 @@ int infllm2_shared_scores(const void* Q, const void* K_c1, const void* K_c2,
 int infllm2_topk_blocks(const float* S, int64_t ld, const infllm2_varlen* vl, int32_t h_kv,
                         int32_t* block_idx, const infllm2_params* p, void* stream);
 
+/* ---------------------------------------------------------------------
+ * Steps 2 and 3 with the first step of the max-pool fused into the score
+ * kernel ([top168] §三 third stage; S_shared itself is not written).  For
+ * query token t and each group of four C1 windows 4i .. 4i+3 whose first
+ * window is visible, the score kernel writes the pair
+ *   P[g, t, 2i]   = max{ S[g,t,j] : 4i <= j <= 4i+3, j visible }
+ *   P[g, t, 2i+1] = S[g,t,4i+3] if visible, else -inf
+ * (S as defined for infllm2_shared_scores; entries of groups with no visible
+ * window are not written), so that
+ *   score(b) = max(P[g,t,2b], P[g,t,2b-1])      (the second term for b >= 1)
+ * equals infllm2_topk_blocks' score(b) bit for bit, and
+ * infllm2_topk_blocks_pooled returns the same lists.  The pairs take half
+ * the bytes of S_shared.
+ *   P          fp32 [h_kv, total, ldp], ldp = infllm2_pooled_ld(vl, p)
+ *              (2 * ceil(max window count / 4), rounded up to a multiple of 4)
+ * Arguments, errors and the other buffers as for infllm2_shared_scores and
+ * infllm2_topk_blocks.
+ * ------------------------------------------------------------------- */
+int64_t infllm2_pooled_ld(const infllm2_varlen* vl, const infllm2_params* p);
+int infllm2_pooled_scores(const void* Q, const void* K_c1, const void* K_c2,
+                          const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
+                          float* P, int64_t ldp, const infllm2_params* p, void* stream);
+int infllm2_topk_blocks_pooled(const float* P, int64_t ldp, const infllm2_varlen* vl, int32_t h_kv,
+                               int32_t* block_idx, const infllm2_params* p, void* stream);
+
 /* Steps 2 and 3 in one call.  S_shared goes to `workspace` (at least
  * infllm2_select_workspace_bytes bytes) unless s_shared_out is non-NULL, in
  * which case it is written there ([h_kv, total, ld] fp32) and the workspace

@@ -187,6 +187,53 @@ def test_exact_lse_mode():
     assert T_status() == 0
 
 
+@pytest.mark.parametrize("name", ["varlen_small", "prefill_32k"])
+def test_pooled_scores(name):
+    # the max-pool's first step fused into the score kernel: the pairs give
+    # the same lists as S_shared on every row (bit for bit), and the block
+    # scores rebuilt from them match the oracle's max-pool at sampled rows
+    import trainable_block_sparse_pool_b200 as T
+    if name == "varlen_small":
+        w = VARLEN_SMALL
+        data = gen.make_prefill(w, lens=VARLEN_SMALL_LENS, seed=12)
+    else:
+        w = gen.WORKLOADS[name]
+        data = gen.make_prefill(w)
+    run = H.GpuRun(data, w)
+    run.compress()
+    run.scores()
+    run.topk()
+    ldp = T.infllm2_pooled_ld(run.vl, run.p)
+    P = torch.zeros(w.h_kv, run.vl.total, ldp, dtype=torch.float32, device="cuda")
+    idx_p = torch.full_like(run.idx, -7)
+    T.infllm2_pooled_scores(run.Q, run.Kc1, run.Kc2, run.vl, w.h_kv, P, ldp, run.p)
+    T.infllm2_topk_blocks_pooled(P, ldp, run.vl, w.h_kv, idx_p, run.p)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_p, run.idx)
+    rows = gen.sample_rows(run.vl.total, 48, seed=w.seed + 23)
+    P_cpu = P[:, torch.from_numpy(rows).cuda(), :].cpu().numpy().astype(np.float64)
+    sidx, tloc = H.seq_of_rows(run.lens, rows)
+    seqs = H.oracle_sequences(data, w, which=sorted(set(int(x) for x in sidx)))
+    op = H.oracle_params(w)
+    worst, n = 0.0, 0
+    for k, (s, t) in enumerate(zip(sidx, tloc)):
+        t = int(t)
+        for g in range(w.h_kv):
+            S_or = seqs[int(s)].shared_scores(t, g)
+            ref = O.block_scores(S_or, t, op)
+            # every block whose first window is visible has its pair
+            nb = (S_or.shape[0] + 3) // 4
+            for b in range(min(nb, ref.shape[0])):
+                got = P_cpu[g, k, 2 * b]
+                if b >= 1:
+                    got = max(got, P_cpu[g, k, 2 * b - 1])
+                worst = max(worst, abs(got - ref[b]) / max(abs(ref[b]), 1e-30))
+                n += 1
+    assert n > 0
+    assert worst <= H.S_RTOL, worst
+    assert T_status() == 0
+
+
 def _sampled_case(name, n_rows):
     w = gen.WORKLOADS[name]
     data = gen.make_prefill(w)

@@ -20,6 +20,7 @@ from . import build as _build
 __all__ = [
     "InfLLM2Error", "Params", "Varlen", "lib", "default_params", "make_varlen", "window_count",
     "infllm2_compress_k", "infllm2_shared_scores", "infllm2_topk_blocks", "infllm2_select_blocks",
+    "infllm2_pooled_ld", "infllm2_pooled_scores", "infllm2_topk_blocks_pooled",
     "infllm2_select_workspace_bytes", "infllm2_scores_ld", "infllm2_sparse_workspace_bytes", "infllm2_sparse_attn",
     "infllm2_dense_attn",
     "infllm2_get_device_status", "infllm2_clear_device_status", "infllm2_debug_wait_timeout",
@@ -90,6 +91,9 @@ def lib() -> ctypes.CDLL:
         "infllm2_compress_k": (ctypes.c_int, [_P, vp, i32, i32, _P, _P, pp, _P]),
         "infllm2_shared_scores": (ctypes.c_int, [_P, _P, _P, vp, i32, i32, i32, _P, i64, pp, _P]),
         "infllm2_topk_blocks": (ctypes.c_int, [_P, i64, vp, i32, _P, pp, _P]),
+        "infllm2_pooled_ld": (i64, [vp, pp]),
+        "infllm2_pooled_scores": (ctypes.c_int, [_P, _P, _P, vp, i32, i32, i32, _P, i64, pp, _P]),
+        "infllm2_topk_blocks_pooled": (ctypes.c_int, [_P, i64, vp, i32, _P, pp, _P]),
         "infllm2_select_workspace_bytes": (ctypes.c_size_t, [vp, i32, pp]),
         "infllm2_select_blocks": (ctypes.c_int, [_P, _P, _P, vp, i32, i32, i32, _P, ctypes.c_size_t, _P, _P, pp, _P]),
         "infllm2_sparse_workspace_bytes": (ctypes.c_size_t, [vp, i32]),
@@ -191,6 +195,25 @@ def infllm2_topk_blocks(S: torch.Tensor, ld: int, vl: Varlen, h_kv: int, block_i
     rc = lib().infllm2_topk_blocks(_ptr(S), ld, ctypes.byref(vl), h_kv, _ptr(block_idx),
                                    ctypes.byref(params or default_params()), _stream(stream))
     _check("infllm2_topk_blocks", rc)
+
+
+def infllm2_pooled_ld(vl: Varlen, params: Optional[Params] = None) -> int:
+    return int(lib().infllm2_pooled_ld(ctypes.byref(vl), ctypes.byref(params or default_params())))
+
+
+def infllm2_pooled_scores(Q: torch.Tensor, K_c1: torch.Tensor, K_c2: torch.Tensor, vl: Varlen, h_kv: int,
+                          P: torch.Tensor, ldp: int, params: Optional[Params] = None, stream=None) -> None:
+    h_q, d = Q.shape[1], Q.shape[2]
+    rc = lib().infllm2_pooled_scores(_ptr(Q), _ptr(K_c1), _ptr(K_c2), ctypes.byref(vl), h_q, h_kv, d, _ptr(P), ldp,
+                                     ctypes.byref(params or default_params()), _stream(stream))
+    _check("infllm2_pooled_scores", rc)
+
+
+def infllm2_topk_blocks_pooled(P: torch.Tensor, ldp: int, vl: Varlen, h_kv: int, block_idx: torch.Tensor,
+                               params: Optional[Params] = None, stream=None) -> None:
+    rc = lib().infllm2_topk_blocks_pooled(_ptr(P), ldp, ctypes.byref(vl), h_kv, _ptr(block_idx),
+                                          ctypes.byref(params or default_params()), _stream(stream))
+    _check("infllm2_topk_blocks_pooled", rc)
 
 
 def infllm2_select_blocks(Q: torch.Tensor, K_c1: torch.Tensor, K_c2: torch.Tensor, vl: Varlen, h_kv: int,

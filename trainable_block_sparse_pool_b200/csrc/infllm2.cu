@@ -159,32 +159,59 @@ int infllm2_compress_k(const void* K, const infllm2_varlen* vl, int32_t h_kv, in
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
 
-int infllm2_shared_scores(const void* Q, const void* K_c1, const void* K_c2, const infllm2_varlen* vl, int32_t h_q,
-                          int32_t h_kv, int32_t d, float* S, int64_t ld, const infllm2_params* p, void* stream) {
+static int scores_common(const void* Q, const void* K_c1, const void* K_c2, const infllm2_varlen* vl, int32_t h_q,
+                         int32_t h_kv, int32_t d, float* S, int64_t ld, int64_t ld_min, bool pool,
+                         const infllm2_params* p, void* stream) {
   int r;
   if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
   if (!Q || !K_c1 || !K_c2 || !S || !aligned16(Q) || !aligned16(K_c1) || !aligned16(K_c2) || !aligned16(S))
     return INFLLM2_ERR_INVALID_ARG;
-  if (ld < infllm2_scores_ld(vl, p) || (ld & 3)) return INFLLM2_ERR_INVALID_ARG;
+  if (ld < ld_min || (ld & 3)) return INFLLM2_ERR_INVALID_ARG;
   bool map_fail = false;
   cudaError_t e = launch_shared_scores(Q, K_c1, K_c2, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total,
                                        vl->total_c1, vl->total_c2, h_q, h_kv, d, S, ld, softmax_scale(p, d),
-                                       p->lse_mode == INFLLM2_LSE_EXACT, static_cast<cudaStream_t>(stream),
+                                       p->lse_mode == INFLLM2_LSE_EXACT, pool, static_cast<cudaStream_t>(stream),
                                        &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
 
-int infllm2_topk_blocks(const float* S, int64_t ld, const infllm2_varlen* vl, int32_t h_kv, int32_t* block_idx,
-                        const infllm2_params* p, void* stream) {
+int infllm2_shared_scores(const void* Q, const void* K_c1, const void* K_c2, const infllm2_varlen* vl, int32_t h_q,
+                          int32_t h_kv, int32_t d, float* S, int64_t ld, const infllm2_params* p, void* stream) {
+  return scores_common(Q, K_c1, K_c2, vl, h_q, h_kv, d, S, ld, infllm2_scores_ld(vl, p), false, p, stream);
+}
+
+int64_t infllm2_pooled_ld(const infllm2_varlen* vl, const infllm2_params* p) {
+  if (!vl || !p || vl->max_seqlen < 0) return 0;
+  const int64_t n1 = infllm2_window_count(vl->max_seqlen, p->c1_len, p->c1_stride);
+  return std::max<int64_t>(4, (2 * ((n1 + 3) / 4) + 3) & ~int64_t(3));
+}
+
+int infllm2_pooled_scores(const void* Q, const void* K_c1, const void* K_c2, const infllm2_varlen* vl, int32_t h_q,
+                          int32_t h_kv, int32_t d, float* P, int64_t ldp, const infllm2_params* p, void* stream) {
+  return scores_common(Q, K_c1, K_c2, vl, h_q, h_kv, d, P, ldp, infllm2_pooled_ld(vl, p), true, p, stream);
+}
+
+static int topk_common(const float* S, int64_t ld, int64_t ld_min, bool pool, const infllm2_varlen* vl,
+                       int32_t h_kv, int32_t* block_idx, const infllm2_params* p, void* stream) {
   int r;
   if ((r = check_varlen(vl)) || (r = check_params(p))) return r;
   if (!S || !block_idx || !aligned16(S) || h_kv <= 0) return INFLLM2_ERR_INVALID_ARG;
-  if (ld < infllm2_scores_ld(vl, p) || (ld & 3)) return INFLLM2_ERR_INVALID_ARG;
+  if (ld < ld_min || (ld & 3)) return INFLLM2_ERR_INVALID_ARG;
   cudaError_t e = launch_topk(S, ld, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_kv, p->n_init,
-                              p->n_local, p->top_k, static_cast<cudaStream_t>(stream), block_idx);
+                              p->n_local, p->top_k, pool, static_cast<cudaStream_t>(stream), block_idx);
   if (e == cudaErrorInvalidValue) return INFLLM2_ERR_UNSUPPORTED;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+int infllm2_topk_blocks(const float* S, int64_t ld, const infllm2_varlen* vl, int32_t h_kv, int32_t* block_idx,
+                        const infllm2_params* p, void* stream) {
+  return topk_common(S, ld, infllm2_scores_ld(vl, p), false, vl, h_kv, block_idx, p, stream);
+}
+
+int infllm2_topk_blocks_pooled(const float* P, int64_t ldp, const infllm2_varlen* vl, int32_t h_kv,
+                               int32_t* block_idx, const infllm2_params* p, void* stream) {
+  return topk_common(P, ldp, infllm2_pooled_ld(vl, p), true, vl, h_kv, block_idx, p, stream);
 }
 
 size_t infllm2_select_workspace_bytes(const infllm2_varlen* vl, int32_t h_kv, const infllm2_params* p) {

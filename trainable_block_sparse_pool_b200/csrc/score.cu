@@ -11,7 +11,10 @@
 //   phase B  S[g,t,j] = sum_h exp(scale * q[t,h] . K_c1[g,j] - LSE(t,h))
 //            over the visible stage-1 windows,
 // and writes only S (the group sum happens on chip, the per-head scores
-// never reach HBM).
+// never reach HBM).  With POOL the kernel writes, instead of S, the first
+// step of the 5/4/1 max-pool: for every group of four windows 4i .. 4i+3 the
+// pair (max of its visible windows, window 4i+3 or -inf), half the bytes of
+// S.  Block i's score is then max(pair i's max, pair i-1's last window).
 //
 // Both contractions run on the tcgen05 tensor cores with the Q tile resident
 // in shared memory:
@@ -66,7 +69,7 @@ __device__ __forceinline__ void set_abort(Bars* b) {
   *reinterpret_cast<volatile int*>(&b->abort) = 1;
 }
 
-template <int D, int G, bool EXACT>
+template <int D, int G, bool EXACT, bool POOL>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK1,
     const __grid_constant__ CUtensorMap tmK2, const __nv_bfloat16* __restrict__ Q,
@@ -294,11 +297,29 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(
 #pragma unroll
           for (int i = 0; i < 32; i += 2 * w) v[i] += v[i + w];
         }
+        if constexpr (POOL) {
+          // lanes 4k .. 4k+3 hold windows 4i .. 4i+3 of one group (j is a
+          // multiple of 4 on lane 4k): two xor shuffles give all four the
+          // group's maximum, and lane 4k+3, which holds the last window,
+          // writes the pair when the group's first window (48 positions
+          // earlier) is visible
 #pragma unroll
-        for (int i = 0; i < 32; i += G) {
-          const int tl = (cc + i) / G;          // token index within this half
-          const int tt = tt0 + tl;
-          if (tt < len && tt >= need) srow0[static_cast<int64_t>(tl) * ld + j] = v[i];
+          for (int i = 0; i < 32; i += G) {
+            const int tl = (cc + i) / G;
+            const int tt = tt0 + tl;
+            const float x = (tt < len && tt >= need) ? v[i] : -INFINITY;
+            float m = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            if ((lane & 3) == 3 && tt < len && tt >= need - 48)
+              *reinterpret_cast<float2*>(srow0 + static_cast<int64_t>(tl) * ld + 2 * (j >> 2)) = make_float2(m, x);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += G) {
+            const int tl = (cc + i) / G;          // token index within this half
+            const int tt = tt0 + tl;
+            if (tt < len && tt >= need) srow0[static_cast<int64_t>(tl) * ld + j] = v[i];
+          }
         }
         if (cc + 32 < 128) tmem_wait_ld32(vn);
       }
@@ -336,7 +357,7 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dim
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int G, bool EXACT>
+template <int D, int G, bool EXACT, bool POOL>
 static cudaError_t launch_score_t(const void* Q, const void* Kc1, const void* Kc2, const int32_t* cu, int batch,
                                   int max_seqlen, int64_t total, int64_t total_c1, int64_t total_c2, int h_q,
                                   int h_kv, float* S, int64_t ld, float scale, cudaStream_t st, bool* map_fail) {
@@ -360,7 +381,7 @@ static cudaError_t launch_score_t(const void* Q, const void* Kc1, const void* Kc
     const uint32_t box[3] = {64, score::kKeysPerTile, 1};
     if (!make_tmap(&mK2, Kc2, 3, dims, strides, box)) { *map_fail = true; return cudaErrorInvalidValue; }
   }
-  auto kern = score::score_kernel<D, G, EXACT>;
+  auto kern = score::score_kernel<D, G, EXACT, POOL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((max_seqlen + C::TQ - 1) / C::TQ, batch, h_kv);
@@ -373,15 +394,16 @@ static cudaError_t launch_score_t(const void* Q, const void* Kc1, const void* Kc
 
 cudaError_t launch_shared_scores(const void* Q, const void* Kc1, const void* Kc2, const int32_t* cu, int batch,
                                  int max_seqlen, int64_t total, int64_t total_c1, int64_t total_c2, int h_q,
-                                 int h_kv, int d, float* S, int64_t ld, float scale, bool exact, cudaStream_t st,
-                                 bool* map_fail) {
+                                 int h_kv, int d, float* S, int64_t ld, float scale, bool exact, bool pool,
+                                 cudaStream_t st, bool* map_fail) {
   const int G = h_q / h_kv;
+#define INFLLM2_SCORE_ARGS Q, Kc1, Kc2, cu, batch, max_seqlen, total, total_c1, total_c2, h_q, h_kv, S, ld, scale, st, map_fail
 #define INFLLM2_SCORE_CASE(DD, GG)                                                                                 \
   if (d == DD && G == GG)                                                                                         \
-    return exact ? launch_score_t<DD, GG, true>(Q, Kc1, Kc2, cu, batch, max_seqlen, total, total_c1, total_c2, h_q, \
-                                                h_kv, S, ld, scale, st, map_fail)                                 \
-                 : launch_score_t<DD, GG, false>(Q, Kc1, Kc2, cu, batch, max_seqlen, total, total_c1, total_c2,   \
-                                                 h_q, h_kv, S, ld, scale, st, map_fail);
+    return exact ? (pool ? launch_score_t<DD, GG, true, true>(INFLLM2_SCORE_ARGS)                                 \
+                         : launch_score_t<DD, GG, true, false>(INFLLM2_SCORE_ARGS))                               \
+                 : (pool ? launch_score_t<DD, GG, false, true>(INFLLM2_SCORE_ARGS)                                \
+                         : launch_score_t<DD, GG, false, false>(INFLLM2_SCORE_ARGS));
   INFLLM2_SCORE_CASE(128, 16)
   INFLLM2_SCORE_CASE(128, 8)
   INFLLM2_SCORE_CASE(128, 4)
@@ -393,6 +415,7 @@ cudaError_t launch_shared_scores(const void* Q, const void* Kc1, const void* Kc2
   INFLLM2_SCORE_CASE(64, 2)
   INFLLM2_SCORE_CASE(64, 1)
 #undef INFLLM2_SCORE_CASE
+#undef INFLLM2_SCORE_ARGS
   return cudaErrorInvalidValue;
 }
 

@@ -134,6 +134,10 @@ __device__ __noinline__ void warp_select_write(uint32_t* keys, int* hist, int nc
   for (int i = pos + lane; i < n_sel; i += 32) out[i] = -1;
 }
 
+// POOL: S holds the score kernel's pooled pairs (per group of four windows,
+// its visible maximum and its last window); block b takes the maximum of
+// pair b's first value and pair b-1's second.
+template <bool POOL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, int64_t ld,
                                                    const int32_t* __restrict__ cu, int batch, int64_t total,
                                                    int h_kv, int n_init, int n_local, int top_k, int n_sel,
@@ -179,22 +183,40 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
   for (int i0 = 0; i0 < ncand; i0 += 32 * kU) {
     float4 v4[kU];
     float pv[kU];
+    if constexpr (POOL) {
+      // pair b and the second value of pair b-1 (every candidate's first
+      // window is visible, so both pairs were written)
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = i0 + u * 32 + lane;
-      const int b = cand_lo + i;
-      const bool fast = i < ncand && b >= 1 && 4 * b + 3 < n1;
-      v4[u] = fast ? __ldg(reinterpret_cast<const float4*>(srow + 4 * b)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      pv[u] = fast ? __ldg(srow + 4 * b - 1) : 0.f;
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * 32 + lane;
+        const int b = cand_lo + i;
+        const bool ok = i < ncand;
+        const float2 pr = ok ? __ldg(reinterpret_cast<const float2*>(srow + 2 * b)) : make_float2(0.f, 0.f);
+        v4[u] = make_float4(pr.x, pr.y, 0.f, 0.f);
+        pv[u] = (ok && b >= 1) ? __ldg(srow + 2 * b - 1) : -INFINITY;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * 32 + lane;
+        const int b = cand_lo + i;
+        const bool fast = i < ncand && b >= 1 && 4 * b + 3 < n1;
+        v4[u] = fast ? __ldg(reinterpret_cast<const float4*>(srow + 4 * b)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        pv[u] = fast ? __ldg(srow + 4 * b - 1) : 0.f;
+      }
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int i = i0 + u * 32 + lane;
       if (i < ncand) {
         const int b = cand_lo + i;
-        const float m = (b >= 1 && 4 * b + 3 < n1)
-                            ? fmaxf(fmaxf(pv[u], v4[u].x), fmaxf(fmaxf(v4[u].y, v4[u].z), v4[u].w))
-                            : block_score(srow, b, n1);
+        float m;
+        if constexpr (POOL)
+          m = fmaxf(v4[u].x, pv[u]);
+        else
+          m = (b >= 1 && 4 * b + 3 < n1)
+                  ? fmaxf(fmaxf(pv[u], v4[u].x), fmaxf(fmaxf(v4[u].y, v4[u].z), v4[u].w))
+                  : block_score(srow, b, n1);
         const uint32_t k = __float_as_uint(fmaxf(m, 0.f));
         keys[i] = k;
         kmin = min(kmin, k);
@@ -208,7 +230,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
 }  // namespace sel
 
 cudaError_t launch_topk(const float* S, int64_t ld, const int32_t* cu, int batch, int max_seqlen, int64_t total,
-                        int h_kv, int n_init, int n_local, int top_k, cudaStream_t st, int32_t* out) {
+                        int h_kv, int n_init, int n_local, int top_k, bool pool, cudaStream_t st, int32_t* out) {
   const int n_sel = n_init + n_local + top_k;
   const int cand_cap = ((max_seqlen + 63) / 64 + 31) & ~31;
   const size_t per_warp = (static_cast<size_t>(cand_cap) + sel::kHistBins) * 4;
@@ -216,14 +238,14 @@ cudaError_t launch_topk(const float* S, int64_t ld, const int32_t* cu, int batch
   wpb = max(1, min(8, wpb));
   const size_t smem = per_warp * wpb;
   if (smem > 220 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(sel::topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  auto kern = pool ? sel::topk_kernel<true> : sel::topk_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t units = static_cast<int64_t>(h_kv) * total;
   const int64_t blocks = (units + wpb - 1) / wpb;
   if (blocks == 0) return cudaSuccess;
-  sel::topk_kernel<<<static_cast<unsigned>(blocks), wpb * 32, smem, st>>>(S, ld, cu, batch, total, h_kv, n_init,
-                                                                         n_local, top_k, n_sel, cand_cap, out);
+  kern<<<static_cast<unsigned>(blocks), wpb * 32, smem, st>>>(S, ld, cu, batch, total, h_kv, n_init, n_local, top_k,
+                                                              n_sel, cand_cap, out);
   return cudaGetLastError();
 }
 
