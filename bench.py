@@ -245,6 +245,134 @@ def decode_bytes_per_step(prefix: int, steps: int, batch: int, h_kv: int, d: int
     return tot / steps
 
 
+def bench_layer(T, gen, torch, dev, reps: int = 3, decode_steps: int = 8):
+    """One attention layer with random bf16 weights: the q/k/v and output
+    projections (cuBLAS GEMMs through torch) around the attention, with this
+    library's sparse attention and with a dense attention (torch SDPA on a
+    fused backend: a library kernel, the baseline).  Time to first token of a
+    131072-token prefill and time per output token of a 16 x 131072 decode, at
+    the bench workload's heads (32 query, 2 kv, d = 128, hidden 4096).  No norm
+    or positional encoding: the layers differ only in the attention."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    backends = [SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]
+    w = gen.WORKLOADS["prefill_128k"]
+    n, hq, hkv, d = w.seqlen, w.h_q, w.h_kv, w.d
+    hidden = hq * d
+    gen_t = torch.Generator(device=dev).manual_seed(1234)
+
+    def rand(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=gen_t, device=dev) * scale).to(torch.bfloat16)
+
+    Wq, Wk = rand(hidden, hq * d, scale=hidden ** -0.5), rand(hidden, hkv * d, scale=hidden ** -0.5)
+    Wv, Wo = rand(hidden, hkv * d, scale=hidden ** -0.5), rand(hq * d, hidden, scale=(hq * d) ** -0.5)
+    p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+
+    def timed(fn, n_iter=1, before=None):
+        fn()                                   # warm-up
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            if before is not None:
+                before()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(n_iter):
+                fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) / n_iter)
+        return statistics.median(ts)
+
+    res = {"workload": {"prefill": f"1 x {n}", "decode": f"16 x {n} cache"}, "hidden": hidden, "h_q": hq,
+           "h_kv": hkv, "d": d, "n_sel": w.n_sel, "weights": "random bf16 (no norm, no positional encoding)",
+           "dense": "torch scaled_dot_product_attention, cuDNN / flash / efficient backend"}
+    # ---- prefill: time to first token of one layer
+    x = rand(n, hidden)
+    cu = torch.tensor([0, n], dtype=torch.int32, device=dev)
+    vl = T.make_varlen([n], cu, p)
+    Kc1 = torch.empty(hkv, vl.total_c1, d, dtype=torch.bfloat16, device=dev)
+    Kc2 = torch.empty(hkv, vl.total_c2, d, dtype=torch.bfloat16, device=dev)
+    ld = T.infllm2_scores_ld(vl, p)
+    S = torch.empty(hkv, n, ld, dtype=torch.float32, device=dev)
+    idx = torch.empty(hkv, n, p.n_sel, dtype=torch.int32, device=dev)
+    o = torch.empty(n, hq, d, dtype=torch.bfloat16, device=dev)
+    sws = torch.empty(T.infllm2_sparse_workspace_bytes(vl, hq), dtype=torch.uint8, device=dev)
+
+    def sparse_prefill():
+        q = (x @ Wq).view(n, hq, d)
+        k = (x @ Wk).view(n, hkv, d)
+        v = (x @ Wv).view(n, hkv, d)
+        T.infllm2_compress_k(k, vl, Kc1, Kc2, p)
+        T.infllm2_shared_scores(q, Kc1, Kc2, vl, hkv, S, ld, p)
+        T.infllm2_topk_blocks(S, ld, vl, hkv, idx, p)
+        T.infllm2_sparse_attn(q, k, v, idx, vl, o, p, workspace=sws)
+        return o.view(n, hidden) @ Wo
+
+    def dense_prefill():
+        q = (x @ Wq).view(1, n, hq, d).transpose(1, 2)
+        k = (x @ Wk).view(1, n, hkv, d).transpose(1, 2)
+        v = (x @ Wv).view(1, n, hkv, d).transpose(1, 2)
+        with sdpa_kernel(backends):
+            a = F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+        return a.transpose(1, 2).reshape(n, hidden) @ Wo
+
+    res["ttft_ms"] = {"sparse": timed(sparse_prefill)}
+    try:
+        res["ttft_ms"]["dense"] = timed(dense_prefill)
+        res["ttft_speedup"] = res["ttft_ms"]["dense"] / res["ttft_ms"]["sparse"]
+    except RuntimeError as e:                  # no fused SDPA backend for this shape
+        res["ttft_ms"]["dense"] = None
+        res["dense_error"] = str(e).splitlines()[0][:200]
+    del x, Kc1, Kc2, S, idx, o, sws
+    torch.cuda.empty_cache()
+    # ---- decode: time per output token of one layer
+    batch, cap = 16, n + decode_steps + 1
+    k_cache = rand(batch, cap, hkv, d)
+    v_cache = rand(batch, cap, hkv, d)
+    kc1 = torch.empty(batch, hkv, T.window_count(cap, 32, 16), d, dtype=torch.bfloat16, device=dev)
+    kc2 = torch.empty(batch, hkv, T.window_count(cap, 128, 64), d, dtype=torch.bfloat16, device=dev)
+    seq_len = torch.full((batch,), n, dtype=torch.int32, device=dev)
+    st = T.make_decode_state(k_cache, v_cache, kc1, kc2, seq_len, hq)
+    ws = torch.empty(T.infllm2_decode_workspace_bytes(st, p), dtype=torch.uint8, device=dev)
+    od = torch.empty(batch, hq, d, dtype=torch.bfloat16, device=dev)
+    T.infllm2_decode_build_caches(st, p)
+    xd = rand(batch, hidden)
+
+    def sparse_decode():
+        q = (xd @ Wq).view(batch, hq, d)
+        kn = (xd @ Wk).view(batch, hkv, d)
+        vn = (xd @ Wv).view(batch, hkv, d)
+        T.infllm2_decode_step(st, q, kn, vn, od, ws, p)
+        return od.view(batch, hidden) @ Wo
+
+    def reset():
+        seq_len.fill_(n)
+
+    res["tpot_us"] = {"sparse": 1e3 * timed(sparse_decode, decode_steps, before=reset)}
+    reset()
+    del k_cache, v_cache, kc1, kc2, ws
+    torch.cuda.empty_cache()
+    kd = rand(batch, hkv, n, d)                # the dense cache, laid out for SDPA
+    vd = rand(batch, hkv, n, d)
+
+    def dense_decode():
+        q = (xd @ Wq).view(batch, hq, 1, d)
+        with sdpa_kernel(backends):
+            a = F.scaled_dot_product_attention(q, kd, vd, enable_gqa=True)
+        return a.reshape(batch, hidden) @ Wo
+
+    try:
+        res["tpot_us"]["dense"] = 1e3 * timed(dense_decode, decode_steps)
+        res["tpot_speedup"] = res["tpot_us"]["dense"] / res["tpot_us"]["sparse"]
+    except RuntimeError as e:
+        res["tpot_us"]["dense"] = None
+        res["dense_decode_error"] = str(e).splitlines()[0][:200]
+    res["device_status"] = T.infllm2_get_device_status()
+    return res
+
+
 def bench_decode(T, gen, torch, dev, graph_steps: int = 64, reps: int = 3, batch: int = 0):
     """µs per decode step of the 16 x 131072 workload, steps replayed from a
     CUDA graph of `graph_steps` consecutive steps (inputs staged on device).
@@ -320,6 +448,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
+    ap.add_argument("--layer", action="store_true",
+                    help="time one attention layer with random weights: sparse vs dense TTFT (128K prefill) and "
+                         "TPOT (16 x 128K decode)")
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--decode-batch", type=int, default=0, help="sequences of the decode case (0: the workload's 16)")
     ap.add_argument("--pool", default="s_shared", choices=["fused", "s_shared"],
@@ -365,6 +496,12 @@ def main():
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
     T.lib()
+
+    if args.layer:
+        res = bench_layer(T, gen, torch, dev)
+        if rank == 0:
+            print(json.dumps({"layer": res}), flush=True)
+        return
 
     if args.decode_only:
         dd = bench_decode(T, gen, torch, dev, graph_steps=args.decode_steps, batch=args.decode_batch)
