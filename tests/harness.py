@@ -27,7 +27,7 @@ def lib_params(w) -> "T.Params":
     return T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
 
 
-class GpuRun:
+class DeviceRun:
     """Device buffers and the CUDA path's steps for one packed batch."""
 
     def __init__(self, data: dict, w, keep_scores: bool = True):

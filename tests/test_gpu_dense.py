@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 
 def _dense_case(w, lens, seed, rows=None):
     data = gen.make_prefill(w, lens=lens, seed=seed)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.dense()
     torch.cuda.synchronize()
     total = run.vl.total
@@ -60,7 +60,7 @@ def test_sparse_equals_dense_when_every_block_is_selected():
     # |I| >= causal blocks: the sparse kernel must reproduce the dense one
     w = dataclasses.replace(gen.WORKLOADS["tiny_1k"], name="all_blocks", n_local=16, top_k=2, seed=24)
     data = gen.make_prefill(w, lens=[1024], seed=24)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.compress(); run.scores(); run.topk(); run.sparse()
     sparse_out = run.out.clone()
     run.dense()

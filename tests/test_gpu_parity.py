@@ -81,7 +81,7 @@ def _check_attention(run, w, rows, seqs, ref_idx):
 
 def _full_case(w, lens, seed):
     data = gen.make_prefill(w, lens=lens, seed=seed)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.compress()
     run.scores()
     run.topk()
@@ -160,7 +160,7 @@ def test_exact_lse_mode():
     import trainable_block_sparse_pool_b200 as T
     w = VARLEN_SMALL
     data = gen.make_prefill(w, lens=VARLEN_SMALL_LENS, seed=12)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.p.lse_mode = T.LSE_EXACT
     run.compress()
     run.scores()
@@ -199,7 +199,7 @@ def test_pooled_scores(name):
     else:
         w = gen.WORKLOADS[name]
         data = gen.make_prefill(w)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.compress()
     run.scores()
     run.topk()
@@ -237,7 +237,7 @@ def test_pooled_scores(name):
 def _sampled_case(name, n_rows):
     w = gen.WORKLOADS[name]
     data = gen.make_prefill(w)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.compress()
     run.scores()
     run.topk()
@@ -274,7 +274,7 @@ def test_deterministic_reruns():
     data = gen.make_prefill(w, lens=VARLEN_SMALL_LENS, seed=11)
     outs = []
     for _ in range(2):
-        run = H.GpuRun(data, w)
+        run = H.DeviceRun(data, w)
         run.compress(); run.scores(); run.topk(); run.sparse()
         torch.cuda.synchronize()
         outs.append((run.Kc1.cpu(), run.S.cpu(), run.idx.cpu(), run.out.cpu()))

@@ -33,7 +33,7 @@ def test_varlen_128k_dense_sparse_switch():
     errs = []
     # dense side
     dd = _sub(data, dense_ids)
-    run = H.GpuRun(dd, w)
+    run = H.DeviceRun(dd, w)
     run.dense()
     torch.cuda.synchronize()
     rows = gen.sample_rows(run.vl.total, 40, seed=3)
@@ -46,7 +46,7 @@ def test_varlen_128k_dense_sparse_switch():
             errs.append(np.abs(out[r, g * w.group:(g + 1) * w.group] - ref).ravel())
     # sparse side
     sd = _sub(data, sparse_ids)
-    run = H.GpuRun(sd, w)
+    run = H.DeviceRun(sd, w)
     run.compress(); run.scores(); run.topk()
     torch.cuda.synchronize()
     rows = gen.sample_rows(run.vl.total, 40, seed=4)

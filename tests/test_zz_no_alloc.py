@@ -50,7 +50,7 @@ CASES = [
 def test_noalloc_matches_workspace_entry_point(w, lens, seed):
     f = _entry()
     data = gen.make_prefill(w, lens=lens, seed=seed)
-    run = H.GpuRun(data, w)
+    run = H.DeviceRun(data, w)
     run.compress()
     ws = torch.empty(T.infllm2_select_workspace_bytes(run.vl, w.h_kv, run.p), dtype=torch.uint8, device="cuda")
     T.infllm2_select_blocks(run.Q, run.Kc1, run.Kc2, run.vl, w.h_kv, ws, run.idx, None, run.p)
