@@ -272,9 +272,12 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V,
  * to the next; one workspace must not serve two steps in flight at once).
  * The decode step takes the LSE approximation only (lse_mode EXACT is
  * INFLLM2_ERR_UNSUPPORTED here).
- * Capacities above 1441792 tokens (more than 22528 candidate blocks) are
- * INFLLM2_ERR_UNSUPPORTED, and infllm2_decode_workspace_bytes returns 0 for
- * them.  infllm2_decode_build_caches pools the seq_len[b] tokens already in
+ * Capacities above 1441792 tokens (more than 22528 candidate blocks) and
+ * batch * h_kv above 65535 are INFLLM2_ERR_UNSUPPORTED, and
+ * infllm2_decode_workspace_bytes returns 0 for them.  The three kernels are
+ * chained with programmatic dependent launch among themselves only: the
+ * first waits for whatever precedes it on the stream, and the last releases
+ * nothing early to what follows.  infllm2_decode_build_caches pools the seq_len[b] tokens already in
  * the cache into k_c1 / k_c2 (for a prefix written by the caller).
  * ------------------------------------------------------------------- */
 typedef struct {

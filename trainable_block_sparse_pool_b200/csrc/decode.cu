@@ -12,13 +12,17 @@
 //      rounding); per-head log-sum-exp partials over the visible coarse
 //      windows, split over CTAs
 //   K2 S over the visible stage-1 windows (head-group sum fused) and the
-//      max-pool to block scores, split over CTAs; the last CTA of each
-//      (sequence, group) selects the blocks
-//   K3 split-KV block-sparse attention over the selected blocks; the last
-//      CTA of each (sequence, group) merges the splits and writes the
-//      output, and the last group of a sequence advances seq_len
-// The "last CTA" hand-offs use a completion counter per (sequence, group)
-// (threadfence, then atomicAdd): no CTA ever waits for another.
+//      max-pool to block scores, streamed through TMA in one wave of CTAs;
+//      the CTA that completes the last piece of a (sequence, group) selects
+//      its blocks
+//   K3 split-KV block-sparse attention over the selected blocks; the splits
+//      of a (sequence, group) merge through distributed shared memory inside
+//      a thread-block cluster (or, past 8 splits, through the workspace and
+//      a completion counter), and the last group of a sequence advances
+//      seq_len
+// The hand-offs between CTAs are completion counters (threadfence, then
+// atomicAdd) and cluster barriers; the kernels are chained with
+// programmatic dependent launch.  No CTA spins on another's progress.
 // All of it is HBM-bound (the pooled keys and the selected K/V are read
 // once); the small contractions (16 heads against 8 keys or windows per
 // instruction) use warp-level mma.sync, which is far from being the limit.
@@ -1421,8 +1425,9 @@ struct DecodePlan {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Largest capacity whose candidate keys fit the selecting CTA's shared memory
-// next to the two staging buffers of the score kernel.
+// Limits: the selecting CTA's candidate keys fit its shared memory (capacity
+// up to about 1.44 M tokens), and the piece list packs (sequence, group) and
+// piece indices into 16 bits each.
 static bool decode_plan_supported(const DecodePlan& p) {
   return static_cast<size_t>(p.cand_cap) * 4 <= 88 * 1024 && p.nbg <= 65535 && p.np_cap <= 65535;
 }
