@@ -26,7 +26,9 @@ max-pool (kernel 5, stride 4, padding 1), |I| = n_init + n_local + top_k.
 
 Parity status: every function below is pinned by ``tests/test_oracle.py``
 (closed forms, invariants, brute force, a library routine, and the worked
-example of the [blog] section "先看一个具体例子").
+example of the [blog] section "先看一个具体例子"); the attention backward by
+central finite differences and, with every causal block selected, by fp64
+autograd of dense causal attention.
 """
 from __future__ import annotations
 
@@ -255,6 +257,60 @@ def dense_keys(t: int) -> np.ndarray:
     """All positions u <= t (dense causal attention, the short-sequence mode
     of the dense/sparse switch, [blog] "Dense-Sparse Switchable Attention")."""
     return np.arange(t + 1, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# step 4, backward: gradients of the block-sparse attention over a fixed
+# selection.  The method is trained end to end with no added parameters
+# ([news] §二, [top168] §一): the block selection is a discrete choice with no
+# gradient, and the loss reaches Q, K and V through the attention over the
+# selected keys.  Reading: the gradient is that of attend() with the key set
+# held fixed.
+# ----------------------------------------------------------------------------
+def attend_backward(q_g: np.ndarray, K_g: np.ndarray, V_g: np.ndarray, keys: np.ndarray,
+                    dO_g: np.ndarray, scale: float):
+    """Gradients of sum(dO_g * attend(q_g, K_g, V_g, t, keys, scale)) with
+    respect to q_g [G, d] and to the rows K_g[keys], V_g[keys] ([nk, d] each),
+    by the chain rule through O = P V, P = softmax(S), S = scale q K^T:
+      dV = P^T dO,   dP = dO V^T,
+      dS = P * (dP - rowsum(P * dP))      (the softmax Jacobian),
+      dq = scale dS K,   dK = scale dS^T q."""
+    G, d = q_g.shape
+    if keys.size == 0:
+        return np.zeros((G, d)), np.zeros((0, d)), np.zeros((0, d))
+    Kk, Vk = K_g[keys], V_g[keys]
+    s = (q_g @ Kk.T) * scale
+    s = s - s.max(axis=1, keepdims=True)
+    P = np.exp(s)
+    P = P / P.sum(axis=1, keepdims=True)
+    dV = P.T @ dO_g
+    dP = dO_g @ Vk.T
+    dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+    return scale * (dS @ Kk), scale * (dS.T @ q_g), dV
+
+
+def sparse_attention_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, blocks: np.ndarray,
+                              dO: np.ndarray, p: "Params"):
+    """Gradients of sum(dO * O) for one sequence, O[t, h] the block-sparse
+    attention of token t, query head h over the keys of its group's selected
+    blocks blocks[t, g] (-1 entries ignored), as sparse_keys() lists them.
+    Q, dO [n, h_q, d]; K, V [n, h_kv, d]; returns dQ, dK, dV in fp64.  A key's
+    gradient sums over the G heads of its group and every token whose
+    selection holds it."""
+    n, h_q, d = Q.shape
+    h_kv = K.shape[1]
+    G = h_q // h_kv
+    scale = p.softmax_scale(d)
+    dQ, dK, dV = np.zeros(Q.shape), np.zeros(K.shape), np.zeros(V.shape)
+    for t in range(n):
+        for g in range(h_kv):
+            keys = sparse_keys(t, blocks[t, g], p.block)
+            hs = slice(g * G, (g + 1) * G)
+            dq, dk, dv = attend_backward(Q[t, hs], K[:, g], V[:, g], keys, dO[t, hs], scale)
+            dQ[t, hs] = dq
+            dK[keys, g] += dk                  # keys are distinct within one row
+            dV[keys, g] += dv
+    return dQ, dK, dV
 
 
 # ----------------------------------------------------------------------------

@@ -276,3 +276,103 @@ def test_zero_query_gives_mean_of_visible_values():
 
 def test_dense_route_threshold():
     assert O.dense_route(8192) and not O.dense_route(8193) and O.dense_route(1)
+
+
+# ---------------------------------------------------------------- attention backward
+def _random_selection(rng, n, h_kv, n_sel, block=64):
+    """A valid selection per (token, group): the token's own block plus a
+    random subset of its earlier blocks, ascending, padded with -1."""
+    out = np.full((n, h_kv, n_sel), -1, dtype=np.int64)
+    for t in range(n):
+        bt = t // block
+        for g in range(h_kv):
+            earlier = [b for b in range(bt) if rng.random() < 0.5][: n_sel - 1]
+            sel = sorted(earlier + [bt])
+            out[t, g, :len(sel)] = sel
+    return out
+
+
+def _sparse_forward(Q, K, V, blocks, p):
+    n, h_q, d = Q.shape
+    h_kv = K.shape[1]
+    G = h_q // h_kv
+    scale = p.softmax_scale(d)
+    O_ = np.zeros(Q.shape)
+    for t in range(n):
+        for g in range(h_kv):
+            keys = O.sparse_keys(t, blocks[t, g], p.block)
+            O_[t, g * G:(g + 1) * G] = O.attend(Q[t, g * G:(g + 1) * G], K[:, g], V[:, g], t, keys, scale)
+    return O_
+
+
+def test_backward_matches_finite_differences():
+    # central differences of sum(dO * O) on a small case with a random
+    # (fixed) selection; the loss is smooth in Q, K and V
+    rng = np.random.default_rng(30)
+    n, h_q, h_kv, d = 160, 4, 2, 8
+    p = O.Params(n_init=1, n_local=1, top_k=2)
+    Q = rng.standard_normal((n, h_q, d))
+    K = rng.standard_normal((n, h_kv, d))
+    V = rng.standard_normal((n, h_kv, d))
+    dO = rng.standard_normal((n, h_q, d))
+    blocks = _random_selection(rng, n, h_kv, p.n_sel)
+    dQ, dK, dV = O.sparse_attention_backward(Q, K, V, blocks, dO, p)
+    eps = 1e-6
+
+    def loss(Qx, Kx, Vx):
+        return float((dO * _sparse_forward(Qx, Kx, Vx, blocks, p)).sum())
+
+    for name, X, dX in (("Q", Q, dQ), ("K", K, dK), ("V", V, dV)):
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, s)) for s in X.shape)
+            Xp, Xm = X.copy(), X.copy()
+            Xp[idx] += eps
+            Xm[idx] -= eps
+            args_p = {"Q": (Xp, K, V), "K": (Q, Xp, V), "V": (Q, K, Xp)}[name]
+            args_m = {"Q": (Xm, K, V), "K": (Q, Xm, V), "V": (Q, K, Xm)}[name]
+            num = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(num - dX[idx]) <= 1e-6 * max(1.0, abs(num)), (name, idx, num, dX[idx])
+
+
+def test_backward_equals_dense_autograd_when_every_block_is_selected():
+    # every causal block selected: the gradients are those of dense causal
+    # GQA attention, here from fp64 autograd of the library routine
+    rng = np.random.default_rng(31)
+    n, h_q, h_kv, d = 200, 4, 2, 16
+    p = O.Params(n_init=1, n_local=4, top_k=0)
+    G = h_q // h_kv
+    Q = rng.standard_normal((n, h_q, d))
+    K = rng.standard_normal((n, h_kv, d))
+    V = rng.standard_normal((n, h_kv, d))
+    dO = rng.standard_normal((n, h_q, d))
+    blocks = np.full((n, h_kv, p.n_sel), -1, dtype=np.int64)
+    for t in range(n):
+        blocks[t, :, :t // 64 + 1] = np.arange(t // 64 + 1)
+    dQ, dK, dV = O.sparse_attention_backward(Q, K, V, blocks, dO, p)
+    q = torch.from_numpy(Q).permute(1, 0, 2)[None].requires_grad_(True)
+    k = torch.from_numpy(K).permute(1, 0, 2)[None].requires_grad_(True)
+    v = torch.from_numpy(V).permute(1, 0, 2)[None].requires_grad_(True)
+    out = torch.nn.functional.scaled_dot_product_attention(q, k.repeat_interleave(G, 1), v.repeat_interleave(G, 1),
+                                                           is_causal=True)
+    (out * torch.from_numpy(dO).permute(1, 0, 2)[None]).sum().backward()
+    np.testing.assert_allclose(dQ, q.grad[0].permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK, k.grad[0].permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dV, v.grad[0].permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_value_gradient_sums_to_output_gradient():
+    # the attention weights of a row sum to one, so the value gradients of a
+    # group add up to the sum of its heads' output gradients over all tokens
+    rng = np.random.default_rng(32)
+    n, h_q, h_kv, d = 130, 4, 2, 8
+    p = O.Params(n_init=1, n_local=1, top_k=1)
+    Q = rng.standard_normal((n, h_q, d))
+    K = rng.standard_normal((n, h_kv, d))
+    V = rng.standard_normal((n, h_kv, d))
+    dO = rng.standard_normal((n, h_q, d))
+    blocks = _random_selection(rng, n, h_kv, p.n_sel)
+    _, _, dV = O.sparse_attention_backward(Q, K, V, blocks, dO, p)
+    G = h_q // h_kv
+    for g in range(h_kv):
+        np.testing.assert_allclose(dV[:, g].sum(axis=0), dO[:, g * G:(g + 1) * G].sum(axis=(0, 1)), rtol=1e-12,
+                                   atol=1e-12)
