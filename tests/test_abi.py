@@ -47,6 +47,12 @@ def test_window_count_and_ld(L):
     vl = T.Varlen()
     vl.max_seqlen = 131072
     assert T.infllm2_scores_ld(vl) == 8192      # 8191 windows rounded up to a multiple of 4
+    # pooled pairs: 2 * ceil(8191 / 4) = 4096, already a multiple of 4
+    assert T.infllm2_pooled_ld(vl) == 4096
+    vl.max_seqlen = 1024                        # 63 windows: 16 groups, 32 floats
+    assert T.infllm2_pooled_ld(vl) == 32
+    vl.max_seqlen = 100                         # 5 windows: 2 groups, 4 floats
+    assert T.infllm2_pooled_ld(vl) == 4
 
 
 def test_status_strings(L):
@@ -76,6 +82,11 @@ def test_argument_errors_are_caught_on_host(L):
     assert L.infllm2_shared_scores(0x1000, 0x1000, 0x1000, by(vl), 5, 2, 64, 0x1000, 64, by(p), None) == -1
     # ld too small
     assert L.infllm2_shared_scores(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 60, by(p), None) == -1
+    # the pooled pairs' ld is checked against infllm2_pooled_ld (32 floats here) and must be a multiple of 4
+    assert L.infllm2_pooled_scores(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 28, by(p), None) == -1
+    assert L.infllm2_pooled_scores(0x1000, 0x1000, 0x1000, by(vl), 4, 1, 64, 0x1000, 34, by(p), None) == -1
+    assert L.infllm2_topk_blocks_pooled(0x1000, 28, by(vl), 1, 0x1000, by(p), None) == -1
+    assert L.infllm2_topk_blocks_pooled(None, 32, by(vl), 1, 0x1000, by(p), None) == -1
     # unsupported pooling geometry
     q = T.default_params(c1_len=48)
     assert L.infllm2_topk_blocks(0x1000, 64, by(vl), 1, 0x1000, by(q), None) == -2
