@@ -68,25 +68,10 @@ __device__ __forceinline__ void load_qfrag(QFrag<D>& f, const __nv_bfloat16* q_h
   }
 }
 
-// Scores of 16 heads against the 8 keys rows[gid] (a row pointer per lane
-// group, nullptr = zero row).  c[0..1]: head gid, keys 2tig, 2tig+1;
-// c[2..3]: head gid+8.
-template <int D>
-__device__ __forceinline__ void scores_16x8(float (&c)[4], const QFrag<D>& f, const __nv_bfloat16* row, int lane) {
-  const int tig = lane & 3;
-  c[0] = c[1] = c[2] = c[3] = 0.f;
-#pragma unroll
-  for (int p = 0; p < D / 32; ++p) {
-    const uint4 kv = row ? *reinterpret_cast<const uint4*>(row + 32 * p + 8 * tig) : make_uint4(0, 0, 0, 0);
-    const uint32_t a0[4] = {f.lo[p].x, f.hi[p].x, f.lo[p].y, f.hi[p].y};
-    mma16816(c, a0, kv.x, kv.y);
-    const uint32_t a1[4] = {f.lo[p].z, f.hi[p].z, f.lo[p].w, f.hi[p].w};
-    mma16816(c, a1, kv.z, kv.w);
-  }
-}
-
-// Same product as scores_16x8, with the key row already loaded into
-// registers (so a warp can issue every load it needs before the first MMA).
+// Scores of 16 heads against 8 keys whose rows (one per lane group gid)
+// are already in registers: c[0..1] head gid, keys 2tig, 2tig+1; c[2..3]
+// head gid+8.  load_krow fetches a row (nullptr = zero row), so a warp can
+// issue every load it needs before the first MMA.
 template <int D>
 __device__ __forceinline__ void load_krow(uint4 (&kv)[D / 32], const __nv_bfloat16* row, int lane) {
   const int tig = lane & 3;
@@ -112,7 +97,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool f
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait_n() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
