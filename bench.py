@@ -196,7 +196,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle baseline
-def oracle_sample(w, data, seconds: float):
+def oracle_sample(w, data, seconds: float, lse: str = "approx"):
     """Time the fp64 oracle on rows of the workload until ~`seconds` of CPU
     time: pooling of the whole sequence, then scores, selection and sparse
     attention for uniformly sampled (token, group) rows.  Returns tokens/s
@@ -207,7 +207,7 @@ def oracle_sample(w, data, seconds: float):
     except Exception:  # pragma: no cover
         limiter = None
     from oracle import infllm2_oracle as O
-    p = O.Params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+    p = O.Params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k, lse_mode=lse)
     t0 = time.perf_counter()
     seq = O.Sequence1(O.to_f64(data["Q"]), O.to_f64(data["K"]), O.to_f64(data["V"]), p)
     t_pool = time.perf_counter() - t0
@@ -471,13 +471,14 @@ def main():
         if rank != 0:
             return
         data = gen.make_prefill(w)
-        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds / max(1, args.steps) * args.steps)
+        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds / max(1, args.steps) * args.steps, args.lse)
         line = {
             "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.seqlen / tok_s,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q,
-                                             "h_kv": w.h_kv, "d": w.d, "n_sel": w.n_sel},
+                                             "h_kv": w.h_kv, "d": w.d, "n_sel": w.n_sel, "lse": args.lse,
+                                             "pool": args.pool, "parallelism": "single GPU"},
             "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"pooling of the whole sequence + {rows} sampled (token, group) rows, "
                                        f"{secs:.1f} s, extrapolated to all rows"},
@@ -685,7 +686,7 @@ def main():
         dd["bound"] = "hbm"
         line["decode"] = dd
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds)
+        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds, args.lse)
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"pooling of the whole 128K sequence + {rows} uniformly sampled "
                                           f"(token, group) rows ({secs:.1f} s), extrapolated to all rows"}
