@@ -613,8 +613,14 @@ def main():
     if dom == "sparse":
         # the top-k gather (and the shared tiles) are L2 -> SM bound: see the design doc
         ach = work["sparse_gather_bytes"] / (per_kernel["sparse"] / 1e3) / 1e9
+        # DRAM bytes of the step's two sparse kernels (top-k and LOCAL), read
+        # and written, from one ncu capture of the 32K workload (327 + 230 MB and
+        # 562 + 228 MB), scaled by tokens: Q, the output and the partials
+        # grow with them, while the K/V gather stays in L2
+        traffic = (327.0 + 230.0 + 561.9 + 228.3) * 1e6 * (w.seqlen / 32768) if w.name.startswith("prefill_") else None
         roof = {"kernel": "sparse_attn (top-k gather + shared init/local tiles)", "bound": "l2", "achieved": ach,
-                "peak": l2["GB/s"], "unit": "GB/s", "frac": ach / l2["GB/s"], "traffic": None,
+                "peak": l2["GB/s"], "unit": "GB/s", "frac": ach / l2["GB/s"], "traffic": traffic,
+                "traffic_source": "DRAM read + write per step of the two sparse kernels, ncu at 32K scaled by tokens",
                 "peak_source": "L2 gather probe, same tile shape, same run (measured)"}
     elif dom == "scores":
         ach = work["score_flops"] / (per_kernel["scores"] / 1e3) / 1e12
