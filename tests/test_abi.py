@@ -119,3 +119,31 @@ def test_workspace_size(L):
     assert T.infllm2_select_workspace_bytes(vl, 2) == 2 * 131072 * 8192 * 4
     # one fp32 log-sum-exp per (token, query head)
     assert T.infllm2_sparse_workspace_bytes(vl, 32) == 131072 * 32 * 4
+
+
+def _decode_state(batch, capacity, h_q=32, h_kv=2, d=128):
+    st = T.DecodeState()
+    st.k_cache = st.v_cache = st.k_c1 = st.k_c2 = st.seq_len = 0x1000
+    st.batch, st.capacity, st.h_q, st.h_kv, st.d = batch, capacity, h_q, h_kv, d
+    return st
+
+
+def test_decode_plan_limits(L):
+    # the host-side decode plan: supported shapes get a workspace, the
+    # documented limits (candidate keys of one selection in shared memory;
+    # batch * h_kv and pieces in 16 bits) and the exact LSE give 0
+    p = T.default_params()
+    by = ctypes.byref
+    ws = L.infllm2_decode_workspace_bytes(by(_decode_state(16, 131072 + 64)), by(p))
+    assert ws > 0 and ws % 256 == 0
+    # at least, per (b, g): the block scores of 2049 blocks and the 96-entry block list
+    assert ws >= 32 * (2049 * 4 + 96 * 4)
+    assert L.infllm2_decode_workspace_bytes(by(_decode_state(1, 1441792)), by(p)) > 0
+    assert L.infllm2_decode_workspace_bytes(by(_decode_state(1, 1441792 + 64)), by(p)) == 0
+    assert L.infllm2_decode_workspace_bytes(by(_decode_state(32767, 4096)), by(p)) > 0
+    assert L.infllm2_decode_workspace_bytes(by(_decode_state(32768, 4096)), by(p)) == 0   # 65536 (b, g) pairs
+    q = T.default_params(lse_mode=T.LSE_EXACT)
+    assert L.infllm2_decode_workspace_bytes(by(_decode_state(16, 131072 + 64)), by(q)) == 0
+    # a step with too small a workspace is refused on the host
+    st = _decode_state(16, 131072 + 64)
+    assert L.infllm2_decode_step(by(st), 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, ws - 256, by(p), None) == -3
