@@ -376,3 +376,15 @@ def test_backward_value_gradient_sums_to_output_gradient():
     for g in range(h_kv):
         np.testing.assert_allclose(dV[:, g].sum(axis=0), dO[:, g * G:(g + 1) * G].sum(axis=(0, 1)), rtol=1e-12,
                                    atol=1e-12)
+
+
+def test_lse_approximation_cost_ratio():
+    # [top168] §四: the coarse windows are 4x longer and 4x sparser, so the
+    # approximation's coarse pass adds a quarter of a scoring pass (1.25x in
+    # all) while the exact two-pass form doubles it (2x); counted here as
+    # visible (token, window) products over a 128K sequence
+    n = 131072
+    fine = sum(O.visible_windows(t, 32, 16) for t in range(n))
+    coarse = sum(O.visible_windows(t, 128, 64) for t in range(n))
+    assert abs((fine + coarse) / fine - 1.25) < 2e-3
+    assert (fine + fine) / fine == 2.0
