@@ -313,6 +313,47 @@ def sparse_attention_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block
     return dQ, dK, dV
 
 
+def invert_block_lists(blocks: np.ndarray, n: int, block: int) -> List[List[List[int]]]:
+    """For every kv group g and key block kb, the tokens t whose selection
+    blocks[t, g] holds kb, ascending: the inverse of the block lists, the
+    order in which a key-block-major backward visits its query rows."""
+    h_kv = blocks.shape[1]
+    nblk = (n + block - 1) // block
+    inv: List[List[List[int]]] = [[[] for _ in range(nblk)] for _ in range(h_kv)]
+    for t in range(n):
+        for g in range(h_kv):
+            for kb in blocks[t, g]:
+                if kb >= 0:
+                    inv[g][int(kb)].append(t)
+    return inv
+
+
+def key_block_gradients(Q: np.ndarray, K: np.ndarray, V: np.ndarray, blocks: np.ndarray,
+                        dO: np.ndarray, p: "Params"):
+    """dK and dV of sparse_attention_backward() gathered per key block instead
+    of scattered per query row: for block kb of group g, the sum over the
+    tokens that selected it of that row's contribution to the block's keys
+    (only keys <= t count for token t).  Same result, no two rows writing
+    one key at once."""
+    n, h_q, d = Q.shape
+    h_kv = K.shape[1]
+    G = h_q // h_kv
+    scale = p.softmax_scale(d)
+    inv = invert_block_lists(blocks, n, p.block)
+    dK, dV = np.zeros(K.shape), np.zeros(V.shape)
+    for g in range(h_kv):
+        hs = slice(g * G, (g + 1) * G)
+        for kb, rows in enumerate(inv[g]):
+            lo = kb * p.block
+            for t in rows:
+                keys = sparse_keys(t, blocks[t, g], p.block)
+                _, dk, dv = attend_backward(Q[t, hs], K[:, g], V[:, g], keys, dO[t, hs], scale)
+                mine = (keys >= lo) & (keys < lo + p.block)
+                dK[keys[mine], g] += dk[mine]
+                dV[keys[mine], g] += dv[mine]
+    return dK, dV
+
+
 # ----------------------------------------------------------------------------
 # per-sequence drivers
 # ----------------------------------------------------------------------------

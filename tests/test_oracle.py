@@ -388,3 +388,22 @@ def test_lse_approximation_cost_ratio():
     coarse = sum(O.visible_windows(t, 128, 64) for t in range(n))
     assert abs((fine + coarse) / fine - 1.25) < 2e-3
     assert (fine + fine) / fine == 2.0
+
+
+def test_key_block_gradients_equal_row_scatter():
+    # the key-block-major form (inverse lists) gives the row-major scatter's dK, dV
+    rng = np.random.default_rng(33)
+    n, h_q, h_kv, d = 300, 4, 2, 8
+    p = O.Params(n_init=1, n_local=1, top_k=2)
+    Q = rng.standard_normal((n, h_q, d))
+    K = rng.standard_normal((n, h_kv, d))
+    V = rng.standard_normal((n, h_kv, d))
+    dO = rng.standard_normal((n, h_q, d))
+    blocks = _random_selection(rng, n, h_kv, p.n_sel)
+    _, dK, dV = O.sparse_attention_backward(Q, K, V, blocks, dO, p)
+    dK2, dV2 = O.key_block_gradients(Q, K, V, blocks, dO, p)
+    np.testing.assert_allclose(dK2, dK, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dV2, dV, rtol=1e-12, atol=1e-12)
+    # every selected (token, block) pair appears once in the inverse lists
+    inv = O.invert_block_lists(blocks, n, p.block)
+    assert sum(len(r) for g in inv for r in g) == int((blocks >= 0).sum())
