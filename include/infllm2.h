@@ -207,9 +207,10 @@ int infllm2_select_blocks(const void* Q, const void* K_c1, const void* K_c2,
  *   - Problems whose S_shared (h_kv * total * ld floats, ld =
  *     infllm2_scores_ld) exceeds the array return
  *     INFLLM2_ERR_WORKSPACE_TOO_SMALL before anything is launched.
- *   - The first call on a device looks up the array's device address for
- *     that device (cudaGetSymbolAddress); make that first call before
- *     capturing the stream into a graph.
+ *   - Every call looks up the array's device address on the current
+ *     device (cudaGetSymbolAddress, which allocates nothing); the first call
+ *     on a device is also the one that sets the array up there, so make that
+ *     first call before any stream capture.
  *   - Every call uses the same array: calls whose kernels can overlap on the
  *     GPU race on it.  It keeps the last call's scores; none of it needs to
  *     start at zero.
@@ -232,7 +233,10 @@ int infllm2_select_blocks_noalloc(const void* Q, const void* K_c1, const void* K
  * of infllm2_select_blocks / infllm2_topk_blocks does: the shared init and
  * local blocks are attended once per group of query tokens and the other
  * entries per token, and the two partials are merged.  A row that breaks
- * this rule gets a wrong result (no fault).
+ * this rule (also: entries out of [0, b_t], repeated, unsorted, or valid
+ * entries after a -1) is detected on the device and recorded in the device
+ * status word as INFLLM2_ERR_DEVICE_BOUNDS; its output is then undefined
+ * (no fault, no out-of-range read).
  * workspace: device, 16-byte aligned, at least
  * infllm2_sparse_workspace_bytes(vl, h_q) bytes (one fp32 per (token,
  * query head)); nothing in it outlives the call's kernels.
@@ -294,22 +298,23 @@ typedef struct {
 } infllm2_decode_state;
 
 size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infllm2_params* p);
+
+/* The blocks each decode step selected ([top168] §三 third stage, §七: the
+ * same init U local U top-k rule as infllm2_topk_blocks, applied to row t).
+ * Returns the byte offset inside the decode workspace of an int32 array
+ * [batch, h_kv, n_init + n_local + top_k]: for sequence b and kv group g,
+ * the blocks attended by the new token, ascending, padded with -1.  The
+ * array is written by infllm2_decode_step and holds the lists of the last
+ * step that ran on this workspace, for every sequence whose step ran (t <
+ * capacity), until the next step on the same workspace overwrites it; read
+ * it after that step's kernels have completed (stream order).  The call
+ * launches nothing.  Returns -1 where infllm2_decode_workspace_bytes
+ * returns 0 (invalid or unsupported state or parameters). */
+int64_t infllm2_decode_block_idx_offset(const infllm2_decode_state* st, const infllm2_params* p);
 int infllm2_decode_build_caches(const infllm2_decode_state* st, const infllm2_params* p, void* stream);
 int infllm2_decode_step(const infllm2_decode_state* st, const void* q, const void* k_new, const void* v_new,
                         void* out, void* workspace, size_t workspace_bytes, const infllm2_params* p,
                         void* stream);
-
-/* Measurement: L2 -> SM gather bandwidth with the block-sparse attention's
- * access pattern: the roofline denominator of the gather-bound attention
- * kernel.  K, V: [rows, h_kv, 128] bf16 device tensors (any contents).
- * One CTA per SM; `producers` (1, 2, 3 or 6) warps each gather `tiles`
- * tiles of two random 64-key blocks (32 KB) of kv group 0 from the first
- * nblk blocks, with 192 KB in flight per SM, and discard them.  The caller
- * times the call (bytes = num_SMs * producers * tiles * 32768).  Returns
- * INFLLM2_ERR_INVALID_ARG for null or misaligned tensors, nblk * 64 > rows
- * or tiles < 1. */
-int infllm2_probe_l2_gather(const void* K, const void* V, int64_t rows, int32_t h_kv, int32_t nblk,
-                            int32_t tiles, int32_t producers, void* stream);
 
 /* Device status word (per device).  Returns INFLLM2_OK or the first
  * INFLLM2_ERR_DEVICE_* recorded by a kernel since the last clear.

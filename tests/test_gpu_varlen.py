@@ -54,15 +54,17 @@ def test_varlen_128k_dense_sparse_switch():
     seqs = H.oracle_sequences(sd, w, which=sorted(set(int(s) for s in sidx)))
     idx_all = np.stack([H.default_index_rows(run.lens, w) for _ in range(w.h_kv)])
     gpu_idx = run.idx.cpu().numpy()
-    mism = 0
+    lists, S_rows, ts = [], [], []
     for r, s, t in zip(rows, sidx, tloc):
         for g in range(w.h_kv):
             S = seqs[int(s)].shared_scores(int(t), g)
-            sel = O.select_blocks(S, int(t), op)
-            idx_all[g, r] = sel
-            if O.topk_gap(S, int(t), op) > H.GAP_MIN and not np.array_equal(gpu_idx[g, r], sel):
-                mism += 1
-    assert mism == 0
+            idx_all[g, r] = O.select_blocks(S, int(t), op)
+            lists.append(gpu_idx[g, r])
+            S_rows.append(S)
+            ts.append(int(t))
+    exact, tie, bad = H.compare_lists(lists, S_rows, ts, op)
+    print(f"[varlen_128k] selection: {exact} rows bit-exact, {tie} near-tie rows valid")
+    assert bad == 0 and exact >= 0.8 * (exact + tie), (bad, exact, tie)
     run.sparse(torch.from_numpy(idx_all).cuda())
     torch.cuda.synchronize()
     out = run.out.float().cpu().numpy()

@@ -407,3 +407,100 @@ def test_key_block_gradients_equal_row_scatter():
     # every selected (token, block) pair appears once in the inverse lists
     inv = O.invert_block_lists(blocks, n, p.block)
     assert sum(len(r) for g in inv for r in g) == int((blocks >= 0).sum())
+
+
+# ---------------------------------------------------------------- parity helpers
+def _row_with_block_scores(t, values):
+    """A C1 score row whose max-pooled block scores are exactly `values`
+    ({block: score}; other blocks score 1e-9): block b's score is placed in
+    window 4b+1, which lies in block b's pooling range [4b-1, 4b+3] only."""
+    S = np.full(O.visible_windows(t, 32, 16), 1e-9)
+    for b, v in values.items():
+        S[4 * b + 1] = v
+    return S
+
+
+def test_topk_gap_hand_built_row():
+    # n_init=1, n_local=2, top_k=2; t in block 9: init {0}, local {8, 9},
+    # candidates {1..7}.  Candidate scores sorted: 0.9, 0.8 | 0.7, 0.5, ...
+    # so the k-th is 0.8 and the (k+1)-th 0.7: gap = 0.1 / 0.8.
+    p = O.Params(n_init=1, n_local=2, top_k=2)
+    t = 9 * 64 + 63
+    cand = {1: 0.5, 2: 0.9, 3: 0.3, 4: 0.8, 5: 0.1, 6: 0.7, 7: 0.2}
+    S = _row_with_block_scores(t, cand)
+    np.testing.assert_array_equal(O.block_scores(S, t, p)[1:8], [cand[b] for b in range(1, 8)])
+    assert O.topk_gap(S, t, p) == pytest.approx(0.125, rel=1e-12)
+    # init and local blocks are not candidates: large scores there change nothing
+    S2 = _row_with_block_scores(t, {**cand, 0: 5.0, 8: 4.0, 9: 3.0})
+    assert O.topk_gap(S2, t, p) == pytest.approx(0.125, rel=1e-12)
+    # a tie at the boundary gives a zero gap; the gap is never negative
+    S3 = _row_with_block_scores(t, {**cand, 6: 0.8})
+    assert O.topk_gap(S3, t, p) == 0.0
+    rng = np.random.default_rng(21)
+    for _ in range(50):
+        R = rng.random(O.visible_windows(t, 32, 16))
+        assert O.topk_gap(R, t, p) >= 0.0
+
+
+def test_topk_gap_infinite_when_every_candidate_is_taken():
+    # block 4: init {0}, local {3, 4}, candidates {1, 2} = top_k: nothing to
+    # choose, the gap is +inf; one more block makes it finite
+    p = O.Params(n_init=1, n_local=2, top_k=2)
+    rng = np.random.default_rng(22)
+    t = 4 * 64 + 63
+    assert O.topk_gap(rng.random(O.visible_windows(t, 32, 16)), t, p) == math.inf
+    t = 5 * 64
+    assert math.isfinite(O.topk_gap(rng.random(O.visible_windows(t, 32, 16)), t, p))
+    # the default parameters: candidates exist only from block 1 + 32 + 63 = 96 on
+    pd = O.Params()
+    for t in (0, 2111, 96 * 64 - 1):
+        assert O.topk_gap(rng.random(O.visible_windows(t, 32, 16)), t, pd) == math.inf
+    t = 96 * 64
+    assert math.isfinite(O.topk_gap(rng.random(O.visible_windows(t, 32, 16)), t, pd))
+
+
+def test_lse_rows_comparable_boundary():
+    # a row uses the coarse approximation from t = l_C2 - 1 = 127 on (its
+    # first complete coarse window); before that the approximate and the
+    # exact modes are the same computation, after it they differ
+    p = O.Params()
+    assert [O.lse_rows_comparable(t, p) for t in (0, 126, 127, 128, 5000)] == [False, False, True, True, True]
+    pa, pe = O.Params(n_local=2, top_k=2), O.Params(n_local=2, top_k=2, lse_mode="exact")
+    sa, se = _seq(400, 4, 1, 16, 23, p=pa), _seq(400, 4, 1, 16, 23, p=pe)
+    for t in range(31, 400, 3):
+        a, e = sa.shared_scores(t, 0), se.shared_scores(t, 0)
+        if O.lse_rows_comparable(t, pa):
+            assert np.abs(a - e).max() > 1e-6, t
+        else:
+            np.testing.assert_array_equal(a, e)
+    # rows that are not comparable never reach the top-k: no candidates yet
+    # (t < 127 lies in blocks 0 and 1, which are init or local)
+    for t in range(127):
+        assert O.topk_gap(np.ones(O.visible_windows(t, 32, 16)), t, O.Params(n_init=1, n_local=1, top_k=1)) == math.inf
+
+
+def test_decode_row_is_row_t_of_the_prefill_rule():
+    # decode of the token at t on the prefix K[:t+1] gives the selection and
+    # output of row t of the prefill oracle on a LONGER sequence (causality:
+    # later tokens change nothing for row t), and pooled keys that are the
+    # prefix of the longer sequence's pooled keys
+    p = O.Params(n_init=1, n_local=2, top_k=3)
+    n, h_q, h_kv, d = 900, 4, 2, 16
+    full = _seq(n, h_q, h_kv, d, 24, p=p)
+    for t in (0, 31, 127, 128, 300, 511, 640, 899):
+        sel, out, scores, Kc1, Kc2 = O.decode_row(full.K[:t + 1], full.V[:t + 1], full.Q[t], p)
+        n1, n2 = O.window_count(t + 1, 32, 16), O.window_count(t + 1, 128, 64)
+        assert Kc1.shape[1] == n1 and Kc2.shape[1] == n2
+        np.testing.assert_array_equal(Kc1, full.Kc1[:, :n1])
+        np.testing.assert_array_equal(Kc2, full.Kc2[:, :n2])
+        for g in range(h_kv):
+            np.testing.assert_array_equal(scores[g], full.shared_scores(t, g))
+            np.testing.assert_array_equal(sel[g], full.select(t, g))
+            np.testing.assert_allclose(out[g * 2:(g + 1) * 2], full.sparse_out(t, g, sel[g]), rtol=1e-13, atol=1e-15)
+    # the last row of a sequence sees its own token: changing it changes the output
+    t = 640
+    V2 = full.V[:t + 1].copy()
+    V2[t] += 1.0
+    _, o1, _, _, _ = O.decode_row(full.K[:t + 1], full.V[:t + 1], full.Q[t], p)
+    _, o2, _, _, _ = O.decode_row(full.K[:t + 1], V2, full.Q[t], p)
+    assert np.abs(o1 - o2).min() > 0

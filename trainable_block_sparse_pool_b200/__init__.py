@@ -105,6 +105,7 @@ def lib() -> ctypes.CDLL:
         "infllm2_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
         "infllm2_probe_l2_gather": (ctypes.c_int, [_P, _P, i64, i32, i32, i32, i32, _P]),
         "infllm2_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(DecodeState), pp]),
+        "infllm2_decode_block_idx_offset": (i64, [ctypes.POINTER(DecodeState), pp]),
         "infllm2_decode_build_caches": (ctypes.c_int, [ctypes.POINTER(DecodeState), pp, _P]),
         "infllm2_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeState), _P, _P, _P, _P, _P, ctypes.c_size_t, pp,
                                                 _P]),
@@ -294,6 +295,19 @@ def make_decode_state(k_cache: torch.Tensor, v_cache: torch.Tensor, k_c1: torch.
 
 def infllm2_decode_workspace_bytes(st: DecodeState, params: Optional[Params] = None) -> int:
     return int(lib().infllm2_decode_workspace_bytes(ctypes.byref(st), ctypes.byref(params or default_params())))
+
+
+def infllm2_decode_block_lists(st: DecodeState, workspace: torch.Tensor, params: Optional[Params] = None) -> torch.Tensor:
+    """View of the block lists the last decode step on `workspace` selected:
+    int32 [batch, h_kv, n_sel], ascending, -1 padded (read after the step)."""
+    params = params or default_params()
+    off = int(lib().infllm2_decode_block_idx_offset(ctypes.byref(st), ctypes.byref(params)))
+    if off < 0:
+        raise InfLLM2Error("infllm2_decode_block_idx_offset: invalid or unsupported decode state")
+    n = st.batch * st.h_kv * params.n_sel
+    if off + 4 * n > workspace.numel() * workspace.element_size():
+        raise InfLLM2Error("decode workspace smaller than its block lists")
+    return workspace.view(torch.uint8)[off:off + 4 * n].view(torch.int32).view(st.batch, st.h_kv, params.n_sel)
 
 
 def infllm2_decode_build_caches(st: DecodeState, params: Optional[Params] = None, stream=None) -> None:

@@ -27,7 +27,7 @@ NVCC_FLAGS = [
 
 
 def _sources():
-    out = [os.path.join(INCLUDE, "infllm2.h")]
+    out = [os.path.join(INCLUDE, f) for f in sorted(os.listdir(INCLUDE)) if f.endswith(".h")]
     for f in sorted(os.listdir(CSRC)):
         if f.endswith((".cu", ".cuh", ".h")):
             out.append(os.path.join(CSRC, f))

@@ -21,6 +21,7 @@
 #include "dense_attn.cu"
 #include "decode.cu"
 #include "probe.cu"
+#include "../../include/infllm2_measure.h"
 
 namespace infllm2 {
 
@@ -301,6 +302,12 @@ size_t infllm2_decode_workspace_bytes(const infllm2_decode_state* st, const infl
   if (check_decode_state(st) || check_params(p) || p->lse_mode != INFLLM2_LSE_APPROX) return 0;
   const DecodePlan P = plan_of(st, p);
   return decode_plan_supported(P) ? P.bytes : 0;
+}
+
+int64_t infllm2_decode_block_idx_offset(const infllm2_decode_state* st, const infllm2_params* p) {
+  if (check_decode_state(st) || check_params(p) || p->lse_mode != INFLLM2_LSE_APPROX) return -1;
+  const DecodePlan P = plan_of(st, p);
+  return decode_plan_supported(P) ? static_cast<int64_t>(P.off_idx) : -1;
 }
 
 int infllm2_decode_build_caches(const infllm2_decode_state* st, const infllm2_params* p, void* stream) {

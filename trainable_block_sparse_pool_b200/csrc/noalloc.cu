@@ -23,27 +23,21 @@ namespace infllm2 {
 // covers one 8192-token sequence (ld = 512), the longest the dense/sparse
 // switch keeps on the dense path by default, or any batch of that size.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static_assert(kNoAllocScratchBytes == INFLLM2_NOALLOC_SCRATCH_BYTES,
+              "the array's size is the limit the public header documents");
 
 static __device__ __align__(256) float g_noalloc_scores[kNoAllocScratchBytes / sizeof(float)];
 
 // Device address of g_noalloc_scores on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// with cudaGetSymbolAddress, once per device, with that device current.
+// with cudaGetSymbolAddress (which allocates nothing) with the device
+// current.  It is looked up on every call rather than cached, so a primary
+// context that was torn down and created again never leaves a stale address.
 static int noalloc_scratch(float** out) {
-  static std::mutex mu;
-  static float* addr[256] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scores);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= 256) return INFLLM2_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scores);
-    if (e != cudaSuccess) return cuda_fail(e);
-    addr[dev] = static_cast<float*>(p);
-  }
-  *out = addr[dev];
+  *out = static_cast<float*>(p);
   return INFLLM2_OK;
 }
 

@@ -174,6 +174,29 @@ __device__ __forceinline__ Unit get_unit(int64_t u, const SparseArgs& a) {
 
 __device__ __forceinline__ int ntiles_of(const Unit& x) { return (x.nvalid + 1) >> 1; }
 
+// Whole warp: does unit x's list have the form the split into a shared part
+// and a top-k part relies on?  Positions [0, i_hi) hold the init blocks
+// 0 .. i_hi-1, the next nvalid positions strictly ascending blocks in
+// [i_hi, l_start), the next ones the local run l_start .. b_t, and the rest
+// -1.  A list that breaks it is recorded as INFLLM2_ERR_DEVICE_BOUNDS (the
+// output of such a row is not the attention over its list).
+__device__ __forceinline__ void check_list_form(const Unit& x, const SparseArgs& a, int lane) {
+  const int32_t* list = x.I - min(a.n_init, (x.t >> 6) + 1);
+  const int bt = x.t >> 6;
+  const int i_hi = min(a.n_init, bt + 1);
+  const int l_start = max(i_hi, max(0, bt - a.n_local + 1));
+  const int e_loc = i_hi + x.nvalid, e_pad = e_loc + max(0, bt - l_start + 1);
+  bool bad = false;
+  for (int e = lane; e < a.n_sel; e += 32) {
+    const int v = __ldg(list + e);
+    if (e < i_hi) bad |= v != e;
+    else if (e < e_loc) bad |= v < i_hi || v >= l_start || (e > i_hi && v <= __ldg(list + e - 1));
+    else if (e < e_pad) bad |= v != l_start + (e - e_loc);
+    else bad |= v != -1;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
+}
+
 template <int D, int G, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -255,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         Le[w] = load_warp_list(x[w].I, x[w].nvalid, 0, lane);
         Lo[w] = load_warp_list(x[w].I, x[w].nvalid, 1, lane);
         if (isV) continue;
+        check_list_form(x[w], args, lane);
         const int qb = ucnt[w] & 1;
         int good = 1;
         if (lane == 0) {
