@@ -12,8 +12,12 @@ extra flush is needed between steps.
 Output: one JSON line (rank 0).  `value` is tokens/s over all ranks;
 `e2e` repeats the measurement through the public API with the inputs copied
 from pinned host memory and the output copied back inside the timed region;
-`roofline` describes the dominant kernel; `cpu_baseline` times the fp64
-oracle on a bounded sample of rows on the host cores.
+`roofline` describes the dominant kernel; `step_roofline` the whole step
+against the sum of its steps' bounds; `decode` the 16 x 131072 decode step
+(µs/step, fraction of HBM); `varlen` the packed 131072-token dense/sparse
+switch workload (tokens/s, dense and sparse time, the dense kernel's
+roofline); `cpu_baseline` times the fp64 oracle on a bounded sample of rows
+on all host cores the process may use, and on one core.
 
 `--impl reference` times the oracle alone (the reference arm for this build:
 there is no installable reference implementation; the pages carry no code).
@@ -88,16 +92,22 @@ def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
     # sparse attention: QK^T and PV over the visible selected keys
     w["sparse_flops"] = 4 * d * h_q * int(keys.sum())
     w["sparse_exps"] = h_q * int(keys.sum())
-    # K and V rows moved L2 -> SM: the top-k blocks of every (token, group),
-    # and the shared blocks once per CTA of 128/G tokens (the union over its
-    # tokens: one 64-token block's init and local blocks when 128/G <= 64)
-    tq = 128 // G
-    t0 = np.arange(0, n, tq)
-    b0 = t0 // 64
-    shared_blocks = np.minimum(1, b0 + 1) + np.maximum(0, b0 - np.maximum(np.minimum(1, b0 + 1), b0 - 31) + 1)
+    # K and V rows the attention must bring to the SMs (algorithmic): the
+    # top-k blocks of every (token, group), and the shared init and local
+    # blocks once per 64-token query block and group (they are the same for
+    # every token of the block)
+    def shared_blocks_at(b0):
+        i_hi = np.minimum(1, b0 + 1)
+        return i_hi + np.maximum(0, b0 - np.maximum(i_hi, b0 - 31) + 1)
+    qb = np.arange(0, (n + 63) // 64)
     w["sparse_topk_gather_bytes"] = h_kv * 2 * d * 2 * int(topk_keys.sum())
-    w["sparse_shared_gather_bytes"] = h_kv * 2 * d * 2 * 64 * int(shared_blocks.sum())
+    w["sparse_shared_gather_bytes"] = h_kv * 2 * d * 2 * 64 * int(shared_blocks_at(qb).sum())
     w["sparse_gather_bytes"] = w["sparse_topk_gather_bytes"] + w["sparse_shared_gather_bytes"]
+    # what the kernels move for the shared blocks: the LOCAL form reads them
+    # once per CTA of 128/G tokens (re-reads counted apart from the
+    # algorithmic bytes)
+    t0 = np.arange(0, n, max(1, 128 // G))
+    w["sparse_shared_gather_bytes_kernel"] = h_kv * 2 * d * 2 * 64 * int(shared_blocks_at(t0 // 64).sum())
     w["ld"] = ld
     return w
 
@@ -196,37 +206,62 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle baseline
-def oracle_sample(w, data, seconds: float, lse: str = "approx"):
-    """Time the fp64 oracle on rows of the workload until ~`seconds` of CPU
-    time: pooling of the whole sequence, then scores, selection and sparse
-    attention for uniformly sampled (token, group) rows.  Returns tokens/s
-    extrapolated to the full sequence, the rows done, and the threads used."""
-    try:
-        from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(limits=1)
-    except Exception:  # pragma: no cover
-        limiter = None
+def oracle_sequence(w, data, lse: str = "approx"):
+    """The fp64 oracle's sequence object (inputs converted, keys pooled) and
+    the seconds that took."""
     from oracle import infllm2_oracle as O
     p = O.Params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k, lse_mode=lse)
     t0 = time.perf_counter()
     seq = O.Sequence1(O.to_f64(data["Q"]), O.to_f64(data["K"]), O.to_f64(data["V"]), p)
-    t_pool = time.perf_counter() - t0
-    rng = np.random.default_rng(123)
-    n = seq.n
-    rows = 0
+    return seq, time.perf_counter() - t0
+
+
+def oracle_rows(seq, rows: int, seed: int) -> float:
+    """Scores, selection and sparse attention of the oracle for `rows`
+    uniformly sampled (token, group) rows; returns the seconds taken."""
+    rng = np.random.default_rng(seed)
     t1 = time.perf_counter()
-    while time.perf_counter() - t1 < seconds:
-        t = int(rng.integers(0, n))
+    for _ in range(rows):
+        t = int(rng.integers(0, seq.n))
         g = int(rng.integers(0, seq.h_kv))
-        sel = seq.select(t, g)
-        seq.sparse_out(t, g, sel)
-        rows += 1
-    t_rows = time.perf_counter() - t1
-    if limiter is not None:
-        limiter.unregister() if hasattr(limiter, "unregister") else None
+        seq.sparse_out(t, g, seq.select(t, g))
+    return time.perf_counter() - t1
+
+
+def oracle_sample(w, data, seconds: float, lse: str = "approx", threads: int = 1, seq=None):
+    """Time the fp64 oracle with NumPy/BLAS limited to `threads` threads:
+    pooling of the whole sequence, then rows sampled until ~`seconds`.
+    Returns tokens/s extrapolated to all rows of the sequence, the rows done,
+    the seconds spent, and the sequence object (reusable)."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        if seq is None:
+            seq, t_pool = oracle_sequence(w, data, lse)
+        else:
+            seq, t_pool = seq
+        rows, t_rows, seed = 0, 0.0, 123
+        while t_rows < seconds:
+            t_rows += oracle_rows(seq, 8, seed)
+            rows += 8
+            seed += 1
     per_row = t_rows / max(rows, 1)
-    total_s = t_pool + per_row * n * seq.h_kv
-    return n / total_s, rows, t_pool + t_rows
+    total_s = t_pool + per_row * seq.n * seq.h_kv
+    return seq.n / total_s, rows, t_pool + t_rows, (seq, t_pool)
+
+
+def cpu_baseline_entry(w, data, seconds: float, lse: str) -> dict:
+    """The oracle on every host core the process may use (BLAS threads =
+    len(sched_getaffinity)) and on one core, half of `seconds` each."""
+    ncores = len(os.sched_getaffinity(0))
+    tok_n, rows_n, secs_n, seq = oracle_sample(w, data, seconds / 2, lse, threads=ncores)
+    tok_1, rows_1, secs_1, _ = oracle_sample(w, data, seconds / 2, lse, threads=1, seq=seq)
+    return {"value": tok_n, "unit": "tokens/s", "cores": ncores, "kind": "oracle",
+            "sample": f"fp64 oracle, NumPy/BLAS threads = {ncores}: pooling of the whole {w.seqlen}-token sequence "
+                      f"({seq[1]:.1f} s) + {rows_n} uniformly sampled (token, group) rows ({secs_n:.1f} s in all), "
+                      f"extrapolated to all {w.seqlen * w.h_kv} rows",
+            "extrapolated": True,
+            "one_core": {"value": tok_1, "unit": "tokens/s", "cores": 1,
+                         "sample": f"same, 1 thread: {rows_1} rows ({secs_1 - seq[1]:.1f} s) + the same pooling"}}
 
 
 # ---------------------------------------------------------------- decode
@@ -435,7 +470,89 @@ def bench_decode(T, gen, torch, dev, graph_steps: int = 64, reps: int = 3, batch
             "device_status": status}
 
 
+def bench_varlen(T, gen, torch, dev, hbm: float, tflops_burst: float, reps: int = 5, warmup: int = 3,
+                 sm_mhz: float = 1965.0) -> dict:
+    """The dense/sparse switch on the packed 131072-token varlen workload:
+    sequences of at most 8192 tokens run the dense causal kernel (one call
+    over their packed batch), the others the sparse path (pool, scores,
+    top-k, sparse attention over their packed batch).  tokens/s = all packed
+    tokens / (dense time + sparse time), CUDA events on one stream."""
+    w = gen.WORKLOADS["varlen_128k"]
+    data = gen.make_prefill(w)
+    p = T.default_params(n_init=w.n_init, n_local=w.n_local, top_k=w.top_k)
+    lens = list(data["lens"])
+    cu = data["cu_seqlens"].tolist()
+    dense_ids = [i for i, n in enumerate(lens) if n <= p.dense_threshold]
+    sparse_ids = [i for i, n in enumerate(lens) if n > p.dense_threshold]
+
+    def sub(ids):
+        parts = {k: torch.cat([data[k][cu[i]:cu[i + 1]] for i in ids]).to(dev) for k in ("Q", "K", "V")}
+        ls = [lens[i] for i in ids]
+        c = torch.tensor([0] + list(np.cumsum(ls)), dtype=torch.int32, device=dev)
+        return parts, ls, c
+
+    stream = torch.cuda.current_stream()
+    dq, dl, dc = sub(dense_ids)
+    dvl = T.make_varlen(dl, dc, p)
+    dout = torch.empty(dvl.total, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
+    sq, sl, sc = sub(sparse_ids)
+    svl = T.make_varlen(sl, sc, p)
+    Kc1 = torch.empty(w.h_kv, svl.total_c1, w.d, dtype=torch.bfloat16, device=dev)
+    Kc2 = torch.empty(w.h_kv, svl.total_c2, w.d, dtype=torch.bfloat16, device=dev)
+    ld = T.infllm2_scores_ld(svl, p)
+    S = torch.empty(w.h_kv, svl.total, ld, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.h_kv, svl.total, p.n_sel, dtype=torch.int32, device=dev)
+    sout = torch.empty(svl.total, w.h_q, w.d, dtype=torch.bfloat16, device=dev)
+    sws = torch.empty(T.infllm2_sparse_workspace_bytes(svl, w.h_q), dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None: ev[0].record(stream)
+        T.infllm2_dense_attn(dq["Q"], dq["K"], dq["V"], dvl, dout, p, stream)
+        if ev is not None: ev[1].record(stream)
+        T.infllm2_compress_k(sq["K"], svl, Kc1, Kc2, p, stream)
+        T.infllm2_shared_scores(sq["Q"], Kc1, Kc2, svl, w.h_kv, S, ld, p, stream)
+        T.infllm2_topk_blocks(S, ld, svl, w.h_kv, idx, p, stream)
+        T.infllm2_sparse_attn(sq["Q"], sq["K"], sq["V"], idx, svl, sout, p, stream, workspace=sws)
+        if ev is not None: ev[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for k in range(reps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    t_dense = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    t_sparse = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    # the dense kernel's roofline: 4 d h_q flop and h_q exps per causal (t, u <= t) pair
+    pairs = sum(n * (n + 1) // 2 for n in dl)
+    flops = 4 * w.d * w.h_q * pairs
+    exps = w.h_q * pairs
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu = 16.0 * nsm * sm_mhz * 1e6
+    t_tensor, t_sfu = flops / (tflops_burst * 1e12), exps / sfu
+    dense_roof = {"bound": "tensor" if t_tensor >= t_sfu else "sfu", "flops": flops, "exps": exps,
+                  "achieved_TFLOP/s": flops / (t_dense / 1e3) / 1e12, "peak_TFLOP/s": tflops_burst,
+                  "frac_tensor": flops / (t_dense / 1e3) / 1e12 / tflops_burst,
+                  "roofline_ms": 1e3 * max(t_tensor, t_sfu), "frac": 1e3 * max(t_tensor, t_sfu) / t_dense,
+                  "peak_source": "MEASURED_PEAKS bf16 burst; ex2 at 16 per SM per clock"}
+    total = dvl.total + svl.total
+    status = T.infllm2_get_device_status()
+    return {"workload": w.name, "tokens": total, "sequences": len(lens), "dense_sequences": len(dense_ids),
+            "sparse_sequences": len(sparse_ids), "dense_tokens": dvl.total, "sparse_tokens": svl.total,
+            "ms_per_step": t_dense + t_sparse, "dense_ms": t_dense, "sparse_ms": t_sparse,
+            "tokens/s": total / ((t_dense + t_sparse) / 1e3), "dense_kernel_roofline": dense_roof,
+            "steps": reps, "warmup": warmup, "device_status": status}
+
+
 # ---------------------------------------------------------------- main
+def config_of(w, args, world: int) -> dict:
+    return {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
+            "n_sel": w.n_sel, "lse": args.lse, "pool": args.pool,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "working set larger than L2 (Q 1 GiB; S_shared 4.3 GB, or its pooled pairs 2.2 GB); no extra flush"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -443,10 +560,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed varlen dense/sparse switch workload")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
     ap.add_argument("--layer", action="store_true",
                     help="time one attention layer with random weights: sparse vs dense TTFT (128K prefill) and "
@@ -470,18 +588,37 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        # The oracle as it stands, on the host cores.  One step is a bounded
+        # sample of the workload: R uniformly sampled (token, group) rows
+        # (scores, selection, attention); the pooling of the whole sequence is
+        # timed once before the steps.  `value` extrapolates the per-row time
+        # to every row of the sequence plus the pooling; `ms_per_step` is the
+        # wall time of one sample step as actually run.
+        from threadpoolctl import threadpool_limits
+        ncores = len(os.sched_getaffinity(0))
         data = gen.make_prefill(w)
-        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds / max(1, args.steps) * args.steps, args.lse)
+        with threadpool_limits(limits=ncores):
+            seq, t_pool = oracle_sequence(w, data, args.lse)
+            probe = oracle_rows(seq, 8, 7) / 8
+            R = max(8, int(args.cpu_seconds / max(1, args.steps) / max(probe, 1e-4)))
+            for k in range(args.warmup):
+                oracle_rows(seq, max(1, R // 8), 1000 + k)
+            times = [oracle_rows(seq, R, 2000 + k) for k in range(args.steps)]
+        per_row = sum(times) / (R * args.steps)
+        tok_s = seq.n / (t_pool + per_row * seq.n * seq.h_kv)
+        sample = (f"fp64 oracle, NumPy/BLAS threads = {ncores}: {args.steps} steps of {R} uniformly sampled "
+                  f"(token, group) rows (warm-up steps of {max(1, R // 8)} rows), pooling of the whole "
+                  f"{w.seqlen}-token sequence timed once ({t_pool:.1f} s); extrapolated to all "
+                  f"{seq.n * seq.h_kv} rows")
         line = {
             "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.seqlen / tok_s,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+            "extrapolated": True, "rows_per_step": R, "ms_per_full_step_extrapolated": 1e3 * w.seqlen / tok_s,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q,
-                                             "h_kv": w.h_kv, "d": w.d, "n_sel": w.n_sel, "lse": args.lse,
-                                             "pool": args.pool, "parallelism": "single GPU"},
-            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"pooling of the whole sequence + {rows} sampled (token, group) rows, "
-                                       f"{secs:.1f} s, extrapolated to all rows"},
+            "data": "synthetic (seeded N(0,1) Q,V; K with per-block offsets)",
+            "config": config_of(w, args, 1),
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": ncores, "kind": "oracle", "sample": sample,
+                             "extrapolated": True},
             "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
         print(json.dumps(line), flush=True)
@@ -499,7 +636,10 @@ def main():
     T.lib()
 
     if args.layer:
+        clocks = ClockSampler()
+        clocks.start()
         res = bench_layer(T, gen, torch, dev)
+        res["clocks"] = clocks.stop()
         if rank == 0:
             print(json.dumps({"layer": res}), flush=True)
         return
@@ -611,17 +751,20 @@ def main():
         work["score_bytes"], work["topk_bytes"] = work["score_bytes_pooled"], work["topk_bytes_pooled"]
     dom = max(per_kernel, key=per_kernel.get)
     if dom == "sparse":
-        # the top-k gather (and the shared tiles) are L2 -> SM bound: see the design doc
+        # the attention is bound by moving the selected K/V rows from L2 to
+        # the SMs: algorithmic bytes = the top-k blocks per (token, group) +
+        # the shared init/local blocks once per 64-token query block and group
         ach = work["sparse_gather_bytes"] / (per_kernel["sparse"] / 1e3) / 1e9
-        # DRAM bytes of the step's two sparse kernels (top-k and LOCAL), read
-        # and written, from one ncu capture of the 32K workload (327 + 230 MB and
-        # 562 + 228 MB), scaled by tokens: Q, the output and the partials
-        # grow with them, while the K/V gather stays in L2
-        traffic = (327.0 + 230.0 + 561.9 + 228.3) * 1e6 * (w.seqlen / 32768) if w.name.startswith("prefill_") else None
+        tflop = work["sparse_flops"] / (per_kernel["sparse"] / 1e3) / 1e12
         roof = {"kernel": "sparse_attn (top-k gather + shared init/local tiles)", "bound": "l2", "achieved": ach,
-                "peak": l2["GB/s"], "unit": "GB/s", "frac": ach / l2["GB/s"], "traffic": traffic,
-                "traffic_source": "DRAM read + write per step of the two sparse kernels, ncu at 32K scaled by tokens",
-                "peak_source": "L2 gather probe, same tile shape, same run (measured)"}
+                "peak": l2["GB/s"], "unit": "GB/s", "frac": ach / l2["GB/s"], "traffic": None,
+                "algorithmic_bytes": work["sparse_gather_bytes"],
+                "kernel_gather_bytes": work["sparse_topk_gather_bytes"] + work["sparse_shared_gather_bytes_kernel"],
+                "peak_source": "L2 -> SM gather bandwidth measured in this run by the library's own probe "
+                               "(infllm2_probe_l2_gather, same tile shape); no driver-measured L2 figure exists",
+                "tensor": {"achieved": tflop, "peak": tflops, "unit": "TFLOP/s", "frac": tflop / tflops,
+                           "peak_source": f"{src} bf16 burst (MEASURED_PEAKS)"},
+                "hbm_traffic_note": "DRAM bytes come from ncu captures, summarised under profiles/"}
     elif dom == "scores":
         ach = work["score_flops"] / (per_kernel["scores"] / 1e3) / 1e12
         roof = {"kernel": "shared_scores", "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
@@ -672,10 +815,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q,V; K with per-block offsets)",
-        "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
-                   "n_sel": w.n_sel, "lse": args.lse, "pool": args.pool,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "working set larger than L2 (Q 1 GiB; S_shared 4.3 GB, or its pooled pairs 2.2 GB); no extra flush"},
+        "config": config_of(w, args, world),
         "e2e": e2e,
         "gpu_launches": (len(kernels) + 1) * args.steps,   # the sparse call is two launches (local + top-k)
         "kernels": kern_detail,
@@ -691,11 +831,11 @@ def main():
         dd["frac"] = dd["achieved_GB/s"] / hbm
         dd["bound"] = "hbm"
         line["decode"] = dd
+    if not args.no_varlen:
+        line["varlen"] = bench_varlen(T, gen, torch, dev, hbm, tflops, sm_mhz=sm_mhz)
+        line["gpu_launches_varlen_step"] = 6   # dense; compress, scores, top-k, sparse (two launches)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, rows, secs = oracle_sample(w, data, args.cpu_seconds, args.lse)
-        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"pooling of the whole 128K sequence + {rows} uniformly sampled "
-                                          f"(token, group) rows ({secs:.1f} s), extrapolated to all rows"}
+        line["cpu_baseline"] = cpu_baseline_entry(w, data, args.cpu_seconds, args.lse)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
