@@ -545,6 +545,45 @@ def bench_varlen(T, gen, torch, dev, hbm: float, tflops_burst: float, reps: int 
             "steps": reps, "warmup": warmup, "device_status": status}
 
 
+def bench_backward(T, gen, torch, dev, w, data, p, Q, K, V, idx, out, sws, vl, stream, reps: int = 3,
+                   warmup: int = 2, tflops: float = 1694.5) -> dict:
+    """The backward of the block-sparse attention on the bench workload (the
+    forward's lists, output and row log-sum-exps from the timed step): dQ, dK,
+    dV in fp32.  ms per backward call, CUDA events on the launching stream."""
+    total = vl.total
+    lse = sws[: total * w.h_q * 4].view(torch.float32).view(total, w.h_q)
+    dout = gen.make_grad_out(total, w.h_q, w.d, 7).to(dev)
+    ws = torch.empty(T.infllm2_sparse_backward_workspace_bytes(vl, w.h_q, w.h_kv, p), dtype=torch.uint8, device=dev)
+    dQ = torch.empty(total, w.h_q, w.d, dtype=torch.float32, device=dev)
+    dK = torch.empty(total, w.h_kv, w.d, dtype=torch.float32, device=dev)
+    dV = torch.empty_like(dK)
+
+    def step():
+        T.infllm2_sparse_attn_backward(Q, K, V, out, dout, lse, idx, vl, dQ, dK, dV, ws, p, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = statistics.median(ts)
+    # contractions: dQ pass 3 products and dK/dV pass 4 products of 2 d flop
+    # per (row, attended key): S, dP, dQ / S, dP, dV, dK
+    n1, n2, keys, shared_keys, topk_keys = visible_counts(w.seqlen, w.n_init, w.n_local, w.top_k)
+    flops = (3 + 4) * 2 * w.d * w.h_q * int(keys.sum())
+    status = T.infllm2_get_device_status()
+    del ws, dQ, dK, dV, dout
+    return {"workload": w.name, "ms": ms, "tokens/s": total / (ms / 1e3), "launches": 8,
+            "flops": flops, "TFLOP/s": flops / (ms / 1e3) / 1e12, "frac_tensor": flops / (ms / 1e3) / 1e12 / tflops,
+            "peak_source": "MEASURED_PEAKS bf16 burst", "outputs": "dQ, dK, dV fp32", "device_status": status}
+
+
 # ---------------------------------------------------------------- main
 def config_of(w, args, world: int) -> dict:
     return {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
@@ -565,6 +604,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed varlen dense/sparse switch workload")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward (dQ, dK, dV) timing")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode workload (for profiling)")
     ap.add_argument("--layer", action="store_true",
                     help="time one attention layer with random weights: sparse vs dense TTFT (128K prefill) and "
@@ -817,7 +857,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q,V; K with per-block offsets)",
         "config": config_of(w, args, world),
         "e2e": e2e,
-        "gpu_launches": (len(kernels) + 1) * args.steps,   # the sparse call is two launches (local + top-k)
+        "gpu_launches": (len(kernels) + 2) * args.steps,   # the sparse call is three launches (list check, top-k, local)
         "kernels": kern_detail,
         "roofline": roof,
         "step_roofline": step_roof,
@@ -831,9 +871,12 @@ def main():
         dd["frac"] = dd["achieved_GB/s"] / hbm
         dd["bound"] = "hbm"
         line["decode"] = dd
+    if not args.no_backward:
+        line["backward"] = bench_backward(T, gen, torch, dev, w, data, p, Q, K, V, idx, out, sws, vl, stream,
+                                          tflops=tflops)
     if not args.no_varlen:
         line["varlen"] = bench_varlen(T, gen, torch, dev, hbm, tflops, sm_mhz=sm_mhz)
-        line["gpu_launches_varlen_step"] = 6   # dense; compress, scores, top-k, sparse (two launches)
+        line["gpu_launches_varlen_step"] = 7   # dense; compress, scores, top-k, sparse (three launches)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_entry(w, data, args.cpu_seconds, args.lse)
     if rank == 0:

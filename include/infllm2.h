@@ -239,13 +239,53 @@ int infllm2_select_blocks_noalloc(const void* Q, const void* K_c1, const void* K
  * (no fault, no out-of-range read).
  * workspace: device, 16-byte aligned, at least
  * infllm2_sparse_workspace_bytes(vl, h_q) bytes (one fp32 per (token,
- * query head)); nothing in it outlives the call's kernels.
+ * query head)).  When the call's kernels have completed, its first
+ * total * h_q floats hold, for every token row t and query head h (index
+ * t * h_q + h), the row's log-sum-exp in log2 units over the keys it
+ * attended: lse = log2 sum_u 2^(scale * log2(e) * q[t,h] . K[u,g]) — the
+ * statistic infllm2_sparse_attn_backward takes.
  * ------------------------------------------------------------------- */
 size_t infllm2_sparse_workspace_bytes(const infllm2_varlen* vl, int32_t h_q);
 int infllm2_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* block_idx,
                         const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d,
                         void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
                         const infllm2_params* p, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Backward of step 4: gradients of the block-sparse attention over a fixed
+ * selection (the method trains the sparse attention end to end with no added
+ * parameters: [news] §二, [top168] §一; [blog] "训练是怎么做的").  The block
+ * lists carry no gradient.  For row (t, h) of kv group g and its attended
+ * keys u (those infllm2_sparse_attn attends), with P = softmax_u(scale *
+ * q[t,h] . K[u,g]) and dS = P * (dO[t,h] . V[u,g] - sum_d dO[t,h] * out[t,h]):
+ *   dQ[t,h] = scale * sum_u dS K[u,g]
+ *   dK[u,g] = scale * sum over rows (t,h) that attend u of dS q[t,h]
+ *   dV[u,g] = sum over rows (t,h) that attend u of P dO[t,h]
+ *   Q, K, V, block_idx, vl, h_q, h_kv, d, p: as given to infllm2_sparse_attn
+ *   out        its output [total, h_q, d], out_dtype INFLLM2_OUT_BF16 / _F32
+ *   dout       bf16 [total, h_q, d], the gradient of the loss w.r.t. out
+ *   lse        fp32 [total, h_q]: the first total * h_q floats of
+ *              infllm2_sparse_attn's workspace after that call (row
+ *              log-sum-exps, log2 units)
+ *   dQ         fp32 [total, h_q, d]   (output, every element written)
+ *   dK, dV     fp32 [total, h_kv, d]  (output, every element written)
+ *   workspace  device, at least infllm2_sparse_backward_workspace_bytes
+ *              bytes (per-row sums, the inverse of the block lists); its
+ *              contents need no initialisation and carry nothing between
+ *              calls.
+ * Supported: G = h_q / h_kv of 8 or 16, d of 64 or 128 (other shapes:
+ * INFLLM2_ERR_UNSUPPORTED).  Lists must have the form infllm2_sparse_attn
+ * requires; a list that breaks it is recorded as INFLLM2_ERR_DEVICE_BOUNDS.
+ * The result does not depend on scheduling: each key block's gradient is
+ * summed by one CTA over its rows in ascending token order.
+ * ------------------------------------------------------------------- */
+size_t infllm2_sparse_backward_workspace_bytes(const infllm2_varlen* vl, int32_t h_q, int32_t h_kv,
+                                               const infllm2_params* p);
+int infllm2_sparse_attn_backward(const void* Q, const void* K, const void* V, const void* out, int32_t out_dtype,
+                                 const void* dout, const float* lse, const int32_t* block_idx,
+                                 const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d, float* dQ, float* dK,
+                                 float* dV, void* workspace, size_t workspace_bytes, const infllm2_params* p,
+                                 void* stream);
 
 /* Dense causal attention, the short-sequence side of the dense/sparse switch
  * ([blog] "Dense-Sparse Switchable Attention"; [news] §二.2.c).  Same

@@ -174,3 +174,10 @@ def sample_rows(total: int, count: int, seed: int) -> np.ndarray:
     rng = np.random.Generator(np.random.PCG64(seed))
     count = min(count, total)
     return np.sort(rng.choice(total, size=count, replace=False))
+
+
+def make_grad_out(total: int, h_q: int, d: int, seed: int) -> torch.Tensor:
+    """A seeded upstream gradient dO [total, h_q, d] ~ N(0,1), bf16 (the
+    backward's input; random draws only)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return to_bf16(rng.standard_normal((total, h_q, d), dtype=np.float32))

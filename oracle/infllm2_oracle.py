@@ -354,6 +354,31 @@ def key_block_gradients(Q: np.ndarray, K: np.ndarray, V: np.ndarray, blocks: np.
     return dK, dV
 
 
+def block_rows(blocks: np.ndarray, g: int, kb: int) -> np.ndarray:
+    """The tokens t whose selection blocks[t, g] holds block kb, ascending."""
+    return np.nonzero((blocks[:, g, :] == kb).any(axis=1))[0]
+
+
+def one_block_gradients(Q: np.ndarray, K: np.ndarray, V: np.ndarray, blocks: np.ndarray, dO: np.ndarray,
+                        p: "Params", g: int, kb: int):
+    """dK and dV of the 64 keys of block kb of group g alone ([B, d] each,
+    fewer rows for a partial last block): key_block_gradients() for one
+    block, for checks that cannot afford every block."""
+    n, h_q, d = Q.shape
+    G = h_q // K.shape[1]
+    scale = p.softmax_scale(d)
+    lo, hi = kb * p.block, min(n, kb * p.block + p.block)
+    hs = slice(g * G, (g + 1) * G)
+    dk, dv = np.zeros((hi - lo, d)), np.zeros((hi - lo, d))
+    for t in block_rows(blocks, g, kb):
+        keys = sparse_keys(int(t), blocks[t, g], p.block)
+        _, dkr, dvr = attend_backward(Q[t, hs], K[:, g], V[:, g], keys, dO[t, hs], scale)
+        mine = (keys >= lo) & (keys < hi)
+        dk[keys[mine] - lo] += dkr[mine]
+        dv[keys[mine] - lo] += dvr[mine]
+    return dk, dv
+
+
 # ----------------------------------------------------------------------------
 # per-sequence drivers
 # ----------------------------------------------------------------------------

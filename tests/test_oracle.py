@@ -504,3 +504,25 @@ def test_decode_row_is_row_t_of_the_prefill_rule():
     _, o1, _, _, _ = O.decode_row(full.K[:t + 1], full.V[:t + 1], full.Q[t], p)
     _, o2, _, _, _ = O.decode_row(full.K[:t + 1], V2, full.Q[t], p)
     assert np.abs(o1 - o2).min() > 0
+
+
+def test_one_block_gradients_equal_the_key_block_form():
+    # the per-block form used by sampled GPU checks equals the key-block-major
+    # form over all blocks, block by block
+    p = O.Params(n_init=1, n_local=2, top_k=2)
+    rng = np.random.default_rng(31)
+    n, h_q, h_kv, d = 330, 4, 2, 8
+    Q = _bf16(rng.standard_normal((n, h_q, d)))
+    K = _bf16(rng.standard_normal((n, h_kv, d)))
+    V = _bf16(rng.standard_normal((n, h_kv, d)))
+    dO = rng.standard_normal((n, h_q, d))
+    blocks = _random_selection(rng, n, h_kv, p.n_sel)
+    dK, dV = O.key_block_gradients(Q, K, V, blocks, dO, p)
+    for g in range(h_kv):
+        for kb in range((n + 63) // 64):
+            dk, dv = O.one_block_gradients(Q, K, V, blocks, dO, p, g, kb)
+            lo = 64 * kb
+            np.testing.assert_allclose(dk, dK[lo:lo + dk.shape[0], g], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(dv, dV[lo:lo + dv.shape[0], g], rtol=1e-12, atol=1e-12)
+    rows = O.block_rows(blocks, 0, 1)
+    assert all(1 in blocks[t, 0] for t in rows) and len(rows) == sum(1 in blocks[t, 0] for t in range(n))

@@ -100,6 +100,9 @@ def lib() -> ctypes.CDLL:
         "infllm2_sparse_attn": (ctypes.c_int, [_P, _P, _P, _P, vp, i32, i32, i32, _P, i32, _P, ctypes.c_size_t, pp,
                                                 _P]),
         "infllm2_dense_attn": (ctypes.c_int, [_P, _P, _P, vp, i32, i32, i32, _P, i32, pp, _P]),
+        "infllm2_sparse_backward_workspace_bytes": (ctypes.c_size_t, [vp, i32, i32, pp]),
+        "infllm2_sparse_attn_backward": (ctypes.c_int, [_P, _P, _P, _P, i32, _P, _P, _P, vp, i32, i32, i32, _P, _P, _P,
+                                                         _P, ctypes.c_size_t, pp, _P]),
         "infllm2_get_device_status": (ctypes.c_int, []),
         "infllm2_clear_device_status": (ctypes.c_int, []),
         "infllm2_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
@@ -248,6 +251,27 @@ def infllm2_sparse_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block
                                    _ptr(out), od, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    ctypes.byref(params or default_params()), _stream(stream))
     _check("infllm2_sparse_attn", rc)
+
+
+def infllm2_sparse_backward_workspace_bytes(vl: Varlen, h_q: int, h_kv: int, params: Optional[Params] = None) -> int:
+    return int(lib().infllm2_sparse_backward_workspace_bytes(ctypes.byref(vl), h_q, h_kv,
+                                                             ctypes.byref(params or default_params())))
+
+
+def infllm2_sparse_attn_backward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, out: torch.Tensor,
+                                 dout: torch.Tensor, lse: torch.Tensor, block_idx: torch.Tensor, vl: Varlen,
+                                 dQ: torch.Tensor, dK: torch.Tensor, dV: torch.Tensor, workspace: torch.Tensor,
+                                 params: Optional[Params] = None, stream=None) -> None:
+    """Gradients of the block-sparse attention (fp32 dQ, dK, dV).  `lse`: fp32 [total, h_q], the first
+    total * h_q floats of the workspace infllm2_sparse_attn used."""
+    h_q, d = Q.shape[1], Q.shape[2]
+    h_kv = K.shape[1]
+    od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    rc = lib().infllm2_sparse_attn_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(out), od, _ptr(dout), _ptr(lse),
+                                            _ptr(block_idx), ctypes.byref(vl), h_q, h_kv, d, _ptr(dQ), _ptr(dK),
+                                            _ptr(dV), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                            ctypes.byref(params or default_params()), _stream(stream))
+    _check("infllm2_sparse_attn_backward", rc)
 
 
 def infllm2_probe_l2_gather(K: torch.Tensor, V: torch.Tensor, nblk: int, tiles: int, producers: int,

@@ -51,19 +51,20 @@ def needs_build() -> bool:
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/infllm2.cu into libinfllm2.so next to this file."""
-    if not force and not needs_build():
+def build(force: bool = False, verbose: bool = False, out: str = LIB_PATH, defines=()) -> str:
+    """Compile csrc/infllm2.cu into libinfllm2.so next to this file (or into
+    `out`, with extra -D `defines`)."""
+    if out == LIB_PATH and not defines and not force and not needs_build():
         return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, os.path.join(CSRC, "infllm2.cu"), "-o", tmp]
+    tmp = out + ".tmp"
+    cmd = [_nvcc(), *NVCC_FLAGS, *[f"-D{d}" for d in defines], os.path.join(CSRC, "infllm2.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

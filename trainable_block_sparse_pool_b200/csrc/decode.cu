@@ -574,10 +574,20 @@ __device__ void select_blocks_cta(const float* row, int t, int n_init, int n_loc
 // conflicts.
 // A completion counter per (b, g) counts the pieces done; the CTA that
 // completes the last one runs that selection once its range is done.
-constexpr int kPieceWin = 128;                  // stage-1 windows per piece
+#ifndef INFLLM2_DEC_PIECE
+#define INFLLM2_DEC_PIECE 128
+#endif
+#ifndef INFLLM2_DEC_STAGES
+#define INFLLM2_DEC_STAGES 2
+#endif
+#ifndef INFLLM2_DEC_EARLY
+#define INFLLM2_DEC_EARLY 0
+#endif
+constexpr int kPieceWin = INFLLM2_DEC_PIECE;    // stage-1 windows per piece
 constexpr int kPieceBlk = kPieceWin / 4;        // blocks per piece
 constexpr int kPieceRows = kPieceWin + 8;       // the n-tile before the piece, then the piece
-constexpr int kScoreStages = 2;
+constexpr int kScoreStages = INFLLM2_DEC_STAGES;
+static_assert(kPieceBlk <= 32 && (kPieceRows * 128) % 1024 == 0, "piece geometry");
 constexpr int kMaxRange = 64;                   // pieces per CTA at most (the host sizes the grid)
 
 template <int D>
@@ -706,8 +716,14 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     __syncthreads();
     if (aligned) R = s_R;
   }
-  // the mapping read only seq_len; the pooled keys and the LSE partials come from the append kernel
-  griddep_wait();
+  // The mapping read only seq_len; the LSE partials (and the completion
+  // counters) come from the append kernel.  The stage-1 windows the
+  // selection reads do not: the only window the append kernel may pool ends
+  // at t, and with n_local >= 2 it lies past the pooling range of every
+  // candidate block (4(b_t - n_local) + 3 < (t - 31) / 16), so the first
+  // pieces' copies can go out before the wait and overlap the append kernel.
+  const bool early = INFLLM2_DEC_EARLY && n_local >= 2;
+  if (!early) griddep_wait();
   if (R <= 0) return;
   auto bg_of = [&](int j) { return static_cast<int>(plist[j] >> 16); };
   auto p_of = [&](int j) { return static_cast<int>(plist[j] & 0xffffu); };
@@ -780,6 +796,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
 
 #pragma unroll
   for (int s = 0; s < kScoreStages - 1; ++s) stage(s);
+  if (early) griddep_wait();
   if (pnp[0] > 0) group_lse(0);
   QFrag<D> f;
   {

@@ -331,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
     xch[512 + r * 2 + hf] = l_run;
     bar_red_or(pair, 64, false);
     const float l_row = l_run + xch[512 + r * 2 + (hf ^ 1)];
+    float lse_row = -INFINITY;                    // LOCAL: the row's log-sum-exp over all its keys (log2 units)
     if (ok && t < len) {
       const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
       const int64_t base = (static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h) * D + hf * DH;
@@ -340,13 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
         // out[row] holds the top-k partial (normalised) when its log-sum-exp
         // lb (log2 units) is finite; la is this partial's
         const float lb = lse[static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h];
+        const float la = (l_row > 0.f) ? m_run + log2f(l_row) : -INFINITY;
+        lse_row = la;
         if (lb != -INFINITY && l_row > 0.f) {
-          const float la = m_run + log2f(l_row);
           const float mm = fmaxf(la, lb);
           const float wa = ex2(la - mm), wb = ex2(lb - mm);
           const float iw = 1.f / (wa + wb);
           w_own = inv * wa * iw;
           w_top = wb * iw;
+          lse_row = mm + log2f(wa + wb);
         }
       }
       if (OUT_F32) {
@@ -388,6 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1) dense_attn_kernel(
           o4[j / 8] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+    }
+    if (LOCAL) {
+      // both threads of the row have read the top-k log-sum-exp: the slot
+      // now takes the row's complete one (the statistic a backward pass
+      // needs: P = 2^(scale log2(e) q.k - lse))
+      bar_red_or(pair, 64, false);
+      if (hf == 0 && ok && t < len)
+        lse[static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h] = lse_row;
     }
   }
 

@@ -20,6 +20,7 @@
 #include "sparse_attn.cu"
 #include "dense_attn.cu"
 #include "decode.cu"
+#include "backward.cu"
 #include "probe.cu"
 #include "../../include/infllm2_measure.h"
 
@@ -280,6 +281,52 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V, const infllm
   cudaError_t e = launch_dense_attn(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d,
                                     softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32, 0, 0, nullptr,
                                     static_cast<cudaStream_t>(stream), &map_fail);
+  if (map_fail) return INFLLM2_ERR_INVALID_ARG;
+  return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
+}
+
+size_t infllm2_sparse_backward_workspace_bytes(const infllm2_varlen* vl, int32_t h_q, int32_t h_kv,
+                                               const infllm2_params* p) {
+  if (check_varlen(vl) || check_params(p) || h_q <= 0 || h_kv <= 0) return 0;
+  const BwdPlan P = bwd_plan(vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, p->n_init + p->n_local + p->top_k);
+  return P.bytes;
+}
+
+int infllm2_sparse_attn_backward(const void* Q, const void* K, const void* V, const void* out, int32_t out_dtype,
+                                 const void* dout, const float* lse, const int32_t* block_idx,
+                                 const infllm2_varlen* vl, int32_t h_q, int32_t h_kv, int32_t d, float* dQ, float* dK,
+                                 float* dV, void* workspace, size_t workspace_bytes, const infllm2_params* p,
+                                 void* stream) {
+  int r;
+  if ((r = check_varlen(vl)) || (r = check_params(p)) || (r = check_heads(h_q, h_kv, d))) return r;
+  const void* ptrs[] = {Q, K, V, out, dout, lse, block_idx, dQ, dK, dV, workspace};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return INFLLM2_ERR_INVALID_ARG;
+  if (out_dtype != INFLLM2_OUT_BF16 && out_dtype != INFLLM2_OUT_F32) return INFLLM2_ERR_INVALID_ARG;
+  const int G = h_q / h_kv;
+  if (G != 8 && G != 16) return INFLLM2_ERR_UNSUPPORTED;
+  const int n_sel = p->n_init + p->n_local + p->top_k;
+  const BwdPlan P = bwd_plan(vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, n_sel);
+  if (static_cast<int64_t>(h_kv) * vl->total * n_sel > INT32_MAX ||
+      static_cast<int64_t>(h_kv) * vl->batch * P.nb_max > (int64_t(1) << 24))
+    return INFLLM2_ERR_UNSUPPORTED;
+  if (workspace_bytes < P.bytes) return INFLLM2_ERR_WORKSPACE_TOO_SMALL;
+  if (vl->total == 0) return INFLLM2_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the lists' form first (recorded in the device status word when broken)
+  {
+    sparse::SparseArgs a{};
+    a.block_idx = block_idx; a.cu = vl->cu_seqlens; a.batch = vl->batch; a.total = vl->total; a.h_q = h_q;
+    a.h_kv = h_kv; a.n_sel = n_sel; a.n_init = p->n_init; a.n_local = p->n_local;
+    const int64_t warps = static_cast<int64_t>(h_kv) * vl->total;
+    const int64_t grid = std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(num_sms()) * 8);
+    sparse::check_lists_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(a);
+  }
+  bool map_fail = false;
+  cudaError_t e = launch_sparse_backward(Q, K, V, out, out_dtype == INFLLM2_OUT_F32, dout, lse, block_idx,
+                                         vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d, n_sel,
+                                         p->n_init, p->n_local, softmax_scale(p, d), dQ, dK, dV, workspace, P, st,
+                                         &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }

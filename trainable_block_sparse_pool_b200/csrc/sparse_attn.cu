@@ -174,25 +174,41 @@ __device__ __forceinline__ Unit get_unit(int64_t u, const SparseArgs& a) {
 
 __device__ __forceinline__ int ntiles_of(const Unit& x) { return (x.nvalid + 1) >> 1; }
 
-// Whole warp: does unit x's list have the form the split into a shared part
-// and a top-k part relies on?  Positions [0, i_hi) hold the init blocks
-// 0 .. i_hi-1, the next nvalid positions strictly ascending blocks in
-// [i_hi, l_start), the next ones the local run l_start .. b_t, and the rest
-// -1.  A list that breaks it is recorded as INFLLM2_ERR_DEVICE_BOUNDS (the
-// output of such a row is not the attention over its list).
-__device__ __forceinline__ void check_list_form(const Unit& x, const SparseArgs& a, int lane) {
-  const int32_t* list = x.I - min(a.n_init, (x.t >> 6) + 1);
-  const int bt = x.t >> 6;
-  const int i_hi = min(a.n_init, bt + 1);
-  const int l_start = max(i_hi, max(0, bt - a.n_local + 1));
-  const int e_loc = i_hi + x.nvalid, e_pad = e_loc + max(0, bt - l_start + 1);
+// Does every list have the form the split into a shared part and a top-k
+// part relies on?  One warp per unit (kv group, packed row): positions
+// [0, i_hi) hold the init blocks 0 .. i_hi-1, the next nvalid positions
+// strictly ascending blocks in [i_hi, l_start), the next ones the local run
+// l_start .. b_t, and the rest -1.  A list that breaks it is recorded as
+// INFLLM2_ERR_DEVICE_BOUNDS (the output of such a row is not the attention
+// over its list).  Runs before the attention kernels, off their critical
+// path: 4 bytes per list entry, read once.
+__global__ void __launch_bounds__(256) check_lists_kernel(const SparseArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n_units = num_units(a);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   bool bad = false;
-  for (int e = lane; e < a.n_sel; e += 32) {
-    const int v = __ldg(list + e);
-    if (e < i_hi) bad |= v != e;
-    else if (e < e_loc) bad |= v < i_hi || v >= l_start || (e > i_hi && v <= __ldg(list + e - 1));
-    else if (e < e_pad) bad |= v != l_start + (e - e_loc);
-    else bad |= v != -1;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < n_units;
+       u += stride) {
+    const Unit x = get_unit(u, a);
+    const int32_t* list = a.block_idx + u * a.n_sel;
+    const int bt = x.t >> 6;
+    const int i_hi = min(a.n_init, bt + 1);
+    const int l_start = max(i_hi, max(0, bt - a.n_local + 1));
+    const int e_loc = i_hi + x.nvalid, e_pad = e_loc + max(0, bt - l_start + 1);
+    int carry = -1;                            // entry 32 r - 1 (the previous round's lane 31)
+    for (int e0 = 0; e0 < a.n_sel; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = (e < a.n_sel) ? __ldg(list + e) : -1;
+      int prev = __shfl_up_sync(0xffffffffu, v, 1);
+      if (lane == 0) prev = carry;
+      carry = __shfl_sync(0xffffffffu, v, 31);
+      if (e < a.n_sel) {
+        if (e < i_hi) bad |= v != e;
+        else if (e < e_loc) bad |= v < i_hi || v >= l_start || (e > i_hi && v <= prev);
+        else if (e < e_pad) bad |= v != l_start + (e - e_loc);
+        else bad |= v != -1;
+      }
+    }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(INFLLM2_ERR_DEVICE_BOUNDS);
 }
@@ -278,7 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         Le[w] = load_warp_list(x[w].I, x[w].nvalid, 0, lane);
         Lo[w] = load_warp_list(x[w].I, x[w].nvalid, 1, lane);
         if (isV) continue;
-        check_list_form(x[w], args, lane);
         const int qb = ucnt[w] & 1;
         int good = 1;
         if (lane == 0) {
@@ -641,6 +656,11 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
   a.block_idx = idx; a.cu = cu; a.batch = batch; a.total = total; a.h_q = h_q; a.h_kv = h_kv; a.n_sel = n_sel;
   a.n_init = n_init; a.n_local = n_local; a.scale = scale; a.out = out; a.lse = lse;
   const int G = h_q / h_kv;
+  if (total > 0) {
+    const int64_t warps = static_cast<int64_t>(h_kv) * total;
+    const int64_t grid = std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(num_sms()) * 8);
+    sparse::check_lists_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(a);
+  }
 #define INFLLM2_SPARSE_CASE(DD, GG)                                                            \
   if (d == DD && G == GG)                                                                     \
     return out_f32 ? launch_sparse_t<DD, GG, true>(Q, K, V, total, a, st, map_fail)           \
