@@ -171,10 +171,19 @@ class ClockSampler:
             sel = []
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200", *sel],
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "50", *sel],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: wait for its first sample so the
+        # timed region that follows is covered from its start
+        t0 = time.time()
+        while time.time() - t0 < 10.0:
+            with open(self.path) as f:
+                if f.read().count("\n") >= 1:
+                    break
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -595,7 +604,7 @@ def config_of(w, args, world: int) -> dict:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
@@ -733,10 +742,10 @@ def main():
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler()
+    clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
