@@ -263,8 +263,9 @@ __global__ void __launch_bounds__(256) fill_kernel(const Args a) {
 }
 
 // ---------------------------------------------------------------- dQ: per (kv group, token)
-constexpr int kQThreads = 224;       // warp 0 K/Q/dO producer, 1 MMA, 2-5 softmax, 6 V producer
+constexpr int kQThreads = 256;       // warp 0 K/Q/dO producer, 1 S/dP MMA, 2-5 softmax, 6 V producer, 7 dQ MMA
 constexpr int kQVWarp = 6;
+constexpr int kQDqWarp = 7;
 
 template <int D>
 struct QCfg {
@@ -286,7 +287,7 @@ struct QBars {
   uint64_t s_full[2], s_empty[2];
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_empty[2];
-  uint64_t mma_done;
+  uint64_t mma_done, dq_done;      // each MMA issuer's own products have completed
   uint32_t tmem_base;
   int abort;
 };
@@ -307,7 +308,16 @@ __device__ __forceinline__ QUnit q_unit(int64_t u, const Args& a) {
   x.t = static_cast<int>(x.row - x.row0);
   x.I = a.block_idx + u * a.n_sel;
   int nv = 0;
-  for (int i = 0; i < a.n_sel; ++i) nv += (__ldg(x.I + i) >= 0);
+  if ((a.n_sel & 3) == 0) {                 // rows of n_sel ints start 16-byte aligned
+    const int4* I4 = reinterpret_cast<const int4*>(x.I);
+#pragma unroll 8
+    for (int i = 0; i < a.n_sel / 4; ++i) {
+      const int4 v = __ldg(I4 + i);
+      nv += (v.x >= 0) + (v.y >= 0) + (v.z >= 0) + (v.w >= 0);
+    }
+  } else {
+    for (int i = 0; i < a.n_sel; ++i) nv += (__ldg(x.I + i) >= 0);
+  }
   x.nvalid = nv;
   return x;
 }
@@ -349,6 +359,7 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
       mbar_init(&bars->dq_empty[i], 4);
     }
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->dq_done, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -404,43 +415,22 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
         for (int i = max(0, uc - 2); i < uc; ++i) mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S / dP issuer
+    // per tile: S^T = K_pair Q^T and dP^T = V_pair dO^T; the V slot is free
+    // once dP is done, the K slot only after the dQ product (warp 7)
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 16, 0, 0);
-      const uint32_t idQ = idesc_bf16_f32(128, 16, 1, 1);
-      const uint32_t lboK = (D == 128) ? C::kChunk : 0u;    // d = 64: rows 64-127 of dQ^T repeat 0-63
       int kit = 0, vit = 0, tc = 0, uc = 0;
       bool ok = true;
-      int prev_kst = 0;                                   // K stage of the tile whose dQ product is pending
       for (int64_t k = 0; ok && k < my_units; ++k, ++uc) {
         const QUnit x = q_unit(blockIdx.x + k * gridDim.x, a);
         const int nt = (x.nvalid + 1) >> 1;
-        const int qb = uc & 1, ub = uc & 1;
-        if (!mbar_wait(&bars->q_full[qb], (uc >> 1) & 1) ||
-            !mbar_wait(&bars->dq_empty[ub], ((uc >> 1) & 1) ^ 1) || q_aborted(bars)) {
-          q_set_abort(bars); ok = false; break;
-        }
+        const int qb = uc & 1;
+        if (!mbar_wait(&bars->q_full[qb], (uc >> 1) & 1) || q_aborted(bars)) { q_set_abort(bars); ok = false; break; }
         tc_fence_after();
         const uint32_t q_base = smem_u32(sQ + qb * C::kQBuf);
         const uint32_t do_base = smem_u32(sdO + qb * C::kQBuf);
-        const uint32_t dq_addr = tmem + 64 + 16 * ub;
-        auto issue_dq = [&](int tile, int kst, bool first) -> bool {
-          const int sb = tile & 1;
-          if (!mbar_wait(&bars->ds_full[sb], (tile >> 1) & 1) || q_aborted(bars)) return false;
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(sKr + kst * C::kKBytes);
-          const uint32_t ds_base = smem_u32(sdS + sb * C::kDSBuf);
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint64_t ad = make_sdesc(k_base + kk * 2048, lboK, 1024, kLayoutSW128);
-            const uint64_t bd = make_sdesc(ds_base + kk * 512, 256, 128, kLayoutNone);
-            umma_bf16(dq_addr, ad, bd, idQ, (first && kk == 0) ? 0u : 1u);
-          }
-          umma_commit(&bars->k_empty[kst]);
-          umma_commit(&bars->ds_empty[sb]);
-          return true;
-        };
-        for (int j = 0; ok && j < nt; ++j) {
+        for (int j = 0; ok && j < nt; ++j, ++kit, ++vit, ++tc) {
           const int kst = kit % C::kKStages, vst = vit % C::kVStages, sb = tc & 1;
           if (!mbar_wait(&bars->k_full[kst], (kit / C::kKStages) & 1) ||
               !mbar_wait(&bars->v_full[vst], (vit / C::kVStages) & 1) ||
@@ -464,18 +454,48 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
           }
           umma_commit(&bars->s_full[sb]);
           umma_commit(&bars->v_empty[vst]);
-          // the previous tile's dS has had this tile's products to arrive
-          if (j > 0 && !issue_dq(tc - 1, prev_kst, j == 1)) { q_set_abort(bars); ok = false; break; }
-          prev_kst = kst;
-          ++kit; ++vit; ++tc;
         }
-        if (!ok) break;
-        if (nt > 0 && !issue_dq(tc - 1, prev_kst, nt == 1)) { q_set_abort(bars); ok = false; break; }
-        umma_commit(&bars->dq_full[ub]);
-        umma_commit(&bars->q_empty[qb]);
+        if (ok) umma_commit(&bars->q_empty[qb]);         // Q and dO are read by S and dP only
       }
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0);
+    }
+  } else if (warp == kQDqWarp) {
+    // ------------------------------------------------------------ dQ issuer
+    // per tile, once its dS is in shared memory: dQ^T += K_pair^T dS^T
+    if (lane == 0) {
+      const uint32_t idQ = idesc_bf16_f32(128, 16, 1, 1);
+      const uint32_t lboK = (D == 128) ? C::kChunk : 0u;    // d = 64: rows 64-127 of dQ^T repeat 0-63
+      int kit = 0, tc = 0, uc = 0;
+      bool ok = true;
+      for (int64_t k = 0; ok && k < my_units; ++k, ++uc) {
+        const QUnit x = q_unit(blockIdx.x + k * gridDim.x, a);
+        const int nt = (x.nvalid + 1) >> 1;
+        const int ub = uc & 1;
+        if (!mbar_wait(&bars->dq_empty[ub], ((uc >> 1) & 1) ^ 1) || q_aborted(bars)) {
+          q_set_abort(bars); ok = false; break;
+        }
+        tc_fence_after();
+        const uint32_t dq_addr = tmem + 64 + 16 * ub;
+        for (int j = 0; ok && j < nt; ++j, ++kit, ++tc) {
+          const int kst = kit % C::kKStages, sb = tc & 1;
+          if (!mbar_wait(&bars->ds_full[sb], (tc >> 1) & 1) || q_aborted(bars)) { q_set_abort(bars); ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sKr + kst * C::kKBytes);
+          const uint32_t ds_base = smem_u32(sdS + sb * C::kDSBuf);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t ad = make_sdesc(k_base + kk * 2048, lboK, 1024, kLayoutSW128);
+            const uint64_t bd = make_sdesc(ds_base + kk * 512, 256, 128, kLayoutNone);
+            umma_bf16(dq_addr, ad, bd, idQ, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->k_empty[kst]);
+          umma_commit(&bars->ds_empty[sb]);
+        }
+        if (ok) umma_commit(&bars->dq_full[ub]);
+      }
+      umma_commit(&bars->dq_done);
+      mbar_wait(&bars->dq_done, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warps 2..5 (one key lane each)
@@ -535,7 +555,9 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->ds_full[sb]);
-        if (bar_red_or(1, 128, ab || q_aborted(bars))) { q_set_abort(bars); stop = true; break; }
+        // the four warps need no common step per tile: each stops on its own
+        // failed wait (the others' bounded waits then run out too)
+        if (__any_sync(0xffffffffu, ab || q_aborted(bars))) { q_set_abort(bars); stop = true; break; }
       }
       if (stop) break;
       // ---- unit done: dQ = scale * dQ^T, this lane's d row
@@ -546,7 +568,7 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_empty[ub]);
-      if (bar_red_or(1, 128, !got || q_aborted(bars))) { q_set_abort(bars); stop = true; break; }
+      if (__any_sync(0xffffffffu, !got || q_aborted(bars))) { q_set_abort(bars); stop = true; break; }
       if (kl < D) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -602,6 +624,8 @@ __device__ __forceinline__ int task_of_block(const Args& a, int i) {
 template <int D, int G>
 __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                              const __grid_constant__ CUtensorMap tmdO,
+                                                             const __grid_constant__ CUtensorMap tmQc,
+                                                             const __grid_constant__ CUtensorMap tmdOc,
                                                              const __grid_constant__ CUtensorMap tmK,
                                                              const __grid_constant__ CUtensorMap tmV, const Args a) {
   using C = KVCfg<D>;
@@ -675,14 +699,31 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
         else kv_set_abort(bars);
       }
       if (!__shfl_sync(0xffffffffu, good, 0)) break;
-      for (int q = 0; q < TQ; ++q) {
-        const int t = __shfl_sync(0xffffffffu, t_l, q);
+      // a chunk of TQ consecutive tokens (the init / local part of the list is
+      // one contiguous range) loads as one box per 64 dims; scattered tokens
+      // (the top-k part) one box each
+      const int t_first = __shfl_sync(0xffffffffu, t_l, 0);
+      const int t_lastq = __shfl_sync(0xffffffffu, t_l, TQ - 1);
+      const bool contig = (c * TQ + TQ <= count) && (t_lastq - t_first == TQ - 1);
+      if (contig) {
         if (lane == 0) {
           for (int ch = 0; ch < C::KCH; ++ch) {
-            tma_load_4d(sQ + qb * C::kRows + ch * C::kRowsChunk + q * G * 128, &tmQ, &bars->qd_full[qb], ch * 64, 0,
-                        g, row0 + t);
-            tma_load_4d(sdO + qb * C::kRows + ch * C::kRowsChunk + q * G * 128, &tmdO, &bars->qd_full[qb], ch * 64,
-                        0, g, row0 + t);
+            tma_load_4d(sQ + qb * C::kRows + ch * C::kRowsChunk, &tmQc, &bars->qd_full[qb], ch * 64, 0, g,
+                        row0 + t_first);
+            tma_load_4d(sdO + qb * C::kRows + ch * C::kRowsChunk, &tmdOc, &bars->qd_full[qb], ch * 64, 0, g,
+                        row0 + t_first);
+          }
+        }
+      } else {
+        for (int q = 0; q < TQ; ++q) {
+          const int t = __shfl_sync(0xffffffffu, t_l, q);
+          if (lane == 0) {
+            for (int ch = 0; ch < C::KCH; ++ch) {
+              tma_load_4d(sQ + qb * C::kRows + ch * C::kRowsChunk + q * G * 128, &tmQ, &bars->qd_full[qb], ch * 64,
+                          0, g, row0 + t);
+              tma_load_4d(sdO + qb * C::kRows + ch * C::kRowsChunk + q * G * 128, &tmdO, &bars->qd_full[qb],
+                          ch * 64, 0, g, row0 + t);
+            }
           }
         }
       }
@@ -867,12 +908,14 @@ static cudaError_t launch_bwd_t(const void* Q, const void* K, const void* V, con
                                 const void* dO, bwd::Args a, cudaStream_t st, bool* map_fail) {
   using bf = __nv_bfloat16;
   const int h_q = a.h_q, h_kv = a.h_kv;
-  CUtensorMap mQ, mdO, mK, mV;
+  CUtensorMap mQ, mdO, mQc, mdOc, mK, mV;
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)G, (uint64_t)h_kv, (uint64_t)a.total};
     const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)G * D * 2, (uint64_t)h_q * D * 2};
     const uint32_t box[4] = {64, (uint32_t)G, 1, 1};
-    if (!make_tmap(&mQ, Q, 4, dims, strides, box) || !make_tmap(&mdO, dO, 4, dims, strides, box)) {
+    const uint32_t boxc[4] = {64, (uint32_t)G, 1, (uint32_t)(128 / G)};   // 128/G consecutive tokens
+    if (!make_tmap(&mQ, Q, 4, dims, strides, box) || !make_tmap(&mdO, dO, 4, dims, strides, box) ||
+        !make_tmap(&mQc, Q, 4, dims, strides, boxc) || !make_tmap(&mdOc, dO, 4, dims, strides, boxc)) {
       *map_fail = true;
       return cudaErrorInvalidValue;
     }
@@ -909,7 +952,8 @@ static cudaError_t launch_bwd_t(const void* Q, const void* K, const void* V, con
     auto kern = bwd::dkdv_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(a.h_kv * a.batch * a.nb_max), bwd::kKVThreads, C::kSmem, st>>>(mQ, mdO, mK, mV, a);
+    kern<<<static_cast<unsigned>(a.h_kv * a.batch * a.nb_max), bwd::kKVThreads, C::kSmem, st>>>(mQ, mdO, mQc, mdOc,
+                                                                                                  mK, mV, a);
   }
   return cudaGetLastError();
 }
