@@ -90,12 +90,12 @@ __device__ __noinline__ void warp_select_write(uint32_t* keys, int* hist, int nc
       if (lane + o < 32) suf += v;
     }
     int above = suf - lsum;  // keys in bins above this lane's range
-    int digit = -1, above_digit = 0;
+    int digit = -1, above_digit = 0, in_digit = 0;
     if (above < k_rem && suf >= k_rem) {
       for (int q = 7; q >= 0; --q) {
         const int b = lane * 8 + q;
         const int h = (b < nb) ? hist[b] : 0;
-        if (above + h >= k_rem) { digit = b; above_digit = above; break; }
+        if (above + h >= k_rem) { digit = b; above_digit = above; in_digit = h; break; }
         above += h;
       }
     }
@@ -103,10 +103,42 @@ __device__ __noinline__ void warp_select_write(uint32_t* keys, int* hist, int nc
     const int src = __ffs(who) - 1;
     digit = __shfl_sync(0xffffffffu, digit, src);
     above_digit = __shfl_sync(0xffffffffu, above_digit, src);
+    in_digit = __shfl_sync(0xffffffffu, in_digit, src);
     prefix |= static_cast<uint32_t>(digit) << shift;
     k_rem -= above_digit;
     hi = shift;
     __syncwarp();
+    if (hi > 0 && in_digit <= 32) {
+      // at most 32 keys share the boundary digit: gather them (the histogram
+      // is free now), sort them across the lanes and take the k_rem-th
+      // largest exactly, instead of more passes over every key
+      const uint32_t want_hi = prefix >> hi;
+      int n = 0;
+      for (int base = 0; base < ncand; base += 32) {
+        const int i = base + lane;
+        const uint32_t u = (i < ncand) ? keys[i] - kmin : 0u;
+        const bool m = (i < ncand) && (u >> hi) == want_hi;
+        const uint32_t bm = __ballot_sync(0xffffffffu, m);
+        if (m) hist[n + __popc(bm & lanemask_lt())] = static_cast<int>(u);
+        n += __popc(bm);
+      }
+      __syncwarp();
+      uint32_t x = (lane < n) ? static_cast<uint32_t>(hist[lane]) : 0u;   // 0 sorts last: no key of the bin is below it
+#pragma unroll
+      for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+          const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+          x = keep_max ? max(x, y) : min(x, y);
+        }
+      }
+      const uint32_t tu = __shfl_sync(0xffffffffu, x, k_rem - 1);
+      k_rem -= __popc(__ballot_sync(0xffffffffu, lane < n && x > tu));
+      prefix = tu;
+      hi = 0;
+      __syncwarp();
+    }
   }
   const uint32_t T = kmin + prefix;  // the top_k-th largest key; take k_rem of the keys equal to it
 
