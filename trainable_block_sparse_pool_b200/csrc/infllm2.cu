@@ -14,11 +14,18 @@
 
 #include "sm100.cuh"
 
+// The LOCAL part of the sparse attention and the dense path run on the kernel
+// with two query tiles per CTA (pair_attn.cu); 0 selects the one-tile kernel.
+#ifndef INFLLM2_PAIR_ATTN
+#define INFLLM2_PAIR_ATTN 1
+#endif
+
 #include "compress.cu"
 #include "score.cu"
 #include "select.cu"
 #include "sparse_attn.cu"
 #include "dense_attn.cu"
+#include "pair_attn.cu"
 #include "decode.cu"
 #include "backward.cu"
 #include "probe.cu"
@@ -264,8 +271,8 @@ int infllm2_sparse_attn(const void* Q, const void* K, const void* V, const int32
   cudaError_t e = launch_sparse_attn(Q, K, V, block_idx, vl->cu_seqlens, vl->batch, vl->total, h_q, h_kv, d, n_sel,
                                      p->n_init, p->n_local, scale, out, f32, lse, st, &map_fail);
   if (e == cudaSuccess && !map_fail)
-    e = launch_dense_attn(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d, scale, out,
-                          f32, p->n_init, p->n_local, lse, st, &map_fail);
+    e = (INFLLM2_PAIR_ATTN ? launch_pair_attn : launch_dense_attn)(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen,
+                          vl->total, h_q, h_kv, d, scale, out, f32, p->n_init, p->n_local, lse, st, &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
@@ -278,9 +285,9 @@ int infllm2_dense_attn(const void* Q, const void* K, const void* V, const infllm
     return INFLLM2_ERR_INVALID_ARG;
   if (out_dtype != INFLLM2_OUT_BF16 && out_dtype != INFLLM2_OUT_F32) return INFLLM2_ERR_INVALID_ARG;
   bool map_fail = false;
-  cudaError_t e = launch_dense_attn(Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d,
-                                    softmax_scale(p, d), out, out_dtype == INFLLM2_OUT_F32, 0, 0, nullptr,
-                                    static_cast<cudaStream_t>(stream), &map_fail);
+  cudaError_t e = (INFLLM2_PAIR_ATTN ? launch_pair_attn : launch_dense_attn)(
+      Q, K, V, vl->cu_seqlens, vl->batch, vl->max_seqlen, vl->total, h_q, h_kv, d, softmax_scale(p, d), out,
+      out_dtype == INFLLM2_OUT_F32, 0, 0, nullptr, static_cast<cudaStream_t>(stream), &map_fail);
   if (map_fail) return INFLLM2_ERR_INVALID_ARG;
   return e == cudaSuccess ? INFLLM2_OK : cuda_fail(e);
 }
