@@ -104,9 +104,9 @@ def algorithmic_work(n: int, h_q: int, h_kv: int, d: int):
     w["sparse_shared_gather_bytes"] = h_kv * 2 * d * 2 * 64 * int(shared_blocks_at(qb).sum())
     w["sparse_gather_bytes"] = w["sparse_topk_gather_bytes"] + w["sparse_shared_gather_bytes"]
     # what the kernels move for the shared blocks: the LOCAL form reads them
-    # once per CTA of 128/G tokens (re-reads counted apart from the
-    # algorithmic bytes)
-    t0 = np.arange(0, n, max(1, 128 // G))
+    # once per CTA of two 128-row query tiles, 256/G tokens (re-reads counted
+    # apart from the algorithmic bytes)
+    t0 = np.arange(0, n, max(1, 256 // G))
     w["sparse_shared_gather_bytes_kernel"] = h_kv * 2 * d * 2 * 64 * int(shared_blocks_at(t0 // 64).sum())
     w["ld"] = ld
     return w

@@ -30,7 +30,13 @@ namespace pair {
 
 constexpr int kThreads = 320;              // 10 warps
 constexpr int kKeys = 128;
-constexpr int kKStages = 2;
+#ifndef INFLLM2_PAIR_KSTAGES
+#define INFLLM2_PAIR_KSTAGES 2
+#endif
+#ifndef INFLLM2_PAIR_PIPE
+#define INFLLM2_PAIR_PIPE 0
+#endif
+constexpr int kKStages = INFLLM2_PAIR_KSTAGES;
 constexpr int kVStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.f;            // raise m only past this margin (log2 units)
@@ -245,17 +251,41 @@ __global__ void __launch_bounds__(kThreads, 1) pair_attn_kernel(
         ub[e] = (blk >= 0 && (!LOCAL || in_set(blk, t, n_init, n_local))) ? 64 * blk : INT_MAX / 2;
       }
       // pass 1: the row maximum over both halves (raw scores; the scale c > 0
-      // goes into the exponent); the second half stays in registers
+      // goes into the exponent); the second half stays in registers.  Tiles
+      // whose keys every row of the warp sees skip the masking.
+      const bool vis = __all_sync(0xffffffffu, ub[0] + 63 <= t && ub[1] + 63 <= t);
       float va[64], vb[64];
       tmem_load64(t_s, va);
+#if INFLLM2_PAIR_PIPE
+      // the second half's read is in flight while the first half is reduced
+      float (&vb0)[32] = *reinterpret_cast<float(*)[32]>(&vb[0]);
+      float (&vb1)[32] = *reinterpret_cast<float(*)[32]>(&vb[32]);
+      tmem_ld32(t_s + 64, vb0);
+      tmem_ld32(t_s + 96, vb1);
+#endif
       float mx = -INFINITY;
+      if (vis) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, (ub[0] + i <= t) ? va[i] : -INFINITY);
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, va[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, (ub[0] + i <= t) ? va[i] : -INFINITY);
+      }
+#if INFLLM2_PAIR_PIPE
+      tmem_wait_ld32(vb0);
+      tmem_wait_ld32(vb1);
+#else
       tmem_load64(t_s + 64, vb);
+#endif
+      if (vis) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        vb[i] = (ub[1] + i <= t) ? vb[i] : -INFINITY;
-        mx = fmaxf(mx, vb[i]);
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, vb[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          vb[i] = (ub[1] + i <= t) ? vb[i] : -INFINITY;
+          mx = fmaxf(mx, vb[i]);
+        }
       }
       mx *= c;                                    // -inf stays -inf
       // a raise of the reference: O (once the pending P.V product is done) and
@@ -298,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) pair_attn_kernel(
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float x0 = (ub[0] + 2 * i <= t) ? va[2 * i] : -INFINITY;
-          const float x1 = (ub[0] + 2 * i + 1 <= t) ? va[2 * i + 1] : -INFINITY;
+          const float x0 = (vis || ub[0] + 2 * i <= t) ? va[2 * i] : -INFINITY;
+          const float x1 = (vis || ub[0] + 2 * i + 1 <= t) ? va[2 * i + 1] : -INFINITY;
           const float p0 = none ? 0.f : ex2(fmaf(x0, c, -m_ref));
           const float p1 = none ? 0.f : ex2(fmaf(x1, c, -m_ref));
           lsum += p0 + p1;
