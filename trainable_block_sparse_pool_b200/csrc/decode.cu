@@ -5,17 +5,22 @@
 //
 // The new token of sequence b sits at position t = seq_len[b]; the step is
 // row t of the prefill rule applied to the sequence extended by one token.
-// Three kernels:
+// Three kernels (four with INFLLM2_DEC_SPLIT_SELECT=1):
 //   K1 append k, v at t; if a stage-1 window ends at t (t+1 >= 32,
 //      (t+1) % 16 == 0) pool it into K_c1, likewise a coarse window
 //      (t+1 >= 128, (t+1) % 64 == 0) into K_c2 (exact mean, one bf16
 //      rounding); per-head log-sum-exp partials over the visible coarse
 //      windows, split over CTAs
 //   K2 S over the visible stage-1 windows (head-group sum fused) and the
-//      max-pool to block scores, streamed through TMA in one wave of CTAs;
-//      the CTA that completes the last piece of a (sequence, group) selects
-//      its blocks
-//   K3 split-KV block-sparse attention over the selected blocks; the splits
+//      max-pool to block scores, streamed through TMA in one wave of CTAs
+//   K2b the selection of each (sequence, group), one CTA each, once every
+//      block score of the step is written (built with
+//      INFLLM2_DEC_SPLIT_SELECT=0, K2's CTA that completes the last piece of a
+//      (sequence, group) selects instead)
+//   K3 split-KV block-sparse attention: before the wait for K2b each split
+//      streams its share of the init and local blocks (every list holds
+//      them), after it its share of the top-k blocks and of the query's own
+//      block; the splits
 //      of a (sequence, group) merge through distributed shared memory inside
 //      a thread-block cluster (or, past 8 splits, through the workspace and
 //      a completion counter), and the last group of a sequence advances
@@ -617,7 +622,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
     const __nv_bfloat16* __restrict__ kc1, const int32_t* __restrict__ seq_len,
     const float2* __restrict__ part2, int nsplit2, int batch, int capacity, int h_q, int h_kv, int cap_c1,
     int nblk_cap, int cand_cap, float scale, int n_init, int n_local, int top_k, int n_sel,
-    float* __restrict__ bscore, int32_t* __restrict__ idx, unsigned* __restrict__ cnt) {
+    float* __restrict__ bscore, int32_t* __restrict__ idx, unsigned* __restrict__ cnt, int select_here) {
   using C = ScoreCfg<D>;
   extern __shared__ __align__(128) uint8_t sc_smem[];   // the ring; the selection's keys and bins reuse it
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sc_smem) + 1023) & ~uintptr_t(1023));
@@ -874,7 +879,7 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
         for (int q4 = 1; q4 < 5; ++q4) m = fmaxf(m, swc[4 * lane + q4]);
         if (blk < nblk_cap) bscore[static_cast<int64_t>(bg) * nblk_cap + blk] = m;
       }
-      if (seg_last(j)) {
+      if (select_here && seg_last(j)) {
         // the segment's pieces are done: count them; the CTA that completes
         // the last piece of (b, g) owes its selection
         __threadfence();
@@ -900,6 +905,28 @@ __global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(
                       sel_sh);
     __syncthreads();                           // the scratch is reused by the next selection
   }
+}
+
+// ---------------------------------------------------------------- K2b: the selection of each (sequence, group)
+// One CTA per (b, g), launched between the score kernel and the attention
+// kernel (programmatic dependent launch on both sides): it waits for every
+// block score of the step, then selects as select_blocks_cta does.  The
+// attention kernel meanwhile streams the blocks every list holds (init and
+// local), which need no selection.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ bscore,
+                                                             const int32_t* __restrict__ seq_len, int capacity,
+                                                             int h_kv, int n_init, int n_local, int top_k, int n_sel,
+                                                             int nblk_cap, int cand_cap, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t sel_dyn[];
+  __shared__ SelScratch sel_sh;
+  griddep_launch_dependents();
+  griddep_wait();                              // the block scores of the step
+  const int bg = blockIdx.x;
+  const int t = seq_len[bg / h_kv];
+  if (t < 0 || t >= capacity) return;          // recorded by the append kernel
+  select_blocks_cta(bscore + static_cast<int64_t>(bg) * nblk_cap, t, n_init, n_local, top_k, n_sel, cand_cap,
+                    idx + static_cast<int64_t>(bg) * n_sel, reinterpret_cast<uint32_t*>(sel_dyn),
+                    reinterpret_cast<int*>(sel_dyn + ((static_cast<size_t>(cand_cap) * 4 + 15) & ~size_t(15))), sel_sh);
 }
 
 constexpr int kAttWarps = 6;
@@ -948,11 +975,18 @@ struct AttCfg {
 // last group of b to finish advances seq_len[b].
 // Keys past t (and chunks of invalid or not yet visible blocks) are never
 // read: their staging rows are zero-filled and their scores are -inf.
-template <int D, bool CLUSTER>
+// PHASED: the CTA's work comes in two phases.  Phase 0, before the wait for
+// the selection, covers the CTA's share of the blocks every list holds (the
+// init blocks and the local run, without the query's own block b_t, whose
+// row t the append kernel of this step writes); phase 1, after it, the CTA's
+// share of the top-k blocks and b_t.  Without PHASED the CTA covers entries
+// [sp*bps, sp*bps + bps) of the list, after the wait.
+template <int D, bool CLUSTER, bool PHASED>
 __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
     const int32_t* __restrict__ idx, int32_t* seq_len, int capacity, int h_q, int h_kv, int n_sel, int bps,
-    float scale, float* __restrict__ part, __nv_bfloat16* __restrict__ out, unsigned* __restrict__ cnt) {
+    float scale, float* __restrict__ part, __nv_bfloat16* __restrict__ out, unsigned* __restrict__ cnt, int n_init,
+    int n_local, int top_k) {
   using C = AttCfg<D>;
   extern __shared__ __align__(128) uint8_t att_smem[];
   __shared__ float s_wgt[kAttWarps][16], s_M[16], s_L[16];
@@ -966,7 +1000,19 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
   const int t = seq_len[b];
   const int32_t* list = idx + static_cast<int64_t>(bg) * n_sel + static_cast<int64_t>(sp) * bps;
   const int nb = max(0, min(bps, n_sel - sp * bps));
-  const int nmine = (2 * nb > warp) ? (2 * nb - 1 - warp) / kAttWarps + 1 : 0;
+  // PHASED partition (from t alone): S = init blocks below b_t, then the local
+  // run below b_t; P = the list's top-k entries, then b_t.  This CTA takes
+  // the sp-th share of each.
+  const int b_t = t >> 6;
+  const int i_hi = min(n_init, b_t + 1);
+  const int l_start = max(i_hi, max(0, b_t - n_local + 1));
+  const int s_init = min(i_hi, b_t);
+  const int s_all = s_init + max(0, b_t - l_start);
+  const int ntop = min(top_k, max(0, l_start - i_hi));
+  const int p_all = ntop + 1;
+  const int s_lo = s_all * sp / nsplit, s_cnt = s_all * (sp + 1) / nsplit - s_lo;
+  const int p_lo = p_all * sp / nsplit, p_cnt = p_all * (sp + 1) / nsplit - p_lo;
+  const int32_t* list_all = idx + static_cast<int64_t>(bg) * n_sel;
   const int64_t kstride = static_cast<int64_t>(h_kv) * D;    // elements from one key row to the next
   const int64_t row0 = (static_cast<int64_t>(b) * capacity * h_kv + g) * D;
   // the warp's buffers: K of chunks i and i + 1, then V of chunks i and i + 1
@@ -985,17 +1031,32 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
       qa[kk][3] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qh + (gid + 8) * D + d0 + 8) : 0u;
     }
   }
-  // the block lists come from the score kernel
-  griddep_wait();
+  // the block lists come from the selection (PHASED: only phase 1 reads them)
+  if (!PHASED) griddep_wait();
   if (t < 0 || t >= capacity) return;          // recorded by the append kernel
 
-  // first key of the warp's i-th chunk, or -1 when it has no visible key
+  // chunks of the warp in the current phase, and the first key of its i-th
+  // chunk (-1 when it has no visible key)
+  int phase = 0, nmine = 0;
+  auto phase_chunks = [&](int ph) -> int {
+    const int ne = !PHASED ? nb : (ph == 0 ? s_cnt : p_cnt);
+    return (2 * ne > warp) ? (2 * ne - 1 - warp) / kAttWarps + 1 : 0;
+  };
   auto chunk_key0 = [&](int i) -> int {
     if (i >= nmine) return -1;
     const int ch = warp + kAttWarps * i;
-    const int blk = list[ch >> 1];
+    int blk;
+    if (!PHASED) {
+      blk = list[ch >> 1];
+    } else if (phase == 0) {
+      const int e = s_lo + (ch >> 1);
+      blk = (e < s_init) ? e : l_start + (e - s_init);
+    } else {
+      const int e = p_lo + (ch >> 1);
+      blk = (e < ntop) ? list_all[i_hi + e] : b_t;
+    }
     const int k0 = 64 * blk + kChunkKeys * (ch & 1);
-    return (blk >= 0 && blk <= t / 64 && k0 <= t) ? k0 : -1;
+    return (blk >= 0 && blk <= b_t && k0 <= t) ? k0 : -1;
   };
   auto stage = [&](uint32_t dst, const __nv_bfloat16* cache, int k0) {
     if (k0 >= 0) {
@@ -1019,7 +1080,11 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
 
   // copies in flight per warp: two chunks ahead.  Commit order: K0 V0 K1 V1,
   // then per chunk i: K(i+2) after its S product, V(i+2) after its P.V
-  // product, so K(i) and V(i) each have exactly three younger groups.
+  // product, so K(i) and V(i) each have exactly three younger groups.  Each
+  // phase starts and drains its own stream of copies.
+  for (phase = 0; phase < (PHASED ? 2 : 1); ++phase) {
+  if (PHASED && phase == 1) griddep_wait();     // the lists of this step are selected
+  nmine = phase_chunks(phase);
   int k0 = chunk_key0(0);
   int k1 = chunk_key0(1);
   stage(sbuf, kc, k0);
@@ -1121,6 +1186,8 @@ __global__ void __launch_bounds__(32 * kAttWarps, 1) attend_kernel(
     k1 = k0n;
   }
   cp_async_wait0();
+  __syncwarp();
+  }                                            // phases
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -1461,6 +1528,15 @@ DecodePlan decode_plan(int batch, int capacity, int h_q, int h_kv, int d, int n_
   return p;
 }
 
+// 1: the selection runs as its own launch and the attention streams the init
+// and local blocks while it runs (measured slower: 53.9 vs 49.4 us per step at
+// 16 x 131072); 0: the CTA that completes a (sequence, group)'s last piece in
+// the score kernel selects.
+#ifndef INFLLM2_DEC_SPLIT_SELECT
+#define INFLLM2_DEC_SPLIT_SELECT 0
+#endif
+constexpr bool kSplitSelect = INFLLM2_DEC_SPLIT_SELECT != 0;
+
 template <int D>
 static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, const void* k_new, const void* v_new,
                                  void* out, void* ws, const DecodePlan& P, int n_init, int n_local, int top_k,
@@ -1515,12 +1591,31 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
     e = cudaLaunchKernelEx(&cfg, dec::score_select_kernel<D>, mK1, static_cast<const bf*>(q),
                            static_cast<const bf*>(s->k_c1), static_cast<const int32_t*>(s->seq_len),
                            static_cast<const float2*>(part2), P.nsplit2, s->batch, s->capacity, s->h_q, s->h_kv,
-                           P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt);
+                           P.cap_c1, P.nblk_cap, P.cand_cap, scale, n_init, n_local, top_k, P.n_sel, bscore, idx, cnt,
+                           kSplitSelect ? 0 : 1);
+    if (e != cudaSuccess) return e;
+  }
+  if (kSplitSelect) {
+    // the selection as its own launch, between the scores and the attention
+    const size_t sel_smem = ((static_cast<size_t>(P.cand_cap) * 4 + 15) & ~size_t(15)) + dec::kSelBins * 4;
+    e = cudaFuncSetAttribute(dec::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sel_smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(bg);
+    cfg.blockDim = dim3(dec::kSelThreads);
+    cfg.dynamicSmemBytes = sel_smem;
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dec::select_kernel, static_cast<const float*>(bscore),
+                           static_cast<const int32_t*>(s->seq_len), s->capacity, s->h_kv, n_init, n_local, top_k,
+                           P.n_sel, P.nblk_cap, P.cand_cap, idx);
     if (e != cudaSuccess) return e;
   }
   if (P.nsplit <= 8) {
     // the splits of (b, g) as one cluster: the merge goes through distributed shared memory
-    e = cudaFuncSetAttribute(dec::attend_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(dec::attend_kernel<D, true, kSplitSelect>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(dec::AttCfg<D>::kSmem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -1536,13 +1631,13 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
     attr[1] = pdl[0];
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, dec::attend_kernel<D, true>, static_cast<const bf*>(q),
+    e = cudaLaunchKernelEx(&cfg, dec::attend_kernel<D, true, kSplitSelect>, static_cast<const bf*>(q),
                            static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache),
                            static_cast<const int32_t*>(idx), s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps,
-                           scale, part, static_cast<bf*>(out), cnt);
+                           scale, part, static_cast<bf*>(out), cnt, n_init, n_local, top_k);
     if (e != cudaSuccess) return e;
   } else {
-    e = cudaFuncSetAttribute(dec::attend_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(dec::attend_kernel<D, false, kSplitSelect>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(dec::AttCfg<D>::kSmem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -1552,10 +1647,10 @@ static cudaError_t decode_step_t(const infllm2_decode_state* s, const void* q, c
     cfg.stream = st;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, dec::attend_kernel<D, false>, static_cast<const bf*>(q),
+    e = cudaLaunchKernelEx(&cfg, dec::attend_kernel<D, false, kSplitSelect>, static_cast<const bf*>(q),
                            static_cast<const bf*>(s->k_cache), static_cast<const bf*>(s->v_cache),
                            static_cast<const int32_t*>(idx), s->seq_len, s->capacity, s->h_q, s->h_kv, P.n_sel, P.bps,
-                           scale, part, static_cast<bf*>(out), cnt);
+                           scale, part, static_cast<bf*>(out), cnt, n_init, n_local, top_k);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
