@@ -65,6 +65,8 @@ def _check_rows(run, data, w, rows, seqs, S_gpu, idx_gpu, min_exact=0.85):
 
 
 def _check_attention(run, w, rows, seqs, ref_idx):
+    torch.cuda.synchronize()
+    assert T_status() == 0, T_status()     # a device-side timeout or bounds record voids the output
     p = H.oracle_params(w)
     sidx, tloc = H.seq_of_rows(run.lens, rows)
     out = run.out.float().cpu().numpy()

@@ -40,9 +40,23 @@ namespace infllm2 {
 
 namespace sparse {
 
+// One thread issues tcgen05.mma at a limited rate: measured on the B200,
+// about one M=128, N=16, K=16 product per 100 cycles when independent and per
+// 180 cycles in the 8-step chains of a QK or PV product, while the tensor pipe
+// takes one every ~40 cycles from several issuing threads.  A single QK issuer
+// for both softmax groups (8 chained products per tile) caps the kernel near
+// 0.7 us per tile, so each group has its own QK issuer, as it has its own PV
+// issuer.  0 restores the single QK issuer.
+#ifndef INFLLM2_SPARSE_QK_SPLIT
+#define INFLLM2_SPARSE_QK_SPLIT 1
+#endif
+
 constexpr int kNumWG = 2;
-constexpr int kThreads = 64 + 128 * kNumWG + 32 * kNumWG + 32;   // K producer, QK, softmax groups, PV issuers, V producer
+constexpr bool kQKSplit = INFLLM2_SPARSE_QK_SPLIT != 0;
+// K producer, QK issuer(s), softmax groups, PV issuers, V producer
+constexpr int kThreads = 64 + 128 * kNumWG + 32 * kNumWG + 32 + (kQKSplit ? 32 * (kNumWG - 1) : 0);
 constexpr int kVWarp = 2 + 5 * kNumWG;   // the V producer
+constexpr int kQK1Warp = kVWarp + 1;     // with the split: the QK issuer of softmax group 1 (group 0: warp 1)
 constexpr int kPairKeys = 128;       // keys per tile (two 64-key blocks)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.f;      // raise m_ref only past this margin (log2 units)
@@ -61,7 +75,7 @@ struct Cfg {
   static constexpr uint32_t kPBuf = kPairKeys * 16 * 2;       // 4 KB
   static constexpr uint32_t kRed = kNumWG * 4 * 16 * 4;       // per-warp partial maxima / sums
   static constexpr uint32_t kSmem =
-      1024 + kStages * kKBytes + kNumWG * 2 * kQBuf + kNumWG * 2 * kPBuf + kRed + 512;
+      1024 + kStages * kKBytes + kNumWG * 2 * kQBuf + kNumWG * 2 * kPBuf + kRed + 1024;
 };
 
 struct Bars {
@@ -76,7 +90,7 @@ struct Bars {
   uint64_t p_full[kNumWG][2];
   uint64_t pv_done[kNumWG][2];
   uint64_t o_free[kNumWG][2];
-  uint64_t mma_done[1 + kNumWG];
+  uint64_t mma_done[2 + kNumWG];   // QK issuer(s) of group 0 and 1 at 0 and 1 + kNumWG, PV issuers between
   uint32_t tmem_base;
   int abort;
 };
@@ -219,6 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
     const __grid_constant__ CUtensorMap tmV, const SparseArgs args) {
   using C = Cfg<D>;
   static_assert(G >= 1 && G <= 16, "group size <= 16");
+  static_assert(sizeof(Bars) <= 1024, "barrier area");
+  static_assert(C::kSmem <= 232448, "shared memory per CTA");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem;
@@ -256,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         mbar_init(&bars->pv_done[w][i], 1);
         mbar_init(&bars->o_free[w][i], 4);
       }
-    for (int i = 0; i < 1 + kNumWG; ++i) mbar_init(&bars->mma_done[i], 1);
+    for (int i = 0; i < 2 + kNumWG; ++i) mbar_init(&bars->mma_done[i], 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -345,10 +361,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         for (int w = 0; w < kNumWG; ++w)
           for (int i = max(0, ucnt[w] - 2); i < ucnt[w]; ++i) mbar_wait(&bars->q_full[w][i & 1], (i >> 1) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ QK issuer
-    // Walks the stream in order: a QK product goes out as soon as its K/V
-    // stage has landed and its group's S buffer is free.
+  } else if (warp == 1 || (kQKSplit && warp == kQK1Warp)) {
+    // ------------------------------------------------------------ QK issuer(s)
+    // Walk the stream in order: a QK product goes out as soon as its K stage
+    // has landed and its group's S buffer is free.  With the split each
+    // issuer takes one group's tiles and steps over the other's.
+    const int mine = kQKSplit ? (warp == 1 ? 0 : 1) : -1;   // -1: both groups
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 16, 0, 0);
       int it = 0;
@@ -362,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
           const Unit x = get_unit(blockIdx.x + (k0 + w) * gridDim.x, args);
           nt[w] = ntiles_of(x);
           qb[w] = ucnt[w] & 1;
+          if (mine >= 0 && w != mine) continue;
           if (!mbar_wait(&bars->q_full[w][qb[w]], (ucnt[w] >> 1) & 1)) { set_abort(bars); ok = false; break; }
           if (nt[w] == 0) umma_commit(&bars->q_empty[w][qb[w]]);   // empty list: Q is free at once
           ++ucnt[w];
@@ -370,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         for (int j = 0; ok && j < nmax; ++j) {
           for (int w = 0; w < kNumWG; ++w) {
             if (j >= nt[w]) continue;
+            if (mine >= 0 && w != mine) { ++it; continue; }
             const int st = it % C::kKStages;
             const int sb = tcnt[w] & 1;
             if (!mbar_wait(&bars->k_full[st], (it / C::kKStages) & 1) ||
@@ -393,8 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
           }
         }
       }
-      umma_commit(&bars->mma_done[0]);
-      mbar_wait(&bars->mma_done[0], 0);
+      const int done = (warp == 1) ? 0 : 1 + kNumWG;
+      umma_commit(&bars->mma_done[done]);
+      mbar_wait(&bars->mma_done[done], 0);
     }
   } else if (warp >= 2 + 4 * kNumWG && warp < kVWarp) {
     // ------------------------------------------------------------ PV issuers
