@@ -263,9 +263,20 @@ __global__ void __launch_bounds__(256) fill_kernel(const Args a) {
 }
 
 // ---------------------------------------------------------------- dQ: per (kv group, token)
-constexpr int kQThreads = 256;       // warp 0 K/Q/dO producer, 1 S/dP MMA, 2-5 softmax, 6 V producer, 7 dQ MMA
+// One thread issues tcgen05.mma at about one product per 100-180 cycles
+// (measured on the B200 for M=128, N=16 chains), so the products of a tile
+// are spread over several issuing threads: with the split, S and dP (dQ
+// kernel) and {S, dV^T} / {dP, dK^T} (dK/dV kernel) go out from two threads.
+// 0 restores one issuer for them.
+#ifndef INFLLM2_BWD_SPLIT
+#define INFLLM2_BWD_SPLIT 1
+#endif
+constexpr bool kBwdSplit = INFLLM2_BWD_SPLIT != 0;
+// warp 0 K/Q/dO producer, 1 S (and dP) MMA, 2-5 softmax, 6 V producer, 7 dQ MMA, 8 (split) dP MMA
+constexpr int kQThreads = kBwdSplit ? 288 : 256;
 constexpr int kQVWarp = 6;
 constexpr int kQDqWarp = 7;
+constexpr int kQDpWarp = 8;
 
 template <int D>
 struct QCfg {
@@ -287,7 +298,7 @@ struct QBars {
   uint64_t s_full[2], s_empty[2];
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_empty[2];
-  uint64_t mma_done, dq_done;      // each MMA issuer's own products have completed
+  uint64_t mma_done, dq_done, dp_done;   // each MMA issuer's own products have completed
   uint32_t tmem_base;
   int abort;
 };
@@ -350,8 +361,8 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
     for (int i = 0; i < C::kVStages; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->q_full[i], 1);
-      mbar_init(&bars->q_empty[i], 1);
-      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->q_empty[i], kBwdSplit ? 2 : 1);   // Q read by S, dO by dP
+      mbar_init(&bars->s_full[i], kBwdSplit ? 2 : 1);    // S and dP both in TMEM
       mbar_init(&bars->s_empty[i], 4);
       mbar_init(&bars->ds_full[i], 4);
       mbar_init(&bars->ds_empty[i], 1);
@@ -360,6 +371,7 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
     }
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->dq_done, 1);
+    mbar_init(&bars->dp_done, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -414,10 +426,12 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
       if (!isV)
         for (int i = max(0, uc - 2); i < uc; ++i) mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ S / dP issuer
-    // per tile: S^T = K_pair Q^T and dP^T = V_pair dO^T; the V slot is free
-    // once dP is done, the K slot only after the dQ product (warp 7)
+  } else if (warp == 1 || (kBwdSplit && warp == kQDpWarp)) {
+    // ------------------------------------------------------------ S / dP issuer(s)
+    // per tile: S^T = K_pair Q^T and dP^T = V_pair dO^T (with the split, S
+    // from warp 1 and dP from warp kQDpWarp); the V slot is free once dP is
+    // done, the K slot only after the dQ product (warp kQDqWarp)
+    const bool do_s = (warp == 1), do_dp = !kBwdSplit || warp == kQDpWarp;
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 16, 0, 0);
       int kit = 0, vit = 0, tc = 0, uc = 0;
@@ -432,33 +446,38 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
         const uint32_t do_base = smem_u32(sdO + qb * C::kQBuf);
         for (int j = 0; ok && j < nt; ++j, ++kit, ++vit, ++tc) {
           const int kst = kit % C::kKStages, vst = vit % C::kVStages, sb = tc & 1;
-          if (!mbar_wait(&bars->k_full[kst], (kit / C::kKStages) & 1) ||
-              !mbar_wait(&bars->v_full[vst], (vit / C::kVStages) & 1) ||
+          if ((do_s && !mbar_wait(&bars->k_full[kst], (kit / C::kKStages) & 1)) ||
+              (do_dp && !mbar_wait(&bars->v_full[vst], (vit / C::kVStages) & 1)) ||
               !mbar_wait(&bars->s_empty[sb], ((tc >> 1) & 1) ^ 1) || q_aborted(bars)) {
             q_set_abort(bars); ok = false; break;
           }
           tc_fence_after();
           const uint32_t k_base = smem_u32(sKr + kst * C::kKBytes);
           const uint32_t v_base = smem_u32(sVr + vst * C::kKBytes);
+          if (do_s) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ak = make_sdesc(k_base + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            const uint64_t bq = make_sdesc(q_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            umma_bf16(tmem + 16 * sb, ak, bq, idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ak = make_sdesc(k_base + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              const uint64_t bq = make_sdesc(q_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              umma_bf16(tmem + 16 * sb, ak, bq, idS, kk > 0);
+            }
           }
+          if (do_dp) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t av = make_sdesc(v_base + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            const uint64_t bo = make_sdesc(do_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            umma_bf16(tmem + 32 + 16 * sb, av, bo, idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t av = make_sdesc(v_base + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              const uint64_t bo = make_sdesc(do_base + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              umma_bf16(tmem + 32 + 16 * sb, av, bo, idS, kk > 0);
+            }
           }
           umma_commit(&bars->s_full[sb]);
-          umma_commit(&bars->v_empty[vst]);
+          if (do_dp) umma_commit(&bars->v_empty[vst]);
         }
         if (ok) umma_commit(&bars->q_empty[qb]);         // Q and dO are read by S and dP only
       }
-      umma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0);
+      uint64_t* done = do_s ? &bars->mma_done : &bars->dp_done;
+      umma_commit(done);
+      mbar_wait(done, 0);
     }
   } else if (warp == kQDqWarp) {
     // ------------------------------------------------------------ dQ issuer
@@ -586,7 +605,10 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
 }
 
 // ---------------------------------------------------------------- dK / dV: per (kv group, sequence, key block)
-constexpr int kKVThreads = 192;      // warp 0 producer, 1 MMA, 2-5 softmax / epilogue
+// warp 0 producer, 1 MMA (S, dV^T; without the split all four products), 2-5 softmax / epilogue,
+// 6 (split) MMA for dP and dK^T
+constexpr int kKVThreads = kBwdSplit ? 224 : 192;
+constexpr int kKVIssuerB = 6;
 
 template <int D>
 struct KVCfg {
@@ -604,7 +626,7 @@ struct KVBars {
   uint64_t s_full[2], s_empty[2];
   uint64_t pd_full[2], pd_empty[2];
   uint64_t acc_full;
-  uint64_t mma_done;
+  uint64_t mma_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -656,16 +678,18 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
+    const uint32_t nis = kBwdSplit ? 2 : 1;      // one commit per MMA issuer
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->qd_full[i], 1);
-      mbar_init(&bars->qd_empty[i], 1);
-      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->qd_empty[i], nis);
+      mbar_init(&bars->s_full[i], nis);
       mbar_init(&bars->s_empty[i], 4);
       mbar_init(&bars->pd_full[i], 4);
-      mbar_init(&bars->pd_empty[i], 1);
+      mbar_init(&bars->pd_empty[i], nis);
     }
-    mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->acc_full, nis);
+    mbar_init(&bars->mma_done[0], 1);
+    mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -732,8 +756,11 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
       mbar_wait(&bars->kv_full, 0);
       for (int i = max(0, c - 2); i < c; ++i) mbar_wait(&bars->qd_full[i & 1], (i >> 1) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (kBwdSplit && warp == kKVIssuerB)) {
+    // ------------------------------------------------------------ MMA issuer(s)
+    // warp 1: S and dV^T; warp kKVIssuerB: dP and dK^T (without the split
+    // warp 1 issues all four)
+    const bool do_a = (warp == 1), do_b = !kBwdSplit || warp == kKVIssuerB;
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t idG = idesc_bf16_f32(128, 64, 1, 1);
@@ -747,17 +774,21 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
         tc_fence_after();
         const uint32_t q_base = smem_u32(sQ + pb * C::kRows), do_base = smem_u32(sdO + pb * C::kRows);
         const uint32_t p_base = smem_u32(sP + pb * C::kPB), ds_base = smem_u32(sdS + pb * C::kPB);
+        if (do_a) {
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t ad = make_sdesc(do_base + kk * 2048, lboR, 1024, kLayoutSW128);
-          const uint64_t bp = make_sdesc(p_base + kk * 2048, 1024, 128, kLayoutNone);
-          umma_bf16(tmem + 256, ad, bp, idG, (cc > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t ad = make_sdesc(do_base + kk * 2048, lboR, 1024, kLayoutSW128);
+            const uint64_t bp = make_sdesc(p_base + kk * 2048, 1024, 128, kLayoutNone);
+            umma_bf16(tmem + 256, ad, bp, idG, (cc > 0 || kk > 0) ? 1u : 0u);
+          }
         }
+        if (do_b) {
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t aq = make_sdesc(q_base + kk * 2048, lboR, 1024, kLayoutSW128);
-          const uint64_t bs = make_sdesc(ds_base + kk * 2048, 1024, 128, kLayoutNone);
-          umma_bf16(tmem + 320, aq, bs, idG, (cc > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t aq = make_sdesc(q_base + kk * 2048, lboR, 1024, kLayoutSW128);
+            const uint64_t bs = make_sdesc(ds_base + kk * 2048, 1024, 128, kLayoutNone);
+            umma_bf16(tmem + 320, aq, bs, idG, (cc > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&bars->pd_empty[pb]);
         umma_commit(&bars->qd_empty[pb]);
@@ -772,25 +803,30 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
         }
         tc_fence_after();
         const uint32_t q_base = smem_u32(sQ + qb * C::kRows), do_base = smem_u32(sdO + qb * C::kRows);
+        if (do_a) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t aq = make_sdesc(q_base + (kk >> 2) * C::kRowsChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-          const uint64_t bk = make_sdesc(k_base + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-          umma_bf16(tmem + 64 * sb, aq, bk, idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t aq = make_sdesc(q_base + (kk >> 2) * C::kRowsChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bk = make_sdesc(k_base + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+            umma_bf16(tmem + 64 * sb, aq, bk, idS, kk > 0);
+          }
         }
+        if (do_b) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ao = make_sdesc(do_base + (kk >> 2) * C::kRowsChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-          const uint64_t bv = make_sdesc(v_base + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-          umma_bf16(tmem + 128 + 64 * sb, ao, bv, idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ao = make_sdesc(do_base + (kk >> 2) * C::kRowsChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bv = make_sdesc(v_base + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+            umma_bf16(tmem + 128 + 64 * sb, ao, bv, idS, kk > 0);
+          }
         }
         umma_commit(&bars->s_full[sb]);
         if (cc > 0 && !issue_grad(cc - 1)) { kv_set_abort(bars); ok = false; break; }
       }
       if (ok && !issue_grad(nchunks - 1)) { kv_set_abort(bars); ok = false; }
       umma_commit(&bars->acc_full);
-      umma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0);
+      const int di = do_a ? 0 : 1;
+      umma_commit(&bars->mma_done[di]);
+      mbar_wait(&bars->mma_done[di], 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warps 2..5: row r = (token i, head h)
