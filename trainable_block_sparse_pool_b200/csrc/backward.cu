@@ -264,12 +264,13 @@ __global__ void __launch_bounds__(256) fill_kernel(const Args a) {
 
 // ---------------------------------------------------------------- dQ: per (kv group, token)
 // One thread issues tcgen05.mma at about one product per 100-180 cycles
-// (measured on the B200 for M=128, N=16 chains), so the products of a tile
-// are spread over several issuing threads: with the split, S and dP (dQ
-// kernel) and {S, dV^T} / {dP, dK^T} (dK/dV kernel) go out from two threads.
-// 0 restores one issuer for them.
+// (measured on the B200 for M=128 chains, whatever N), so the products of a
+// tile are spread over several issuing threads: S and dP of the dQ kernel
+// from two threads (1 and 2), and the dK/dV kernel's four products from two
+// threads ({S, dV^T}, {dP, dK^T}: 1) or four (one each: 2).  0 restores one
+// issuer for them.
 #ifndef INFLLM2_BWD_SPLIT
-#define INFLLM2_BWD_SPLIT 1
+#define INFLLM2_BWD_SPLIT 2
 #endif
 constexpr bool kBwdSplit = INFLLM2_BWD_SPLIT != 0;
 // warp 0 K/Q/dO producer, 1 S (and dP) MMA, 2-5 softmax, 6 V producer, 7 dQ MMA, 8 (split) dP MMA
@@ -605,10 +606,18 @@ __global__ void __launch_bounds__(kQThreads, 1) dq_kernel(const __grid_constant_
 }
 
 // ---------------------------------------------------------------- dK / dV: per (kv group, sequence, key block)
-// warp 0 producer, 1 MMA (S, dV^T; without the split all four products), 2-5 softmax / epilogue,
-// 6 (split) MMA for dP and dK^T
-constexpr int kKVThreads = kBwdSplit ? 224 : 192;
+// MMA issuers of the dK/dV kernel and the products each issues (bit 1 S,
+// 2 dP, 4 dV^T, 8 dK^T): one issuer for all four, two ({S, dV^T}, {dP,
+// dK^T}), or, with INFLLM2_BWD_SPLIT=2, one per product.
+constexpr int kKVIssuers = (INFLLM2_BWD_SPLIT >= 2) ? 4 : (kBwdSplit ? 2 : 1);
+__host__ __device__ constexpr uint32_t kv_issuer_mask(int i) {
+  return kKVIssuers == 1 ? 15u : kKVIssuers == 2 ? (i == 0 ? 5u : 10u) : (1u << i);
+}
+// warp 0 producer, 1 the first MMA issuer, 2-5 softmax / epilogue, 6 .. the other issuers
+constexpr int kKVThreads = 192 + 32 * (kKVIssuers - 1);
 constexpr int kKVIssuerB = 6;
+constexpr uint32_t kKVFront = (kKVIssuers == 4) ? 2u : static_cast<uint32_t>(kKVIssuers);   // issuers of S / dP
+constexpr uint32_t kKVBack = kKVFront;                                                       // issuers of dV^T / dK^T
 
 template <int D>
 struct KVCfg {
@@ -626,7 +635,7 @@ struct KVBars {
   uint64_t s_full[2], s_empty[2];
   uint64_t pd_full[2], pd_empty[2];
   uint64_t acc_full;
-  uint64_t mma_done[2];
+  uint64_t mma_done[4];
   uint32_t tmem_base;
   int abort;
 };
@@ -678,18 +687,17 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    const uint32_t nis = kBwdSplit ? 2 : 1;      // one commit per MMA issuer
+    // one commit per MMA issuer that reads the buffer or writes the product
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->qd_full[i], 1);
-      mbar_init(&bars->qd_empty[i], nis);
-      mbar_init(&bars->s_full[i], nis);
+      mbar_init(&bars->qd_empty[i], kKVIssuers);
+      mbar_init(&bars->s_full[i], kKVFront);
       mbar_init(&bars->s_empty[i], 4);
       mbar_init(&bars->pd_full[i], 4);
-      mbar_init(&bars->pd_empty[i], nis);
+      mbar_init(&bars->pd_empty[i], kKVBack);
     }
-    mbar_init(&bars->acc_full, nis);
-    mbar_init(&bars->mma_done[0], 1);
-    mbar_init(&bars->mma_done[1], 1);
+    mbar_init(&bars->acc_full, kKVBack);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->mma_done[i], 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -756,11 +764,16 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
       mbar_wait(&bars->kv_full, 0);
       for (int i = max(0, c - 2); i < c; ++i) mbar_wait(&bars->qd_full[i & 1], (i >> 1) & 1);
     }
-  } else if (warp == 1 || (kBwdSplit && warp == kKVIssuerB)) {
+  } else if (warp == 1 || (warp >= kKVIssuerB && warp < kKVIssuerB + kKVIssuers - 1)) {
     // ------------------------------------------------------------ MMA issuer(s)
-    // warp 1: S and dV^T; warp kKVIssuerB: dP and dK^T (without the split
-    // warp 1 issues all four)
-    const bool do_a = (warp == 1), do_b = !kBwdSplit || warp == kKVIssuerB;
+    // Issuer ir issues the products of kv_issuer_mask(ir).  An issuer of S or
+    // dP ("front") walks the chunks as they land; an issuer of dV^T or dK^T
+    // ("back") as their P and dS are written.  One that does both issues the
+    // gradient products of chunk cc-1 after S / dP of chunk cc.
+    const int ir = (warp == 1) ? 0 : warp - kKVIssuerB + 1;
+    const uint32_t mask = kv_issuer_mask(ir);
+    const bool do_s = mask & 1u, do_dp = mask & 2u, do_dv = mask & 4u, do_dk = mask & 8u;
+    const bool front = do_s || do_dp, back = do_dv || do_dk;
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t idG = idesc_bf16_f32(128, 64, 1, 1);
@@ -774,7 +787,7 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
         tc_fence_after();
         const uint32_t q_base = smem_u32(sQ + pb * C::kRows), do_base = smem_u32(sdO + pb * C::kRows);
         const uint32_t p_base = smem_u32(sP + pb * C::kPB), ds_base = smem_u32(sdS + pb * C::kPB);
-        if (do_a) {
+        if (do_dv) {
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
             const uint64_t ad = make_sdesc(do_base + kk * 2048, lboR, 1024, kLayoutSW128);
@@ -782,7 +795,7 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
             umma_bf16(tmem + 256, ad, bp, idG, (cc > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        if (do_b) {
+        if (do_dk) {
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
             const uint64_t aq = make_sdesc(q_base + kk * 2048, lboR, 1024, kLayoutSW128);
@@ -796,6 +809,10 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
       };
       int cc = 0;
       for (; ok && cc < nchunks; ++cc) {
+        if (!front) {
+          if (!issue_grad(cc)) { kv_set_abort(bars); ok = false; break; }
+          continue;
+        }
         const int qb = cc & 1, sb = cc & 1;
         if (!mbar_wait(&bars->qd_full[qb], (cc >> 1) & 1) ||
             !mbar_wait(&bars->s_empty[sb], ((cc >> 1) & 1) ^ 1) || kv_aborted(bars)) {
@@ -803,7 +820,7 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
         }
         tc_fence_after();
         const uint32_t q_base = smem_u32(sQ + qb * C::kRows), do_base = smem_u32(sdO + qb * C::kRows);
-        if (do_a) {
+        if (do_s) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t aq = make_sdesc(q_base + (kk >> 2) * C::kRowsChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
@@ -811,7 +828,7 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
             umma_bf16(tmem + 64 * sb, aq, bk, idS, kk > 0);
           }
         }
-        if (do_b) {
+        if (do_dp) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t ao = make_sdesc(do_base + (kk >> 2) * C::kRowsChunk + (kk & 3) * 32, 16, 1024, kLayoutSW128);
@@ -820,13 +837,13 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
           }
         }
         umma_commit(&bars->s_full[sb]);
-        if (cc > 0 && !issue_grad(cc - 1)) { kv_set_abort(bars); ok = false; break; }
+        if (!back) umma_commit(&bars->qd_empty[qb]);     // this issuer's last read of the chunk
+        if (back && cc > 0 && !issue_grad(cc - 1)) { kv_set_abort(bars); ok = false; break; }
       }
-      if (ok && !issue_grad(nchunks - 1)) { kv_set_abort(bars); ok = false; }
-      umma_commit(&bars->acc_full);
-      const int di = do_a ? 0 : 1;
-      umma_commit(&bars->mma_done[di]);
-      mbar_wait(&bars->mma_done[di], 0);
+      if (ok && front && back && !issue_grad(nchunks - 1)) { kv_set_abort(bars); ok = false; }
+      if (back) umma_commit(&bars->acc_full);
+      umma_commit(&bars->mma_done[ir]);
+      mbar_wait(&bars->mma_done[ir], 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warps 2..5: row r = (token i, head h)
