@@ -11,7 +11,8 @@ extra flush is needed between steps.
 
 Output: one JSON line (rank 0).  `value` is tokens/s over all ranks;
 `e2e` repeats the measurement through the public API with the inputs copied
-from pinned host memory and the output copied back inside the timed region;
+from pinned host memory and the output copied back inside the timed region
+(pipelined over two buffer sets; the serial figure rides along);
 `roofline` describes the dominant kernel; `step_roofline` the whole step
 against the sum of its steps' bounds; `decode` the 16 x 131072 decode step
 (µs/step, fraction of HBM); `varlen` the packed 131072-token dense/sparse
@@ -717,21 +718,22 @@ def main():
 
     kernels = ["compress", "scores", "topk", "sparse"]
 
-    def step(ev=None):
+    def step(ev=None, bufs=None):
+        q, k, v, o = bufs if bufs is not None else (Q, K, V, out)
         if ev is not None: ev[0].record(stream)
-        T.infllm2_compress_k(K, vl, Kc1, Kc2, p, stream)
+        T.infllm2_compress_k(k, vl, Kc1, Kc2, p, stream)
         if ev is not None: ev[1].record(stream)
         if fused:
-            T.infllm2_pooled_scores(Q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
+            T.infllm2_pooled_scores(q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
         else:
-            T.infllm2_shared_scores(Q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
+            T.infllm2_shared_scores(q, Kc1, Kc2, vl, w.h_kv, S, ld, p, stream)
         if ev is not None: ev[2].record(stream)
         if fused:
             T.infllm2_topk_blocks_pooled(S, ld, vl, w.h_kv, idx, p, stream)
         else:
             T.infllm2_topk_blocks(S, ld, vl, w.h_kv, idx, p, stream)
         if ev is not None: ev[3].record(stream)
-        T.infllm2_sparse_attn(Q, K, V, idx, vl, out, p, stream, workspace=sws)
+        T.infllm2_sparse_attn(q, k, v, idx, vl, o, p, stream, workspace=sws)
         if ev is not None: ev[4].record(stream)
 
     for _ in range(args.warmup):
@@ -784,11 +786,57 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+        serial_ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
         h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
         d2h = outh.numel() * outh.element_size()
+
+        # Pipelined: two sets of device inputs and outputs, the uploads on one
+        # stream and the downloads on another, so the copies of steps k+1 and
+        # k-1 run under the kernels of step k.  Every step still copies its own
+        # Q, K, V in from pinned host memory and its output back, inside the
+        # timed region.
+        sets = [(Q, K, V, out), (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(out))]
+        outs_h = [outh, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def run_pipelined(n):
+            for kk in range(n):
+                bsel = kk & 1
+                q, k, v, o = sets[bsel]
+                if kk >= 2:
+                    up.wait_event(ev_done[bsel])       # step kk-2 has finished reading this set
+                with torch.cuda.stream(up):
+                    q.copy_(Qh, non_blocking=True); k.copy_(Kh, non_blocking=True); v.copy_(Vh, non_blocking=True)
+                    ev_in[bsel].record(up)
+                stream.wait_event(ev_in[bsel])
+                if kk >= 2:
+                    stream.wait_event(ev_out[bsel])    # step kk-2's output has been read back
+                step(bufs=sets[bsel])
+                ev_done[bsel].record(stream)
+                down.wait_event(ev_done[bsel])
+                with torch.cuda.stream(down):
+                    outs_h[bsel].copy_(o, non_blocking=True)
+                    ev_out[bsel].record(down)
+            for e in ev_out:
+                stream.wait_event(e)
+
+        run_pipelined(4)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        up.wait_event(a); down.wait_event(a)
+        run_pipelined(args.steps)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "pipelined": "two buffer sets; uploads and downloads on their own streams overlap the kernels of "
+                            "the neighbouring steps",
+               "serial": {"value": tokens / (serial_ms / 1e3), "unit": "tokens/s", "ms_per_step": serial_ms}}
 
     # ---- L2 -> SM gather bandwidth with the attention's tile shape (this run)
     l2 = measure_l2_gather(T, torch, K, V, stream)
