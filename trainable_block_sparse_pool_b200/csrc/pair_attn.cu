@@ -36,6 +36,14 @@ constexpr int kKeys = 128;
 #ifndef INFLLM2_PAIR_PIPE
 #define INFLLM2_PAIR_PIPE 0
 #endif
+// LOCAL with bf16 output: the row's top-k partial (d bf16) and its
+// log-sum-exp are loaded before the wait for the last P.V, in one batch,
+// instead of chunk by chunk between the TMEM reads of the epilogue (each
+// TMEM read orders the loads around it, so they went out one round trip
+// at a time).
+#ifndef INFLLM2_PAIR_PREFETCH
+#define INFLLM2_PAIR_PREFETCH 1
+#endif
 constexpr int kKStages = INFLLM2_PAIR_KSTAGES;
 constexpr int kVStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -346,6 +354,16 @@ __global__ void __launch_bounds__(kThreads, 1) pair_attn_kernel(
     }
     // ---- the row's output: O / l, merged with the top-k partial (LOCAL).
     // TMEM is read by whole warps; only rows of the sequence are written.
+    constexpr bool kPre = LOCAL && !OUT_F32 && INFLLM2_PAIR_PREFETCH;
+    uint4 topv[kPre ? D / 8 : 1];
+    float lb_pre = -INFINITY;
+    if (kPre && t < len) {
+      const int64_t rh = static_cast<int64_t>(row0 + t) * h_q + static_cast<int64_t>(g) * G + h;
+      lb_pre = lse[rh];
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(out) + rh * D);
+#pragma unroll
+      for (int q = 0; q < (kPre ? D / 8 : 1); ++q) topv[q] = src[q];
+    }
     const bool got = __all_sync(0xffffffffu, ok && (nkt == 0 || mbar_wait(&bars->pv_done[w], (nkt - 1) & 1)));
     tc_fence_after();
     if (!got) {
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_attn_kernel(
       float w_own = inv, w_top = 0.f;
       if (LOCAL && row_ok) {
         // lse[rh] holds the top-k partial's log-sum-exp (log2 units; -inf: none)
-        const float lb = lse[rh];
+        const float lb = kPre ? lb_pre : lse[rh];
         const float la = (l_run > 0.f) ? m_ref + log2f(l_run) : -INFINITY;
         float lse_row = la;
         if (lb != -INFINITY && l_run > 0.f) {
@@ -395,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_attn_kernel(
 #pragma unroll
             for (int e = 0; e < 8; ++e) top[e] = 0.f;
             if (LOCAL && w_top != 0.f) {
-              const uint4 b4 = o4[q];
+              const uint4 b4 = kPre ? topv[(cc >> 3) + q] : o4[q];
               const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b4);
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
