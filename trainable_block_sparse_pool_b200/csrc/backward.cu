@@ -273,6 +273,13 @@ __global__ void __launch_bounds__(256) fill_kernel(const Args a) {
 #define INFLLM2_BWD_SPLIT 2
 #endif
 constexpr bool kBwdSplit = INFLLM2_BWD_SPLIT != 0;
+// The dK/dV kernel's row threads fetch their rows' token ids two chunks
+// ahead and the rows' log-sum-exp and Dsum one chunk ahead, so the two
+// dependent global loads of a chunk are in flight during the chunk before
+// instead of opening it.
+#ifndef INFLLM2_BWD_ROWS_AHEAD
+#define INFLLM2_BWD_ROWS_AHEAD 1
+#endif
 // warp 0 K/Q/dO producer, 1 S (and dP) MMA, 2-5 softmax, 6 V producer, 7 dQ MMA, 8 (split) dP MMA
 constexpr int kQThreads = kBwdSplit ? 288 : 256;
 constexpr int kQVWarp = 6;
@@ -853,14 +860,36 @@ __global__ void __launch_bounds__(kKVThreads, 1) dkdv_kernel(const __grid_consta
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const float c = a.scale * kLog2e;
     bool stop = false;
+    auto row_of = [&](int c2) { const int i2 = c2 * TQ + qi; return (c2 < nchunks && i2 < count) ? __ldg(rows + i2) : -1; };
+    auto stat_of = [&](const float* v, int t2) {
+      return (t2 >= 0) ? __ldg(v + static_cast<int64_t>(row0 + t2) * a.h_q + static_cast<int64_t>(g) * G + h) : 0.f;
+    };
+    int t_a = 0, t_b = 0;
+    float lse_a = 0.f, ds_a = 0.f;
+    if (INFLLM2_BWD_ROWS_AHEAD) {
+      t_a = row_of(0);
+      t_b = row_of(1);
+      lse_a = stat_of(a.lse, t_a);
+      ds_a = stat_of(a.dsum, t_a);
+    }
     for (int cc = 0; cc < nchunks; ++cc) {
       const int sb = cc & 1;
       const int i = cc * TQ + qi;
       const bool rv = i < count;
-      const int t = rv ? __ldg(rows + i) : -1;
-      const int64_t rh = static_cast<int64_t>(row0 + max(t, 0)) * a.h_q + static_cast<int64_t>(g) * G + h;
-      const float lse = rv ? __ldg(a.lse + rh) : 0.f;
-      const float dsum = rv ? __ldg(a.dsum + rh) : 0.f;
+      int t;
+      float lse, dsum;
+      if (INFLLM2_BWD_ROWS_AHEAD) {
+        t = t_a; lse = lse_a; dsum = ds_a;
+        lse_a = stat_of(a.lse, t_b);           // chunk cc + 1
+        ds_a = stat_of(a.dsum, t_b);
+        t_a = t_b;
+        t_b = row_of(cc + 2);                   // chunk cc + 2
+      } else {
+        t = rv ? __ldg(rows + i) : -1;
+        const int64_t rh = static_cast<int64_t>(row0 + max(t, 0)) * a.h_q + static_cast<int64_t>(g) * G + h;
+        lse = rv ? __ldg(a.lse + rh) : 0.f;
+        dsum = rv ? __ldg(a.dsum + rh) : 0.f;
+      }
       bool ab = !mbar_wait(&bars->s_full[sb], (cc >> 1) & 1);
       tc_fence_after();
       float sv[64], pv[64];
