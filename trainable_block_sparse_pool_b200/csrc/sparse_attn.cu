@@ -599,16 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
         xn = get_unit(blockIdx.x + (k + kNumWG) * gridDim.x, args);
         Ln = load_warp_list(xn.I, xn.nvalid, half, lane);
       }
-      // ---- unit done: wait for its last PV, reduce the row sums, write out
-      bool ab = (nt > 0) && !mbar_wait(&bars->pv_done[w][(tcnt - 1) & 1], ((tcnt - 1) >> 1) & 1);
-      if (ab) set_abort(bars);
-      tc_fence_after();
-      float o[16];
-      tmem_load16(t_o + lane_addr + obuf * 16, o);
-      if (nt == 0) {                         // empty list: no PV wrote this buffer
-#pragma unroll
-        for (int h = 0; h < 16; ++h) o[h] = 0.f;
-      }
+      // ---- unit done: reduce the row sums (they do not depend on O, so this
+      // runs while the last PV completes), wait for that PV, write out
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
 #pragma unroll
@@ -619,6 +611,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(
 #pragma unroll
         for (int h = 1; h < 16; ++h) if (lane == h) mine = l_part[h];
         red_w[wq * 16 + lane] = mine;
+      }
+      bool ab = (nt > 0) && !mbar_wait(&bars->pv_done[w][(tcnt - 1) & 1], ((tcnt - 1) >> 1) & 1);
+      if (ab) set_abort(bars);
+      tc_fence_after();
+      float o[16];
+      tmem_load16(t_o + lane_addr + obuf * 16, o);
+      if (nt == 0) {                         // empty list: no PV wrote this buffer
+#pragma unroll
+        for (int h = 0; h < 16; ++h) o[h] = 0.f;
       }
       ab = ab || aborted(bars);
       if (bar_red_or(bar_id, 128, ab)) { stop = true; break; }
